@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark: affine Q4 group-32 GEMV over the full temporal weight stream at M = 1.
+
+One step = one pass of the 32-layer temporal transformer's weight stream plus
+the text head (7 * 32 + 1 = 225 q4_matmul calls, 4,192,337,920 packed bytes),
+activations x [1, 4096] (and [1, 11264] for the down projections) reused per
+layer.  Metric: effective GB/s of packed bytes (and ms per stream).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line on rank 0.  Multi-GPU (torchrun) runs independent
+replicas, one stream per GPU ("weak" scaling); the only collectives are the
+barrier and the max over ranks of the timed region.  --impl reference times
+the CPU oracle (test infrastructure) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Q4-g32 GEMV packed-HBM GB/s & ms per 32-layer temporal weight stream (M=1)"
+STREAM_BYTES = 4_192_337_920
+WORKLOAD = ("temporal_stream: 32 layers x (q,k,v,o 4096x4096; gate,up 11264x4096; down 4096x11264) "
+            "+ text head 32000x4096, Q4 g32, x [1,4096] / [1,11264] bf16, M=1")
+
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# --------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", self.gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_median": statistics.median(r["power"] for r in rows)}
+
+
+def _gpu_id_for(device_index: int) -> str:
+    import torch
+
+    try:
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[device_index]
+        return str(device_index)
+
+
+# --------------------------------------------------------------------- workload
+
+
+def build_stream(device):
+    """Draw and quantize the 225 projections of the stream on the GPU."""
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("temporal_stream")
+    packed = []
+    for t, p in enumerate(workloads.stream_projs()):
+        W = workloads.weight(p.N, p.K, seed, t, device=device)
+        c, s, b = q4.q4_quantize(W)
+        del W
+        packed.append((p, c, s, b))
+    torch.cuda.synchronize(device)
+    x = workloads.activation(1, 4096, seed, 10000).to(device)
+    x_down = workloads.activation(1, 11264, seed, 10001).to(device)
+    return packed, x, x_down
+
+
+def stream_bytes(packed) -> int:
+    return sum(c.numel() + 2 * s.numel() + 2 * b.numel() for _, c, s, b in packed)
+
+
+def enqueue_stream(packed, x, x_down, ys):
+    import weight_only_bit_affine_b200 as q4
+
+    for (p, c, s, b), y in zip(packed, ys):
+        q4.q4_matmul(x_down if p.K == 11264 else x, c, s, b, out=y)
+
+
+def _kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_only_bit_affine_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_per_launch(kernel_hash: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = d.get("gemv_m1_stream")
+    if not ent or ent.get("kernel_source_hash") != kernel_hash:
+        return None
+    return ent.get("dram_bytes_per_launch_avg")
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------- CPU oracle
+
+
+class OracleSample:
+    """A bounded sample of the stream for timing the CPU oracle.
+
+    The first projections of the stream are drawn on the CPU with the same
+    seeds and quantized by the oracle (untimed); `time()` runs the oracle's
+    dequantize-and-matmul over them and returns GB/s of packed bytes.  The
+    sample grows one projection at a time until one pass costs about
+    `budget_s` seconds.
+    """
+
+    def __init__(self, budget_s: float):
+        import oracle
+        import workloads
+
+        seed = workloads.seed_of("temporal_stream")
+        self.x = workloads.bf16_bits(workloads.activation(1, 4096, seed, 10000))
+        self.x_down = workloads.bf16_bits(workloads.activation(1, 11264, seed, 10001))
+        self.items, spent = [], 0.0
+        for t, p in enumerate(workloads.stream_projs()):
+            if spent >= budget_s:
+                break
+            W = workloads.bf16_bits(workloads.weight(p.N, p.K, seed, t))
+            c, s, b = oracle.quantize(W)
+            del W
+            self.items.append((p, c, s, b))
+            spent += self._run_one(self.items[-1])
+        self.nbytes = sum(c.size + 2 * s.size + 2 * b.size for _, c, s, b in self.items)
+        self.threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+        names = [p.name for p, _, _, _ in self.items]
+        self.desc = (f"oracle dequantize+matmul (C, binary64, OpenMP, {self.threads} threads) on the first "
+                     f"{len(names)} of 225 stream projections ({names[0]}..{names[-1]}, {self.nbytes} packed bytes)")
+
+    def _run_one(self, item):
+        import oracle
+
+        p, c, s, b = item
+        t0 = time.perf_counter()
+        oracle.matmul_ref(self.x_down if p.K == 11264 else self.x, c, s, b)
+        return time.perf_counter() - t0
+
+    def time(self):
+        spent = sum(self._run_one(it) for it in self.items)
+        return self.nbytes / spent / 1e9, spent
+
+
+# --------------------------------------------------------------------- arms
+
+
+def run_reference(args):
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    # one untimed sample sizes the steps so the whole run stays within minutes
+    sample = OracleSample(float(os.environ.get("Q4_REF_STEP_SECONDS", "2.0")))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        gbs, spent = sample.time()
+        if i >= args.warmup:
+            vals.append(spent)
+    gbs = sample.nbytes * len(vals) / sum(vals) / 1e9
+    desc, threads = sample.desc, sample.threads
+    ms_per_step = STREAM_BYTES / (gbs * 1e9) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "bytes_per_stream": STREAM_BYTES,
+                   "note": "each step times a bounded sample of the stream; ms_per_step extrapolates to the whole stream"},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import weight_only_bit_affine_b200 as q4
+    from weight_only_bit_affine_b200 import build as q4build
+
+    world, rank, local = _dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (libq4 has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        q4build.build()
+    if world > 1:
+        dist.barrier()
+
+    def barrier_sync():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    packed, x, x_down = build_stream(dev)
+    nbytes = stream_bytes(packed)
+    assert nbytes == STREAM_BYTES, nbytes
+    # all outputs are views of one buffer, so a step's result reads back in one copy
+    y_all = torch.empty(sum(p.N for p, _, _, _ in packed), dtype=torch.bfloat16, device=dev)
+    ys, off = [], 0
+    for p, _, _, _ in packed:
+        ys.append(y_all[off:off + p.N].view(1, p.N))
+        off += p.N
+
+    # Capture the 225 launches once in a CUDA graph (launched with programmatic
+    # dependent launch, so consecutive matmuls overlap their prologues).
+    enqueue_stream(packed, x, x_down, ys)  # warm up: sets kernel attributes
+    torch.cuda.synchronize(dev)
+    n0 = q4.q4_debug_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            enqueue_stream(packed, x, x_down, ys)
+    launches_per_step = q4.q4_debug_launch_count() - n0
+    torch.cuda.synchronize(dev)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        graph.replay()
+    barrier_sync()
+    sampler = ClockSampler(_gpu_id_for(local))
+    sampler.start()
+    time.sleep(0.3)
+    barrier_sync()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(stream)
+    barrier_sync()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+
+    # plain stream launches (no graph), same work
+    for _ in range(3):
+        enqueue_stream(packed, x, x_down, ys)
+    torch.cuda.synchronize(dev)
+    plain_steps = max(3, min(args.steps, 50))
+    ev0.record(stream)
+    for _ in range(plain_steps):
+        enqueue_stream(packed, x, x_down, ys)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_plain = ev0.elapsed_time(ev1) / plain_steps
+
+    # per-launch durations of the GEMV kernel (events around each launch)
+    per = [[] for _ in packed]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in packed]
+    for _ in range(3):
+        for i, ((p, c, s, b), y) in enumerate(zip(packed, ys)):
+            evs[i][0].record(stream)
+            q4.q4_matmul(x_down if p.K == 11264 else x, c, s, b, out=y)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        for i, (a, e) in enumerate(evs):
+            per[i].append(a.elapsed_time(e))
+    launch_ms = [statistics.median(v) for v in per]
+    kernel_gbs = nbytes / (sum(launch_ms) * 1e-3) / 1e9
+    by_shape = {}
+    for (p, c, s, b), t in zip(packed, launch_ms):
+        key = f"{p.N}x{p.K}"
+        nb = c.numel() + 2 * s.numel() + 2 * b.numel()
+        e = by_shape.setdefault(key, [0, 0.0, 0])
+        e[0] += nb
+        e[1] += t
+        e[2] += 1
+    shapes = {k: {"launches": v[2], "us_per_launch": round(v[1] / v[2] * 1e3, 2),
+                  "GBps": round(v[0] / (v[1] * 1e-3) / 1e9, 1)} for k, v in by_shape.items()}
+
+    # end to end through the public API: pinned x H2D, the step, y D2H
+    x_host = x.cpu().pin_memory()
+    xd_host = x_down.cpu().pin_memory()
+    y_host = torch.empty(y_all.numel(), dtype=torch.bfloat16).pin_memory()
+    h2d = (x_host.numel() + xd_host.numel()) * 2
+    d2h = y_all.numel() * 2
+    e2e_steps = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        x_down.copy_(xd_host, non_blocking=True)
+        graph.replay()
+        y_host.copy_(y_all, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = max(ev0.elapsed_time(ev1), (time.perf_counter() - t_wall0) * 1e3) / e2e_steps
+
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+
+    flags = q4.q4_debug_device_flags()
+    peak, peak_kind = _peaks()
+    kh = _kernel_source_hash()
+    traffic = _traffic_per_launch(kh)
+    line = {
+        "metric": METRIC,
+        "value": round(world * nbytes / (ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD,
+            "bytes_per_stream": nbytes,
+            "launches_per_step": int(launches_per_step),
+            "mode": "CUDA graph replay of 225 q4_matmul launches (programmatic dependent launch)",
+            "l2": "inputs larger than L2: 4.19 GB streamed per step vs 126 MB L2",
+            "weights": "u4 codes + bf16 scale/bias per 32 (5 bits/weight), fp32 accumulation",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(kernel_gbs, 1),
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": round(kernel_gbs / peak, 4),
+            "traffic": traffic,
+            "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback",
+            "kernel": "gemv_tma_kernel (M=1), 225 launches per step; per-launch CUDA events",
+        },
+        "e2e": {"value": round(world * nbytes / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "pinned x H2D + graph replay of the 225 public q4_matmul calls + y D2H, per step"},
+        "gpu_launches": int(launches_per_step) * args.steps,
+        "clocks": clocks,
+        "rows": {
+            "stream_ms_graph": round(ms, 4),
+            "stream_ms_plain_launches": round(ms_plain, 4),
+            "stream_GBps_plain_launches": round(nbytes / (ms_plain * 1e-3) / 1e9, 1),
+            "per_shape_isolated_launch": shapes,
+        },
+        "device_flags": flags,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(float(os.environ.get("Q4_CPU_BASELINE_SECONDS", "10")))
+        gbs, spent = sample.time()
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": sample.threads, "kind": "oracle",
+                                "sample": sample.desc, "seconds": round(spent, 2)}
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

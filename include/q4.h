@@ -1,0 +1,151 @@
+/*
+ * q4.h -- C ABI of libq4: affine 4-bit, group-32, weight-only quantized
+ * matmul on NVIDIA B200 (sm_100a).
+ *
+ * Format (model card "personaplex-edge-q4", section "Release details":
+ * "affine Q4, group size 32, BF16 activations"; the packed size it prints,
+ * 4.87 GiB for 8,371,408,896 parameters, is 5 bits per weight):
+ *
+ *   W        [N, K]      bf16, row-major: N outputs ("out"), K inputs ("in").
+ *   codes    [N, K/2]    uint8: byte k/2 of row n holds q[n,k] in bits 0..3
+ *                        when k is even and q[n,k+1] in bits 4..7.  Each
+ *                        16-byte run is one group of 32 codes.
+ *   scales   [N, K/32]   bf16, one per group of 32 consecutive k of a row.
+ *   biases   [N, K/32]   bf16, likewise.
+ *   w_hat[n,k] = scales[n,k/32] * q[n,k] + biases[n,k/32],  q in 0..15.
+ *
+ * The matmul multiplies by the transposed weight, y = x . w_hat^T, as the
+ * Swift/MLX blog "NVIDIA PersonaPlex 7B on Apple Silicon" (section
+ * "Depformer: per-step weight switching") calls quantizedMM with
+ * transpose: true, groupSize and bits.
+ *
+ * Conventions for every entry point:
+ *  - All pointers are DEVICE pointers, allocated and owned by the caller.
+ *    The library allocates no device memory and keeps no pointer after a
+ *    call returns.  bf16 values are passed as their 16-bit patterns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and never synchronize the host or copy between host
+ *    and device.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    non-OK status means nothing was enqueued.  q4_last_error() returns a
+ *    message for the last non-OK status of the calling thread.
+ *  - Alignment: W, W_out, codes and x must be 16-byte aligned; scales,
+ *    biases and y 2-byte aligned.  Row strides are implied by K (dense).
+ *  - Sizes: 0 <= M, N; 32 <= K, K % 32 == 0.  M == 0 or N == 0 is a no-op.
+ *    `group` must be 32.  K <= 2^24, N <= 2^40, M <= 2^31.
+ *  - Output buffers must not overlap inputs.
+ *  - Device: compute capability 10.0 (B200, sm_100a) only; any other device
+ *    returns Q4_ERR_UNSUPPORTED.
+ */
+#ifndef Q4_H_
+#define Q4_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define Q4_API __attribute__((visibility("default")))
+#else
+#define Q4_API
+#endif
+
+typedef uint16_t q4_bf16;                 /* bf16 bit pattern */
+typedef struct CUstream_st* q4_stream_t;  /* same type as cudaStream_t */
+
+typedef enum {
+  Q4_OK = 0,
+  Q4_ERR_NULL = 1,         /* a required pointer is NULL                      */
+  Q4_ERR_SHAPE = 2,        /* negative size, K not a positive multiple of 32  */
+  Q4_ERR_ALIGN = 3,        /* pointer misaligned for its role                 */
+  Q4_ERR_UNSUPPORTED = 4,  /* group != 32, K too large, or not an sm_100 GPU  */
+  Q4_ERR_RANGE = 5,        /* step outside [0, num_steps)                     */
+  Q4_ERR_CUDA = 6          /* a CUDA runtime call or a launch failed          */
+} q4_status;
+
+/*
+ * q4_quantize -- per row n and group g of 32 consecutive k:
+ *   mn, mx = min, max of the group;
+ *   scale  = bf16(fp32(mx - mn) / 15)   (IEEE fp32 subtraction and division,
+ *                                        round to nearest even, then RNE to bf16)
+ *   bias   = bf16(mn)                   (exact)
+ *   q      = 0 if scale == 0, else clamp(round_half_even((w - bias)/scale), 0, 15),
+ *            the quotient taken in IEEE binary64.
+ * The pages name the method (model card "personaplex-edge-q4", opening
+ * paragraph and "Release details"; GeekNews summary of the Swift port,
+ * "Arsitektur model dan konversi": 4-bit quantization in the conversion
+ * script) but not its arithmetic; this is the plainest reading of "affine,
+ * 4-bit, group 32".  Offline: not on the matmul path.
+ * In:  W [N, K] bf16.   Out: codes [N, K/2], scales [N, K/32], biases [N, K/32].
+ * Non-finite weights give unspecified codes (not checked on the device).
+ */
+Q4_API q4_status q4_quantize(const q4_bf16* W, int64_t N, int64_t K, int group,
+                      uint8_t* codes, q4_bf16* scales, q4_bf16* biases,
+                      q4_stream_t stream);
+
+/*
+ * q4_dequantize -- W_out[n,k] = bf16_rne(scale * q + bias), the product and
+ * sum taken in IEEE binary64 (exact for every non-degenerate group).  The
+ * model card "personaplex-edge-q4" (section "Conversion and weight
+ * validation") reconstructs every packed tensor this way to validate it.
+ * In: codes [N, K/2], scales, biases [N, K/32].  Out: W_out [N, K] bf16.
+ */
+Q4_API q4_status q4_dequantize(const uint8_t* codes, const q4_bf16* scales,
+                        const q4_bf16* biases, int64_t N, int64_t K, int group,
+                        q4_bf16* W_out, q4_stream_t stream);
+
+/*
+ * q4_matmul -- y[m,n] = sum_k x[m,k] * w_hat[n,k], accumulated in fp32 and
+ * rounded to bf16 (nearest even), with the weights read in packed form and
+ * never expanded to bf16 in memory (model card "personaplex-edge-q4",
+ * opening paragraph: the packed weights run through a quantized matmul and
+ * are not expanded back to BF16).
+ * In:  x [M, K] bf16 (row-major), codes [N, K/2], scales, biases [N, K/32].
+ * Out: y [M, N] bf16 (row-major).
+ * M < 16 runs the CUDA-core GEMV family; M >= 16 the tensor-core path.
+ * Launch-order contract: the kernels may be launched with programmatic
+ * dependent launch; they read nothing written by an earlier kernel in the
+ * stream before that kernel has completed.
+ */
+Q4_API q4_status q4_matmul(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes,
+                    const q4_bf16* scales, const q4_bf16* biases, int64_t N,
+                    int group, q4_bf16* y, q4_stream_t stream);
+
+/*
+ * q4_matmul_step -- the per-step weight slice of a stacked tensor (Swift/MLX
+ * blog, section "Depformer: per-step weight switching": one weight tensor of
+ * [num_steps * N, K] with scales and biases stacked the same way; step s
+ * uses rows [s*N, (s+1)*N) of all three).  Equivalent to q4_matmul on
+ * codes + s*N*K/2, scales + s*N*K/32, biases + s*N*K/32.
+ * Returns Q4_ERR_RANGE unless 0 <= step < num_steps.
+ */
+Q4_API q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K,
+                         const uint8_t* codes, const q4_bf16* scales,
+                         const q4_bf16* biases, int64_t N, int64_t num_steps,
+                         int64_t step, int group, q4_bf16* y, q4_stream_t stream);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+Q4_API const char* q4_last_error(void);
+
+/*
+ * Diagnostic, not part of the compute path: bit 0 is set on the current
+ * device if any libq4 kernel gave up a bounded internal wait (a pipeline
+ * stage that never arrived within one second; the kernel then finishes
+ * without waiting and its output is invalid).  Synchronizes with the device
+ * (it copies the flag to the host).  clear != 0 resets the flags.  Returns
+ * the flags, or -1 if the copy failed.
+ */
+Q4_API int q4_debug_device_flags(int clear);
+
+/* Diagnostic: number of kernel launches libq4 has enqueued in this process
+ * (counted on the host when each launch is issued; graph replays of captured
+ * launches are not counted again). */
+Q4_API unsigned long long q4_debug_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_H_ */

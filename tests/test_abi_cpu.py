@@ -1,0 +1,119 @@
+"""The C-ABI library builds, loads, exports every entry point include/*.h
+declares, and validates arguments on the host.  No GPU needed: every call
+here returns before any device work (validation precedes the device query;
+on a machine without a GPU, a fully valid call stops at the device query with
+Q4_ERR_CUDA)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+import weight_only_bit_affine_b200 as q4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, NULL, SHAPE, ALIGN, UNSUP, RANGE, CUDA = range(7)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from weight_only_bit_affine_b200 import build
+
+    build.build()
+    return q4.lib()
+
+
+def declared_symbols():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(q4_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ["q4_quantize", "q4_dequantize", "q4_matmul", "q4_matmul_step", "q4_last_error"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(declared_symbols()) <= set(q4.SIGNATURES)
+    out = subprocess.run(["nm", "-D", "--defined-only", q4.library_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (q4_\w+)", out))
+    assert set(declared_symbols()) <= exported
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "q4.h"\nint main(void){ q4_status s = Q4_OK; (void)s; return 0; }\n')
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           "-c", str(src), "-o", str(tmp_path / "t.o")])
+
+
+P = 0x100000  # a fake, 16-byte aligned "device pointer": never dereferenced by validation
+
+
+def _mm(lib, x=P, M=1, K=64, codes=P, s=P, b=P, N=8, group=32, y=P):
+    return lib.q4_matmul(x, M, K, codes, s, b, N, group, y, None)
+
+
+def test_matmul_validation(lib):
+    assert _mm(lib, group=64) == UNSUP
+    assert b"group" in lib.q4_last_error()
+    assert _mm(lib, K=48) == SHAPE
+    assert _mm(lib, K=0) == SHAPE
+    assert _mm(lib, M=-1) == SHAPE
+    assert _mm(lib, N=-3) == SHAPE
+    assert _mm(lib, M=0) == OK  # empty: nothing to do
+    assert _mm(lib, N=0) == OK
+    assert _mm(lib, x=None) == NULL
+    assert _mm(lib, y=None) == NULL
+    assert _mm(lib, x=P + 8) == ALIGN
+    assert _mm(lib, codes=P + 4) == ALIGN
+    assert _mm(lib, s=P + 1) == ALIGN
+    assert _mm(lib, y=P + 1) == ALIGN
+
+
+def test_step_validation(lib):
+    st = lambda steps, step, **kw: lib.q4_matmul_step(P, 1, 64, P, P, P, 8, steps, step, kw.get("group", 32), P, None)
+    assert st(16, 16) == RANGE
+    assert st(16, -1) == RANGE
+    assert st(0, 0) == RANGE
+    assert b"step" in lib.q4_last_error()
+    assert st(16, 3, group=16) == UNSUP
+
+
+def test_quantize_dequantize_validation(lib):
+    assert lib.q4_quantize(P, 4, 64, 32, P + 8, P, P, None) == ALIGN
+    assert lib.q4_quantize(P, 4, 40, 32, P, P, P, None) == SHAPE
+    assert lib.q4_quantize(None, 4, 64, 32, P, P, P, None) == NULL
+    assert lib.q4_quantize(P, 0, 64, 32, P, P, P, None) == OK
+    assert lib.q4_dequantize(P, P, P, 4, 64, 8, P, None) == UNSUP
+    assert lib.q4_dequantize(P, P, P, -1, 64, 32, P, None) == SHAPE
+    assert lib.q4_dequantize(P, P + 1, P, 4, 64, 32, P, None) == ALIGN
+
+
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _mm(lib) == CUDA
+    assert lib.q4_last_error() != b""
+
+
+def test_python_binding_raises_on_status(lib):
+    import torch
+
+    x = torch.zeros((1, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):  # CPU tensors are refused before the ABI
+        q4.q4_matmul(x, torch.zeros((4, 32), dtype=torch.uint8), torch.zeros((4, 2), dtype=torch.bfloat16),
+                     torch.zeros((4, 2), dtype=torch.bfloat16))
+    err = q4.Q4Error(RANGE, "x")
+    assert err.status_name == "Q4_ERR_RANGE"

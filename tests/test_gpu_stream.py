@@ -1,0 +1,64 @@
+"""Full-size temporal weight stream at M = 1 (32 layers x 7 projections + text
+head, 4,192,337,920 packed bytes), in the launch configuration the benchmark
+times: one q4_matmul per projection on one stream, x reused per layer.
+
+The weights are drawn and quantized on the GPU (a host draw of 6.7e9 values is
+too slow); the codes of layers 0 and 31 and of the head are compared bit for
+bit with the oracle's quantization of the same bf16 weights copied to the
+host, and sampled output rows of every projection are compared with the oracle
+within the matmul bound.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+import weight_only_bit_affine_b200 as q4
+from helpers import assert_quantize_bitexact, check_matmul, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def stream():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    seed = workloads.seed_of("temporal_stream")
+    projs = workloads.stream_projs()
+    packed = []
+    last_layer = workloads.TEMPORAL_LAYERS - 1
+    for t, p in enumerate(projs):
+        W = workloads.weight(p.N, p.K, seed, t, device="cuda")
+        c, s, b = q4.q4_quantize(W)
+        if p.name.startswith("L0.") or p.name.startswith(f"L{last_layer}.") or p.name == "head":
+            torch.cuda.synchronize()
+            assert_quantize_bitexact(W, c, s, b)
+        del W
+        packed.append((p, c, s, b))
+    x = workloads.activation(1, 4096, seed, 10000).cuda()
+    x_down = workloads.activation(1, 11264, seed, 10001).cuda()
+    yield packed, x, x_down
+    del packed
+    torch.cuda.empty_cache()
+
+
+def test_stream_packed_bytes(stream):
+    packed, _, _ = stream
+    total = sum(c.numel() + 2 * s.numel() + 2 * b.numel() for _, c, s, b in packed)
+    assert total == 4_192_337_920
+
+
+def test_stream_matmul_sampled(stream):
+    packed, x, x_down = stream
+    outs = []
+    for p, c, s, b in packed:
+        xi = x_down if p.K == 11264 else x
+        outs.append(q4.q4_matmul(xi, c, s, b))
+    torch.cuda.synchronize()
+    worst = 0.0
+    for i, ((p, c, s, b), y) in enumerate(zip(packed, outs)):
+        xi = x_down if p.K == 11264 else x
+        rows = sample_rows(p.N, 12, seed=i)
+        worst = max(worst, check_matmul(xi, c, s, b, y, rows=rows, what=p.name))
+    assert worst < 4e-3
+    assert q4.q4_debug_device_flags() == 0

@@ -1,0 +1,224 @@
+"""Python binding of libq4: affine 4-bit, group-32, weight-only quantized matmul
+for NVIDIA B200 (sm_100a).
+
+Argument marshalling only.  Every step of the computation runs in libq4's CUDA
+kernels, reached through the C ABI declared in ``include/q4.h``; there is no
+fallback of any kind.  If ``libq4.so`` is missing the first call raises.
+
+The functions take torch tensors (device memory and the current CUDA stream
+come from PyTorch) and have the same names as the C entry points:
+
+    codes, scales, biases = q4_quantize(W)            # W [N, K] bf16, cuda
+    W_hat = q4_dequantize(codes, scales, biases)        # [N, K] bf16
+    y = q4_matmul(x, codes, scales, biases)             # x [M, K] -> y [M, N]
+    y = q4_matmul_step(x, codes, scales, biases, num_steps, step)
+
+Layout (model card "personaplex-edge-q4", "Release details": affine Q4,
+group size 32, BF16): codes [N, K/2] uint8 (low nibble = even k), scales
+and biases [N, K/32] bf16, w_hat = scale * q + bias.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "Q4Error",
+    "GROUP",
+    "lib",
+    "library_path",
+    "q4_quantize",
+    "q4_dequantize",
+    "q4_matmul",
+    "q4_matmul_step",
+    "q4_debug_device_flags",
+    "q4_debug_launch_count",
+]
+
+GROUP = 32
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libq4.so")
+
+_STATUS = {
+    0: "Q4_OK",
+    1: "Q4_ERR_NULL",
+    2: "Q4_ERR_SHAPE",
+    3: "Q4_ERR_ALIGN",
+    4: "Q4_ERR_UNSUPPORTED",
+    5: "Q4_ERR_RANGE",
+    6: "Q4_ERR_CUDA",
+}
+
+# Exported C symbols and their ctypes signatures.
+_I64, _P, _INT = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+SIGNATURES = {
+    "q4_quantize": (_INT, [_P, _I64, _I64, _INT, _P, _P, _P, _P]),
+    "q4_dequantize": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),
+    "q4_matmul": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P]),
+    "q4_matmul_step": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P, _P]),
+    "q4_last_error": (ctypes.c_char_p, []),
+    "q4_debug_device_flags": (_INT, [_INT]),
+    "q4_debug_launch_count": (ctypes.c_ulonglong, []),
+}
+
+
+class Q4Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        self.status_name = _STATUS.get(status, str(status))
+        super().__init__(f"{self.status_name}: {message}")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libq4 (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"libq4.so not found at {_LIB_PATH}; build it with "
+                "`python -m weight_only_bit_affine_b200.build` (there is no non-CUDA fallback)")
+        handle = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        msg = lib().q4_last_error()
+        raise Q4Error(status, msg.decode() if msg else "")
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _want(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def q4_quantize(W: torch.Tensor, group: int = GROUP) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """W [N, K] bf16 -> (codes [N, K/2] uint8, scales [N, K/32] bf16, biases [N, K/32] bf16)."""
+    _want(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    dev = W.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, max(K // GROUP, 0)), dtype=torch.bfloat16, device=dev)
+    biases = torch.empty_like(scales)
+    with torch.cuda.device(dev):
+        _check(lib().q4_quantize(_ptr(W), N, K, group, _ptr(codes), _ptr(scales), _ptr(biases), _stream(dev)))
+    return codes, scales, biases
+
+
+def q4_dequantize(codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor, group: int = GROUP,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """(codes, scales, biases) -> W_hat [N, K] bf16 = bf16(scale * q + bias)."""
+    _want(codes, "codes", torch.uint8, 2)
+    _want(scales, "scales", torch.bfloat16, 2)
+    _want(biases, "biases", torch.bfloat16, 2)
+    N, K = codes.shape[0], codes.shape[1] * 2
+    dev = codes.device
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    else:
+        _want(out, "out", torch.bfloat16, 2)
+    if scales.shape != (N, K // GROUP) or biases.shape != (N, K // GROUP) or out.shape != (N, K):
+        raise ValueError("codes / scales / biases / out shapes disagree")
+    with torch.cuda.device(dev):
+        _check(lib().q4_dequantize(_ptr(codes), _ptr(scales), _ptr(biases), N, K, group, _ptr(out), _stream(dev)))
+    return out
+
+
+def _matmul_shapes(x, codes, scales, biases, rows_per_step):
+    _want(x, "x", torch.bfloat16, 2)
+    _want(codes, "codes", torch.uint8, 2)
+    _want(scales, "scales", torch.bfloat16, 2)
+    _want(biases, "biases", torch.bfloat16, 2)
+    M, K = x.shape
+    if codes.shape[1] * 2 != K:
+        raise ValueError(f"x has K = {K} but codes rows hold {codes.shape[1] * 2} codes")
+    if scales.shape != (codes.shape[0], K // GROUP) or biases.shape != scales.shape:
+        raise ValueError("scales / biases must be [rows, K/32]")
+    if not (x.device == codes.device == scales.device == biases.device):
+        raise ValueError("all tensors must be on the same device")
+    return M, K
+
+
+def q4_matmul(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+              group: int = GROUP, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = x . w_hat^T:  x [M, K] bf16, packed W with N rows -> y [M, N] bf16."""
+    M, K = _matmul_shapes(x, codes, scales, biases, None)
+    N = codes.shape[0]
+    dev = x.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    else:
+        _want(out, "out", torch.bfloat16, 2)
+        if out.shape != (M, N):
+            raise ValueError(f"out must be [{M}, {N}]")
+    with torch.cuda.device(dev):
+        _check(lib().q4_matmul(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N, group, _ptr(out),
+                               _stream(dev)))
+    return out
+
+
+def q4_matmul_step(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+                   num_steps: int, step: int, group: int = GROUP,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Step `step` of a stacked [num_steps * N, K] packed weight: rows [step*N, (step+1)*N)."""
+    M, K = _matmul_shapes(x, codes, scales, biases, None)
+    rows = codes.shape[0]
+    if num_steps < 1 or rows % num_steps:
+        raise ValueError(f"stacked rows {rows} not divisible by num_steps {num_steps}")
+    N = rows // num_steps
+    dev = x.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    else:
+        _want(out, "out", torch.bfloat16, 2)
+        if out.shape != (M, N):
+            raise ValueError(f"out must be [{M}, {N}]")
+    with torch.cuda.device(dev):
+        _check(lib().q4_matmul_step(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N, num_steps, step,
+                                    group, _ptr(out), _stream(dev)))
+    return out
+
+
+def q4_debug_device_flags(clear: bool = False) -> int:
+    """Bounded-wait flags of the current device (synchronizes); 0 means none fired."""
+    r = lib().q4_debug_device_flags(1 if clear else 0)
+    if r < 0:
+        raise Q4Error(6, "could not read device flags")
+    return r
+
+
+def q4_debug_launch_count() -> int:
+    """Kernel launches libq4 has enqueued in this process (host-side count)."""
+    return int(lib().q4_debug_launch_count())

@@ -1,0 +1,181 @@
+// q4_api.cu -- the extern "C" boundary of libq4 (declared in include/q4.h):
+// argument validation on the host, device checks, dispatch to the kernels.
+// Nothing throws across the boundary; a non-OK status means nothing was
+// enqueued on the stream.
+#include "q4.h"
+#include "q4_internal.h"
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+
+namespace q4 {
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+q4_status fail(q4_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+std::atomic<unsigned long long> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::atomic<bool> g_device_ready[kMaxDevices];
+std::mutex g_device_mutex;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Common checks of the current device.  Returns Q4_OK with *out set.
+q4_status check_device(const DeviceInfo** out) {
+  const DeviceInfo* d = current_device_info();
+  if (!d) return Q4_ERR_CUDA;
+  if (d->cc_major != 10 || d->cc_minor != 0)
+    return fail(Q4_ERR_UNSUPPORTED, "device %d has compute capability %d.%d; libq4 is built for sm_100a (10.0)",
+                d->device, d->cc_major, d->cc_minor);
+  *out = d;
+  return Q4_OK;
+}
+
+q4_status check_k_group(int64_t K, int group) {
+  if (group != 32) return fail(Q4_ERR_UNSUPPORTED, "group size %d is not supported (only 32)", group);
+  if (K < 32 || K % 32 != 0) return fail(Q4_ERR_SHAPE, "K = %lld must be a positive multiple of 32", (long long)K);
+  return Q4_OK;
+}
+
+q4_status from_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return Q4_OK;
+  return fail(Q4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+q4_status matmul_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* codes, const uint16_t* scales,
+                      const uint16_t* biases, int64_t N, int group, uint16_t* y, cudaStream_t stream) {
+  q4_status st = check_k_group(K, group);
+  if (st != Q4_OK) return st;
+  if (M < 0 || N < 0) return fail(Q4_ERR_SHAPE, "negative size M = %lld, N = %lld", (long long)M, (long long)N);
+  if (M == 0 || N == 0) return Q4_OK;
+  if (!x || !codes || !scales || !biases || !y) return fail(Q4_ERR_NULL, "q4_matmul: NULL pointer argument");
+  if (!aligned(x, 16) || !aligned(codes, 16))
+    return fail(Q4_ERR_ALIGN, "q4_matmul: x and codes must be 16-byte aligned");
+  if (!aligned(scales, 2) || !aligned(biases, 2) || !aligned(y, 2))
+    return fail(Q4_ERR_ALIGN, "q4_matmul: scales, biases and y must be 2-byte aligned");
+  if (N > (int64_t(1) << 40) || M > (int64_t(1) << 31) || K > (int64_t(1) << 24))
+    return fail(Q4_ERR_UNSUPPORTED, "q4_matmul: sizes beyond the supported range");
+  const DeviceInfo* dev;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  MatmulArgs a{x, codes, scales, biases, y, M, N, K};
+  return from_cuda(launch_gemv(a, stream, *dev), "q4_matmul launch");
+}
+
+}  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+const DeviceInfo* current_device_info() {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    fail(Q4_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    fail(Q4_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    return nullptr;
+  }
+  if (g_device_ready[dev].load(std::memory_order_acquire)) return &g_devices[dev];
+  std::lock_guard<std::mutex> lock(g_device_mutex);
+  if (!g_device_ready[dev].load(std::memory_order_relaxed)) {
+    DeviceInfo d;
+    d.device = dev;
+    int smem_optin = 0;
+    if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) {
+      fail(Q4_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    d.smem_optin = static_cast<size_t>(smem_optin);
+    g_devices[dev] = d;
+    g_device_ready[dev].store(true, std::memory_order_release);
+  }
+  return &g_devices[dev];
+}
+
+}  // namespace q4
+
+using namespace q4;
+
+extern "C" {
+
+q4_status q4_quantize(const q4_bf16* W, int64_t N, int64_t K, int group, uint8_t* codes, q4_bf16* scales,
+                      q4_bf16* biases, q4_stream_t stream) {
+  q4_status st = check_k_group(K, group);
+  if (st != Q4_OK) return st;
+  if (N < 0) return fail(Q4_ERR_SHAPE, "negative N = %lld", (long long)N);
+  if (N == 0) return Q4_OK;
+  if (!W || !codes || !scales || !biases) return fail(Q4_ERR_NULL, "q4_quantize: NULL pointer argument");
+  if (!aligned(W, 16) || !aligned(codes, 16))
+    return fail(Q4_ERR_ALIGN, "q4_quantize: W and codes must be 16-byte aligned");
+  if (!aligned(scales, 2) || !aligned(biases, 2))
+    return fail(Q4_ERR_ALIGN, "q4_quantize: scales and biases must be 2-byte aligned");
+  const DeviceInfo* dev;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  return from_cuda(launch_quantize(W, N, K, codes, scales, biases, reinterpret_cast<cudaStream_t>(stream), *dev),
+                   "q4_quantize launch");
+}
+
+q4_status q4_dequantize(const uint8_t* codes, const q4_bf16* scales, const q4_bf16* biases, int64_t N, int64_t K,
+                        int group, q4_bf16* W_out, q4_stream_t stream) {
+  q4_status st = check_k_group(K, group);
+  if (st != Q4_OK) return st;
+  if (N < 0) return fail(Q4_ERR_SHAPE, "negative N = %lld", (long long)N);
+  if (N == 0) return Q4_OK;
+  if (!W_out || !codes || !scales || !biases) return fail(Q4_ERR_NULL, "q4_dequantize: NULL pointer argument");
+  if (!aligned(W_out, 16) || !aligned(codes, 16))
+    return fail(Q4_ERR_ALIGN, "q4_dequantize: W_out and codes must be 16-byte aligned");
+  if (!aligned(scales, 2) || !aligned(biases, 2))
+    return fail(Q4_ERR_ALIGN, "q4_dequantize: scales and biases must be 2-byte aligned");
+  const DeviceInfo* dev;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  return from_cuda(
+      launch_dequantize(codes, scales, biases, N, K, W_out, reinterpret_cast<cudaStream_t>(stream), *dev),
+      "q4_dequantize launch");
+}
+
+q4_status q4_matmul(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes, const q4_bf16* scales,
+                    const q4_bf16* biases, int64_t N, int group, q4_bf16* y, q4_stream_t stream) {
+  return matmul_impl(x, M, K, codes, scales, biases, N, group, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes, const q4_bf16* scales,
+                         const q4_bf16* biases, int64_t N, int64_t num_steps, int64_t step, int group, q4_bf16* y,
+                         q4_stream_t stream) {
+  q4_status st = check_k_group(K, group);
+  if (st != Q4_OK) return st;
+  if (num_steps < 1 || step < 0 || step >= num_steps)
+    return fail(Q4_ERR_RANGE, "q4_matmul_step: step %lld outside [0, %lld)", (long long)step, (long long)num_steps);
+  if (N < 0) return fail(Q4_ERR_SHAPE, "negative N = %lld", (long long)N);
+  if (!codes || !scales || !biases) return fail(Q4_ERR_NULL, "q4_matmul_step: NULL pointer argument");
+  const int64_t row0 = step * N;
+  return matmul_impl(x, M, K, codes + row0 * (K / 2), scales + row0 * (K / 32), biases + row0 * (K / 32), N, group,
+                     y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+const char* q4_last_error(void) { return t_last_error; }
+
+unsigned long long q4_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int q4_debug_device_flags(int clear) {
+  unsigned int f = 0;
+  if (gemv_device_flags(&f, clear != 0) != cudaSuccess) return -1;
+  return static_cast<int>(f);
+}
+
+}  // extern "C"

@@ -1,0 +1,46 @@
+// q4_internal.h -- host-side launcher declarations shared inside libq4.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace q4 {
+
+// Device properties cached per device (first use of a device queries them).
+struct DeviceInfo {
+  int device = -1;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  size_t smem_optin = 0;  // max dynamic shared memory per block (opt-in)
+};
+// Returns nullptr (and sets the error message) if the current device cannot
+// be queried.
+const DeviceInfo* current_device_info();
+
+// Launchers return cudaSuccess or the launch error.  Arguments are already
+// validated by the ABI layer.
+cudaError_t launch_quantize(const uint16_t* W, int64_t N, int64_t K, uint8_t* codes,
+                            uint16_t* scales, uint16_t* biases, cudaStream_t stream,
+                            const DeviceInfo& dev);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint16_t* scales,
+                              const uint16_t* biases, int64_t N, int64_t K, uint16_t* W_out,
+                              cudaStream_t stream, const DeviceInfo& dev);
+
+struct MatmulArgs {
+  const uint16_t* x;  // [M, K]
+  const uint8_t* codes;
+  const uint16_t* scales;
+  const uint16_t* biases;
+  uint16_t* y;  // [M, N]
+  int64_t M, N, K;
+};
+// CUDA-core GEMV family, any M (processed in chunks of at most 4 rows).
+cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev);
+
+// Counts every kernel launch libq4 enqueues (host side).
+void count_launch();
+
+// Diagnostic: the bounded-wait flags of the GEMV kernels (synchronous copy).
+cudaError_t gemv_device_flags(unsigned int* flags, bool clear);
+
+}  // namespace q4
