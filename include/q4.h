@@ -126,6 +126,34 @@ Q4_API q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K,
                          const q4_bf16* biases, int64_t N, int64_t num_steps,
                          int64_t step, int group, q4_bf16* y, q4_stream_t stream);
 
+/* One problem of q4_matmul_batch: pointers and sizes as for q4_matmul. */
+typedef struct {
+  const q4_bf16* x;       /* [M, K] activations, 16-byte aligned   */
+  const uint8_t* codes;   /* [N, K/2], 16-byte aligned               */
+  const q4_bf16* scales;  /* [N, K/32]                               */
+  const q4_bf16* biases;  /* [N, K/32]                               */
+  q4_bf16* y;             /* [M, N] output                           */
+  int64_t N;
+  int64_t K;
+} q4_matmul_desc;
+
+/*
+ * q4_matmul_batch -- `count` independent matmuls sharing the number of
+ * activation rows M, each computing exactly what q4_matmul computes, enqueued
+ * as few kernel launches as possible: one for up to 256 problems that take
+ * the bulk-copy GEMV path.  The Swift/MLX blog ("Performance optimizations":
+ * compiling the temporal transformer fuses its ~450 per-step kernel
+ * dispatches) and the ONNX README ("All four variants": CUDA Graph capture)
+ * both cut per-call launch overhead; this is that fusion for a whole weight
+ * stream (every projection of a decode step) in one launch.
+ * `descs` is a HOST array of `count` entries, read before the call returns.
+ * The problems run concurrently: no output may overlap any input of any
+ * problem in the list.  Validation covers every entry before anything is
+ * enqueued; count == 0 is a no-op; count < 0 is Q4_ERR_SHAPE.
+ */
+Q4_API q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int group,
+                                 q4_stream_t stream);
+
 /* Message for the calling thread's last non-OK status ("" if none). */
 Q4_API const char* q4_last_error(void);
 

@@ -34,6 +34,7 @@ __all__ = [
     "q4_dequantize",
     "q4_matmul",
     "q4_matmul_step",
+    "q4_matmul_batch",
     "q4_debug_device_flags",
     "q4_debug_launch_count",
 ]
@@ -59,10 +60,17 @@ SIGNATURES = {
     "q4_dequantize": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),
     "q4_matmul": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P]),
     "q4_matmul_step": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P, _P]),
+    "q4_matmul_batch": (_INT, [_P, _INT, _I64, _INT, _P]),
     "q4_last_error": (ctypes.c_char_p, []),
     "q4_debug_device_flags": (_INT, [_INT]),
     "q4_debug_launch_count": (ctypes.c_ulonglong, []),
 }
+
+
+class MatmulDesc(ctypes.Structure):
+    """Mirror of q4_matmul_desc (include/q4.h)."""
+
+    _fields_ = [("x", _P), ("codes", _P), ("scales", _P), ("biases", _P), ("y", _P), ("N", _I64), ("K", _I64)]
 
 
 class Q4Error(RuntimeError):
@@ -209,6 +217,35 @@ def q4_matmul_step(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, b
         _check(lib().q4_matmul_step(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N, num_steps, step,
                                     group, _ptr(out), _stream(dev)))
     return out
+
+
+def q4_matmul_batch(problems, group: int = GROUP):
+    """Independent matmuls in as few launches as possible.
+
+    `problems`: a sequence of (x, codes, scales, biases, out) tuples, every x
+    with the same number of rows M; `out` [M, N] bf16 is written.  Returns the
+    list of outputs.
+    """
+    problems = list(problems)
+    if not problems:
+        return []
+    descs = (MatmulDesc * len(problems))()
+    M = None
+    dev = None
+    for i, (x, codes, scales, biases, out) in enumerate(problems):
+        Mi, K = _matmul_shapes(x, codes, scales, biases, None)
+        if M is None:
+            M, dev = Mi, x.device
+        elif Mi != M or x.device != dev:
+            raise ValueError("all problems of a batch need the same M and device")
+        _want(out, "out", torch.bfloat16, 2)
+        if out.shape != (M, codes.shape[0]) or out.device != dev:
+            raise ValueError(f"out of problem {i} must be [{M}, {codes.shape[0]}] on {dev}")
+        descs[i] = MatmulDesc(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
+                              codes.shape[0], K)
+    with torch.cuda.device(dev):
+        _check(lib().q4_matmul_batch(ctypes.cast(descs, ctypes.c_void_p), len(problems), M, group, _stream(dev)))
+    return [p[4] for p in problems]
 
 
 def q4_debug_device_flags(clear: bool = False) -> int:

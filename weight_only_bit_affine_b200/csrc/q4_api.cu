@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
+#include <vector>
 
 namespace q4 {
 namespace {
@@ -54,19 +55,30 @@ q4_status from_cuda(cudaError_t e, const char* what) {
   return fail(Q4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-q4_status matmul_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* codes, const uint16_t* scales,
-                      const uint16_t* biases, int64_t N, int group, uint16_t* y, cudaStream_t stream) {
+// Host checks of one matmul; Q4_OK with *empty set when there is nothing to do.
+q4_status check_matmul(const char* who, const uint16_t* x, int64_t M, int64_t K, const uint8_t* codes,
+                       const uint16_t* scales, const uint16_t* biases, int64_t N, int group, const uint16_t* y,
+                       bool* empty) {
   q4_status st = check_k_group(K, group);
   if (st != Q4_OK) return st;
-  if (M < 0 || N < 0) return fail(Q4_ERR_SHAPE, "negative size M = %lld, N = %lld", (long long)M, (long long)N);
-  if (M == 0 || N == 0) return Q4_OK;
-  if (!x || !codes || !scales || !biases || !y) return fail(Q4_ERR_NULL, "q4_matmul: NULL pointer argument");
+  if (M < 0 || N < 0) return fail(Q4_ERR_SHAPE, "%s: negative size M = %lld, N = %lld", who, (long long)M, (long long)N);
+  *empty = (M == 0 || N == 0);
+  if (*empty) return Q4_OK;
+  if (!x || !codes || !scales || !biases || !y) return fail(Q4_ERR_NULL, "%s: NULL pointer argument", who);
   if (!aligned(x, 16) || !aligned(codes, 16))
-    return fail(Q4_ERR_ALIGN, "q4_matmul: x and codes must be 16-byte aligned");
+    return fail(Q4_ERR_ALIGN, "%s: x and codes must be 16-byte aligned", who);
   if (!aligned(scales, 2) || !aligned(biases, 2) || !aligned(y, 2))
-    return fail(Q4_ERR_ALIGN, "q4_matmul: scales, biases and y must be 2-byte aligned");
+    return fail(Q4_ERR_ALIGN, "%s: scales, biases and y must be 2-byte aligned", who);
   if (N > (int64_t(1) << 40) || M > (int64_t(1) << 31) || K > (int64_t(1) << 24))
-    return fail(Q4_ERR_UNSUPPORTED, "q4_matmul: sizes beyond the supported range");
+    return fail(Q4_ERR_UNSUPPORTED, "%s: sizes beyond the supported range", who);
+  return Q4_OK;
+}
+
+q4_status matmul_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* codes, const uint16_t* scales,
+                      const uint16_t* biases, int64_t N, int group, uint16_t* y, cudaStream_t stream) {
+  bool empty = false;
+  q4_status st = check_matmul("q4_matmul", x, M, K, codes, scales, biases, N, group, y, &empty);
+  if (st != Q4_OK || empty) return st;
   const DeviceInfo* dev;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   MatmulArgs a{x, codes, scales, biases, y, M, N, K};
@@ -166,6 +178,29 @@ q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* 
   const int64_t row0 = step * N;
   return matmul_impl(x, M, K, codes + row0 * (K / 2), scales + row0 * (K / 32), biases + row0 * (K / 32), N, group,
                      y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int group, q4_stream_t stream) {
+  if (count < 0) return fail(Q4_ERR_SHAPE, "q4_matmul_batch: negative count %d", count);
+  if (count == 0) return Q4_OK;
+  if (!descs) return fail(Q4_ERR_NULL, "q4_matmul_batch: NULL descriptor array");
+  std::vector<MatmulArgs> list;
+  list.reserve(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    const q4_matmul_desc& d = descs[i];
+    bool empty = false;
+    char who[48];
+    snprintf(who, sizeof who, "q4_matmul_batch[%d]", i);
+    q4_status st = check_matmul(who, d.x, M, d.K, d.codes, d.scales, d.biases, d.N, group, d.y, &empty);
+    if (st != Q4_OK) return st;
+    if (!empty) list.push_back(MatmulArgs{d.x, d.codes, d.scales, d.biases, d.y, M, d.N, d.K});
+  }
+  if (list.empty()) return Q4_OK;
+  const DeviceInfo* dev;
+  q4_status st;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  return from_cuda(launch_gemv_batch(list.data(), static_cast<int>(list.size()), reinterpret_cast<cudaStream_t>(stream), *dev),
+                   "q4_matmul_batch launch");
 }
 
 const char* q4_last_error(void) { return t_last_error; }

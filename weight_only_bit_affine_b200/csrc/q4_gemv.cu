@@ -1,5 +1,5 @@
 // q4_gemv.cu -- the CUDA-core GEMV family of the affine Q4 group-32 matmul,
-// for few activation rows (decode, M < 16):
+// for one or two activation rows (decode):
 //
 //   y[m,n] = sum_g ( s[n,g] * sum_{k in g} x[m,k] q[n,k]  +  b[n,g] * sum_{k in g} x[m,k] )
 //
@@ -8,36 +8,36 @@
 // matmul).  The weights are read once from HBM in packed form and never
 // expanded in memory.
 //
-// Design (bandwidth-bound: ~1.6 flop per packed byte at M = 1):
-//  * One persistent CTA per SM.  A producer warp streams tiles of `rt` whole
-//    weight rows (codes, scales, biases: contiguous ranges) into a ring of
-//    shared-memory stages with 1-D bulk (TMA) copies; the bytes in flight are
-//    bounded by the ring, not by registers.
-//  * Consumer threads form "teams" of K/KPL lanes; a team owns one weight row
-//    at a time and lane j always covers the same KPL inputs k, so its slice of
-//    x lives in registers for the whole kernel (the row reduction over K is
-//    split across the team and finished with warp shuffles plus a
-//    shared-memory step between the team's warps).
-//  * Nibbles are unpacked in registers into bf16x2 values 128 + q (one LOP3
-//    per two codes) and multiplied with bf16 x by fp32-accumulating FMAs; the
-//    offset is removed per group exactly:  s*sum x(128+q) + (b - 128 s)*sum x.
-//  * Programmatic dependent launch: each kernel lets the next one launch
-//    early; before waiting for its predecessor the next kernel only issues L2
-//    prefetches of its own weights (a hint with no effect on values), so the
-//    weight stream of back-to-back matmuls keeps HBM busy across launches.
+// One launch runs a LIST of independent matmuls ("problems"): the temporal
+// step's projections, or a single q4_matmul.  Design (bandwidth-bound at
+// ~1.6 flop per packed byte):
+//  * One persistent CTA per SM takes a balanced contiguous share of the rows
+//    of every problem in turn.  A producer warp streams those rows (codes,
+//    scales, biases: contiguous byte ranges) through a ring of shared-memory
+//    stages with 1-D bulk (TMA) copies, and each problem's activations into
+//    one of two shared-memory slots; the ring never drains between problems.
+//  * Consumer threads form "teams" of K/32 lanes; a team owns one weight row
+//    at a time and lane j always covers input group j, so its slice of x sits
+//    in registers for the whole problem.  Each warp sums its lanes with a
+//    transpose-reduce; the sums across a team's warps are finished by an
+//    epilogue warp behind mbarriers, so consumers never block on each other.
+//  * Codes are unpacked in registers to bf16x2 "128 + q" (one LOP3 per two
+//    codes) and multiplied with bf16 x by fma.rn.f32.bf16 (exact products,
+//    fp32 accumulation); the offset is removed per group exactly:
+//    s*sum x(128+q) + (b - 128 s)*sum x.
+//  * Programmatic dependent launch: before waiting for the previous kernel a
+//    launch only prefetches its first weight tiles into L2 (a hint, no effect
+//    on values); everything that reads memory another kernel may write comes
+//    after the wait.
 #include "q4_device.cuh"
 #include "q4_internal.h"
 
 #include <algorithm>
+#include <cstdint>
+#include <vector>
 
-#ifndef Q4_GEMV_CTAS_PER_SM
-#define Q4_GEMV_CTAS_PER_SM 1
-#endif
 #ifndef Q4_GEMV_SMEM_BUDGET
 #define Q4_GEMV_SMEM_BUDGET (200 * 1024)
-#endif
-#ifndef Q4_GEMV_TARGET_THREADS
-#define Q4_GEMV_TARGET_THREADS 512
 #endif
 #ifndef Q4_GEMV_MAC
 #define Q4_GEMV_MAC 0
@@ -55,23 +55,6 @@ namespace {
 enum Mac { kMacMixedBf16 = 0, kMacFfma2 = 1, kMacMagicSub = 2 };
 template <int MAC>
 constexpr float mac_offset() { return MAC == kMacMagicSub ? 0.f : 128.f; }
-
-struct TmaGemvParams {
-  const uint16_t* x;       // [MR, K] (row stride K)
-  const uint8_t* codes;    // [N, K/2]
-  const uint16_t* scales;  // [N, G]
-  const uint16_t* biases;  // [N, G]
-  uint16_t* y;             // [MR, y_ld]
-  int64_t N, y_ld;
-  int K, G;
-  int team;              // lanes per weight row (a multiple of 32, or a power of two below 32)
-  int teams;             // teams per CTA
-  int rt;                // rows per tile (= teams * RPT)
-  int stages;
-  int consumer_threads;  // teams * team (a multiple of 32)
-  int chunk_tiles;       // tiles whose cross-warp partial sums are reduced together
-  uint32_t codes_tile_bytes, sb_tile_bytes, stage_bytes;
-};
 
 template <int W>
 __device__ __forceinline__ float seg_allreduce(float v) {
@@ -215,188 +198,300 @@ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
 
 __device__ __forceinline__ uint16_t to_bf16_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 
-template <int MR, int KPL, int RPT, int MAC, int MAXT>
-__global__ void __launch_bounds__(MAXT, 1) gemv_tma_kernel(const __grid_constant__ TmaGemvParams p) {
+
+// Problems per launch: their descriptors travel in the kernel parameters
+// (a small instance for single calls, a large one for batches).
+constexpr int kMaxProblems = 256;
+constexpr int kFewProblems = 4;
+constexpr int kRpt = 4;            // weight rows per team per tile
+
+struct GemvProblem {
+  const uint16_t* x;       // [MR, K]
+  const uint8_t* codes;    // [N, K/2]
+  const uint16_t* scales;  // [N, K/32]
+  const uint16_t* biases;  // [N, K/32]
+  uint16_t* y;             // [MR, y_ld]
+  int64_t N, y_ld;
+  int32_t K, pad_;
+};
+
+template <int NP>
+struct GemvLaunch {
+  int count;
+  int consumer_threads;  // a multiple of 32
+  int stages;
+  uint32_t stage_bytes;  // >= every problem's tile, 128-byte multiple
+  uint32_t xslot_bytes;  // >= MR * K * 2 for every problem, 128-byte multiple
+  uint32_t red_floats;   // per reduction buffer
+  GemvProblem prob[NP];
+};
+
+// Shape of one problem for a given consumer count (host and device agree).
+struct Geometry {
+  int G;      // groups per row
+  int team;   // lanes per weight row: G rounded up to 32, or to a power of two below 32
+  int teams;  // teams in the CTA
+  int wpt;    // warps per team (0 when a warp holds several teams)
+  int rt;     // rows per tile
+};
+__host__ __device__ inline Geometry geometry_of(int K, int consumer_threads) {
+  Geometry g;
+  g.G = K / 32;
+  if (g.G >= 32) {
+    g.team = (g.G + 31) / 32 * 32;
+  } else {
+    g.team = 1;
+    while (g.team < g.G) g.team <<= 1;
+  }
+  g.teams = consumer_threads / g.team;
+  g.wpt = g.team >= 32 ? g.team / 32 : 0;
+  g.rt = g.teams * kRpt;
+  return g;
+}
+
+__device__ __forceinline__ uint32_t tile_rows(int64_t r_end, int64_t row0, int rt) {
+  return static_cast<uint32_t>((r_end - row0 < rt) ? (r_end - row0) : rt);
+}
+
+template <int MR, int MAXT, int NP>
+__global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ GemvLaunch<NP> L) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int WORDS = KPL / 8;
-  constexpr int V = RPT * MR;
+  constexpr int V = kRpt * MR;
   constexpr int VP = pow2_at_least(V);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int consumer_warps = p.consumer_threads >> 5;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);
-  uint64_t* empty_bar = full_bar + p.stages;
-  float* red = reinterpret_cast<float*>(empty_bar + p.stages);
+  const int consumer_warps = L.consumer_threads >> 5;
 
-  // This CTA's contiguous share of the weight rows (balanced to within one row).
-  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * p.N / gridDim.x;
-  const int64_t r_end = static_cast<int64_t>(blockIdx.x + 1) * p.N / gridDim.x;
-  const int64_t cta_rows = r_end - r_begin;
-  const int ntiles = static_cast<int>((cta_rows + p.rt - 1) / p.rt);
+  uint8_t* xslots = smem + static_cast<size_t>(L.stages) * L.stage_bytes;
+  float* red = reinterpret_cast<float*>(xslots + 2 * static_cast<size_t>(L.xslot_bytes));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(red + 2 * static_cast<size_t>(L.red_floats));
+  uint64_t* empty_bar = full_bar + L.stages;
+  uint64_t* xfull_bar = empty_bar + L.stages;  // [2]
+  uint64_t* xempty_bar = xfull_bar + 2;        // [2]
+  uint64_t* rfull_bar = xempty_bar + 2;        // [2]
+  uint64_t* rempty_bar = rfull_bar + 2;        // [2]
 
   if (tid == 0) {
-    for (int s = 0; s < p.stages; ++s) {
+    for (int s = 0; s < L.stages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], consumer_warps);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&xfull_bar[s], 1);
+      mbar_init(&xempty_bar[s], consumer_warps);
+      mbar_init(&rfull_bar[s], consumer_warps);
+      mbar_init(&rempty_bar[s], 1);
     }
     fence_mbar_init();
   }
   __syncthreads();
   pdl_launch_dependents();
 
-  const int half_k = p.K >> 1;
+  const int64_t cta = blockIdx.x, grid = gridDim.x;
+
   if (warp == consumer_warps) {
     // ---------------- producer warp ----------------
     if (lane == 0) {
-      // Warm L2 with the first tiles while the previous kernel may still run
-      // (a prefetch is a hint: it changes no value any thread observes).
-      for (int t = 0; t < ntiles && t < p.stages; ++t) {
-        const int64_t row0 = r_begin + static_cast<int64_t>(t) * p.rt;
-        const uint32_t rows = static_cast<uint32_t>((r_end - row0 < p.rt) ? (r_end - row0) : p.rt);
-        bulk_prefetch_l2(p.codes + row0 * half_k, rows * half_k);
-        bulk_prefetch_l2(p.scales + row0 * p.G, rows * p.G * 2);
-        bulk_prefetch_l2(p.biases + row0 * p.G, rows * p.G * 2);
+      {  // warm L2 with the first problem's first tiles (a hint; changes no value)
+        const GemvProblem& P = L.prob[0];
+        const Geometry geo = geometry_of(P.K, L.consumer_threads);
+        const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
+        const int half_k = P.K >> 1;
+        for (int i = 0; i < L.stages; ++i) {
+          const int64_t row0 = r_begin + static_cast<int64_t>(i) * geo.rt;
+          if (row0 >= r_end) break;
+          const uint32_t rows = tile_rows(r_end, row0, geo.rt);
+          bulk_prefetch_l2(P.codes + row0 * half_k, rows * half_k);
+          bulk_prefetch_l2(P.scales + row0 * geo.G, rows * geo.G * 2);
+          bulk_prefetch_l2(P.biases + row0 * geo.G, rows * geo.G * 2);
+        }
       }
-    }
-    pdl_wait_predecessors();
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      for (int t = 0; t < ntiles; ++t) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) break;
-        const int64_t row0 = r_begin + static_cast<int64_t>(t) * p.rt;
-        const uint32_t rows = static_cast<uint32_t>((r_end - row0 < p.rt) ? (r_end - row0) : p.rt);
-        const uint32_t cb = rows * half_k, sb = rows * p.G * 2;
-        uint8_t* st = smem + static_cast<size_t>(stage) * p.stage_bytes;
-        mbar_arrive_expect_tx(&full_bar[stage], cb + 2 * sb);
-        bulk_g2s(st, p.codes + row0 * half_k, cb, &full_bar[stage]);
-        bulk_g2s(st + p.codes_tile_bytes, p.scales + row0 * p.G, sb, &full_bar[stage]);
-        bulk_g2s(st + p.codes_tile_bytes + p.sb_tile_bytes, p.biases + row0 * p.G, sb, &full_bar[stage]);
-        ++issued;
-        if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+      pdl_wait_predecessors();
+      int stage = 0, xs = 0, issued = 0, xissued = 0;
+      uint32_t phase = 0, xphase = 0;
+      bool dead = false;
+      for (int pi = 0; pi < L.count && !dead; ++pi) {
+        const GemvProblem& P = L.prob[pi];
+        const Geometry geo = geometry_of(P.K, L.consumer_threads);
+        const int half_k = P.K >> 1;
+        const uint32_t xbytes = static_cast<uint32_t>(MR) * P.K * 2;
+        if (!mbar_wait(&xempty_bar[xs], xphase ^ 1u)) { dead = true; break; }
+        mbar_arrive_expect_tx(&xfull_bar[xs], xbytes);
+        bulk_g2s(xslots + static_cast<size_t>(xs) * L.xslot_bytes, P.x, xbytes, &xfull_bar[xs]);
+        ++xissued;
+        if (++xs == 2) { xs = 0; xphase ^= 1u; }
+        const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
+        for (int64_t row0 = r_begin; row0 < r_end; row0 += geo.rt) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; break; }
+          const uint32_t rows = tile_rows(r_end, row0, geo.rt);
+          const uint32_t cb = rows * half_k, sb = rows * geo.G * 2;
+          const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
+          const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
+          uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
+          mbar_arrive_expect_tx(&full_bar[stage], cb + 2 * sb);
+          bulk_g2s(st, P.codes + row0 * half_k, cb, &full_bar[stage]);
+          bulk_g2s(st + sb_off, P.scales + row0 * geo.G, sb, &full_bar[stage]);
+          bulk_g2s(st + sb_off + sb_tile, P.biases + row0 * geo.G, sb, &full_bar[stage]);
+          ++issued;
+          if (++stage == L.stages) { stage = 0; phase ^= 1u; }
+        }
       }
-      // No copy may still target this CTA's shared memory when it exits: wait
-      // (bounded) for the last issued tile of every stage.
-      const int tail = min(issued, p.stages);
-      for (int i = 0; i < tail; ++i) {
+      // No copy may still target this CTA's shared memory when it exits.
+      for (int i = 0; i < min(issued, L.stages); ++i) {
         int s = stage - 1 - i;
         uint32_t ph = phase;
-        if (s < 0) { s += p.stages; ph ^= 1u; }
+        if (s < 0) { s += L.stages; ph ^= 1u; }
         mbar_wait(&full_bar[s], ph);
+      }
+      for (int i = 0; i < min(xissued, 2); ++i) {
+        int s = xs - 1 - i;
+        uint32_t ph = xphase;
+        if (s < 0) { s += 2; ph ^= 1u; }
+        mbar_wait(&xfull_bar[s], ph);
       }
     }
     return;
   }
 
-  // ---------------- consumer threads ----------------
-  const int team_idx = tid / p.team;
-  const int j = tid - team_idx * p.team;
-  const bool active = j < p.K / KPL;  // lanes past K own no inputs (padding)
-  const int g = (j * KPL) >> 5;
-  const int wpt = p.team >> 5;  // warps per team (0 when a warp holds several teams)
-  const int warp_in_team = (p.team >= 32) ? (j >> 5) : 0;
-  constexpr float kOffset = mac_offset<MAC>();
+  pdl_wait_predecessors();  // consumers and epilogue read x and write y
 
-  pdl_wait_predecessors();
-
-  XSlice<WORDS, MAC> xs[MR];
-#pragma unroll
-  for (int m = 0; m < MR; ++m) {
-    if (active)
-      xs[m].load(p.x + static_cast<int64_t>(m) * p.K + j * KPL);
-    else
-      xs[m].zero();
+  if (warp == consumer_warps + 1) {
+    // ---------------- epilogue warp: sums across a team's warps ----------------
+    int rb = 0;
+    uint32_t rph = 0;
+    bool dead = false;
+    for (int pi = 0; pi < L.count; ++pi) {
+      const GemvProblem& P = L.prob[pi];
+      const Geometry geo = geometry_of(P.K, L.consumer_threads);
+      if (geo.wpt <= 1) continue;
+      if (!dead && !mbar_wait(&rfull_bar[rb], rph)) dead = true;
+      const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
+      const int n_out = static_cast<int>(r_end - r_begin) * MR;
+      const float* rbuf = red + static_cast<size_t>(rb) * L.red_floats;
+      for (int i = lane; i < n_out; i += 32) {
+        float v = 0.f;
+        for (int w = 0; w < geo.wpt; ++w) v += rbuf[i * geo.wpt + w];
+        const int lr = i / MR, m = i - lr * MR;
+        P.y[static_cast<int64_t>(m) * P.y_ld + r_begin + lr] = to_bf16_bits(v);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rempty_bar[rb]);
+      if (++rb == 2) { rb = 0; rph ^= 1u; }
+    }
+    return;
   }
 
-  int stage = 0;
-  uint32_t phase = 0;
+  // ---------------- consumer threads ----------------
+  int stage = 0, xs = 0, rb = 0;
+  uint32_t phase = 0, xphase = 0, rph = 0;
   bool dead = false;
-  for (int c0 = 0; c0 < ntiles; c0 += p.chunk_tiles) {
-    const int c1 = min(ntiles, c0 + p.chunk_tiles);
-    for (int t = c0; t < c1; ++t) {
-      if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;  // on timeout: finish without waiting
-      const uint8_t* st = smem + static_cast<size_t>(stage) * p.stage_bytes;
-      const uint16_t* ssc = reinterpret_cast<const uint16_t*>(st + p.codes_tile_bytes);
-      const uint16_t* sbi = reinterpret_cast<const uint16_t*>(st + p.codes_tile_bytes + p.sb_tile_bytes);
-      const int r_first = team_idx * RPT;                        // first row of this team in the tile
-      const int64_t grow0 = r_begin + static_cast<int64_t>(t) * p.rt + r_first;
+  for (int pi = 0; pi < L.count; ++pi) {
+    const GemvProblem& P = L.prob[pi];
+    const Geometry geo = geometry_of(P.K, L.consumer_threads);
+    const int half_k = P.K >> 1;
+    const int team_idx = tid / geo.team;
+    const int j = tid - team_idx * geo.team;
+    const bool active = team_idx < geo.teams && j < geo.G;
+    const int warp_in_team = (geo.team >= 32) ? (j >> 5) : 0;
+    const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
+    const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
+    const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
+
+    // Activations: this lane's 32 inputs of each row, from the staged slot.
+    if (!dead && !mbar_wait(&xfull_bar[xs], xphase)) dead = true;
+    XSlice<4, Q4_GEMV_MAC> xsl[MR];
+    {
+      const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(xslots + static_cast<size_t>(xs) * L.xslot_bytes);
+#pragma unroll
+      for (int m = 0; m < MR; ++m) {
+        if (active)
+          xsl[m].load(xsrc + m * P.K + j * 32);
+        else
+          xsl[m].zero();
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&xempty_bar[xs]);
+    if (++xs == 2) { xs = 0; xphase ^= 1u; }
+
+    const bool use_red = geo.wpt > 1;
+    if (use_red && !dead && !mbar_wait(&rempty_bar[rb], rph ^ 1u)) dead = true;
+    float* rbuf = red + static_cast<size_t>(rb) * L.red_floats;
+    constexpr float kOffset = mac_offset<Q4_GEMV_MAC>();
+
+    for (int64_t row0 = r_begin; row0 < r_end; row0 += geo.rt) {
+      if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
+      const uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
+      const uint16_t* ssc = reinterpret_cast<const uint16_t*>(st + sb_off);
+      const uint16_t* sbi = reinterpret_cast<const uint16_t*>(st + sb_off + sb_tile);
+      const int r_first = team_idx * kRpt;
+      const int64_t grow0 = row0 + r_first;
+
+      uint32_t words[kRpt][4];
+      float sc[kRpt], bi[kRpt];
+#pragma unroll
+      for (int rr = 0; rr < kRpt; ++rr) {  // all shared-memory loads first
+        const int r = r_first + rr;
+        if (active && grow0 + rr < r_end) {
+          load_words_smem<4>(st + static_cast<size_t>(r) * half_k + j * 16, words[rr]);
+          sc[rr] = bf16_bits_to_float(ssc[r * geo.G + j]);
+          bi[rr] = bf16_bits_to_float(sbi[r * geo.G + j]);
+        } else {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) words[rr][w] = 0u;
+          sc[rr] = bi[rr] = 0.f;
+        }
+      }
+      // The stage's bytes are in registers now: hand it back to the producer.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[stage]);
+      if (++stage == L.stages) { stage = 0; phase ^= 1u; }
 
       float vals[VP];
 #pragma unroll
       for (int i = 0; i < VP; ++i) vals[i] = 0.f;
-      uint32_t words[RPT][WORDS];
-      float sc[RPT], bi[RPT];
 #pragma unroll
-      for (int rr = 0; rr < RPT; ++rr) {  // issue all shared-memory loads first
-        const int r = r_first + rr;
-        if (active && grow0 + rr < r_end) {
-          load_words_smem<WORDS>(st + static_cast<size_t>(r) * half_k + j * (KPL / 2), words[rr]);
-          sc[rr] = bf16_bits_to_float(ssc[r * p.G + g]);
-          bi[rr] = bf16_bits_to_float(sbi[r * p.G + g]);
-        } else {
-#pragma unroll
-          for (int w = 0; w < WORDS; ++w) words[rr][w] = 0u;
-          sc[rr] = bi[rr] = 0.f;
-        }
-      }
-      // The stage's bytes are now in registers: hand it back to the producer.
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[stage]);
-      if (++stage == p.stages) { stage = 0; phase ^= 1u; }
-
-#pragma unroll
-      for (int rr = 0; rr < RPT; ++rr) {
+      for (int rr = 0; rr < kRpt; ++rr) {
         float a0[MR], a1[MR];
 #pragma unroll
         for (int m = 0; m < MR; ++m) a0[m] = a1[m] = 0.f;
-        dot_plus128<MR, WORDS, MAC>(words[rr], xs, a0, a1);
+        dot_plus128<MR, 4, Q4_GEMV_MAC>(words[rr], xsl, a0, a1);
         const float c = fmaf(-kOffset, sc[rr], bi[rr]);
 #pragma unroll
-        for (int m = 0; m < MR; ++m) vals[rr * MR + m] = fmaf(sc[rr], a0[m] + a1[m], c * xs[m].sum);
+        for (int m = 0; m < MR; ++m) vals[rr * MR + m] = fmaf(sc[rr], a0[m] + a1[m], c * xsl[m].sum);
       }
 
-      if (p.team >= 32) {
+      if (geo.team >= 32) {
         const float tot = transpose_reduce<VP>(vals, lane);
         const int idx = lane >> (5 - ilog2(VP));
-        const bool holder = (lane & ((32 / VP) - 1)) == 0 && idx < V;
+        const bool holder = (lane & ((32 / VP) - 1)) == 0 && idx < V && team_idx < geo.teams;
         const int rr = idx / MR, m = idx % MR;
         if (holder && grow0 + rr < r_end) {
-          if (wpt == 1) {
-            p.y[static_cast<int64_t>(m) * p.y_ld + grow0 + rr] = to_bf16_bits(tot);
+          if (!use_red) {
+            P.y[static_cast<int64_t>(m) * P.y_ld + grow0 + rr] = to_bf16_bits(tot);
           } else {
-            const int lr = (t - c0) * p.rt + r_first + rr;  // row within the chunk
-            red[(lr * MR + m) * wpt + warp_in_team] = tot;
+            const int lr = static_cast<int>(grow0 + rr - r_begin);  // row within this CTA's share
+            rbuf[(lr * MR + m) * geo.wpt + warp_in_team] = tot;
           }
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < V; ++i) vals[i] = seg_allreduce_dyn(vals[i], p.team);
-        if (j == 0) {
+        for (int i = 0; i < V; ++i) vals[i] = seg_allreduce_dyn(vals[i], geo.team);
+        if (j == 0 && team_idx < geo.teams) {
 #pragma unroll
-          for (int rr = 0; rr < RPT; ++rr)
+          for (int rr = 0; rr < kRpt; ++rr)
             if (grow0 + rr < r_end) {
 #pragma unroll
               for (int m = 0; m < MR; ++m)
-                p.y[static_cast<int64_t>(m) * p.y_ld + grow0 + rr] = to_bf16_bits(vals[rr * MR + m]);
+                P.y[static_cast<int64_t>(m) * P.y_ld + grow0 + rr] = to_bf16_bits(vals[rr * MR + m]);
             }
         }
       }
     }
-    if (wpt > 1) {
-      // Cross-warp sums of this chunk's rows, once per chunk (consumers only).
-      named_bar_sync(1, p.consumer_threads);
-      const int64_t row_a = r_begin + static_cast<int64_t>(c0) * p.rt;
-      const int64_t row_b = min(r_end, r_begin + static_cast<int64_t>(c1) * p.rt);
-      const int n_out = static_cast<int>(row_b - row_a) * MR;
-      for (int i = tid; i < n_out; i += p.consumer_threads) {
-        const float* rp = red + i * wpt;
-        float v = 0.f;
-        for (int w = 0; w < wpt; ++w) v += rp[w];
-        const int lr = i / MR, m = i - lr * MR;
-        p.y[static_cast<int64_t>(m) * p.y_ld + row_a + lr] = to_bf16_bits(v);
-      }
-      named_bar_sync(1, p.consumer_threads);
+    if (use_red) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfull_bar[rb]);
+      if (++rb == 2) { rb = 0; rph ^= 1u; }
     }
   }
 }
@@ -465,24 +560,20 @@ cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStre
   return cudaLaunchKernelEx(&cfg, kernel, prm);
 }
 
-constexpr int kKpl = 32;       // inputs per lane: one whole group (16 code bytes)
-constexpr int kMaxRows = 4;    // activation rows per chunk (x slice: 16*MR registers)
-constexpr int rpt_for(int mr) { return mr <= 2 ? 4 : 2; }  // weight rows per team per tile
+// Block shapes: consumers + producer warp + epilogue warp.  The thread
+// counts bound the registers (576 threads: 113 per thread; 416: 157).
+constexpr int kConsumers1 = 512, kThreads1 = kConsumers1 + 64;  // one activation row
+constexpr int kConsumers2 = 352, kThreads2 = kConsumers2 + 64;  // two activation rows
 
-template <int MR, int MAXT>
-cudaError_t run_tma(const MatmulArgs& a, int64_t m0, const TmaGemvParams& base, size_t smem, int grid,
-                    cudaStream_t stream) {
-  TmaGemvParams p = base;
-  p.x = a.x + m0 * a.K;
-  p.y = a.y + m0 * a.N;
-  auto kern = gemv_tma_kernel<MR, kKpl, rpt_for(MR), Q4_GEMV_MAC, MAXT>;
-  static bool attr_set = false;  // per template instance; idempotent if raced
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  return launch_pdl(kern, dim3(grid), dim3(p.consumer_threads + 32), smem, stream, p);
+int consumers_for(int mr) { return mr == 1 ? kConsumers1 : kConsumers2; }
+
+// Does the bulk-copy kernel take this problem (else: the generic kernel)?
+bool tma_ok(const MatmulArgs& a, int mr) {
+  const int64_t G = a.K / 32;
+  if (G % 8 != 0) return false;  // scale rows must be whole 16-byte runs for bulk copies
+  if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) return false;
+  const Geometry geo = geometry_of(static_cast<int>(a.K), consumers_for(mr));
+  return geo.teams >= 1 && geo.team <= consumers_for(mr);
 }
 
 template <int MR>
@@ -502,82 +593,80 @@ cudaError_t run_generic(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, 
   return launch_pdl(gemv_generic_kernel<MR>, dim3(grid), dim3(256), 0, stream, p);
 }
 
-// Chooses the TMA kernel's shape for one chunk of `mr` activation rows.
-// Returns false when the shape needs the generic kernel.
-bool plan_tma(const MatmulArgs& a, int mr, const DeviceInfo& dev, TmaGemvParams& p, size_t& smem, int& grid) {
-  const int64_t K = a.K, G = K / 32;
-  if (G % 8 != 0) return false;  // scale rows must be whole 16-byte runs for bulk copies
-  if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) return false;
-  const int64_t lanes = K / kKpl;
-  int64_t team;
-  if (lanes >= 32) {
-    team = (lanes + 31) / 32 * 32;
-  } else {
-    team = 1;
-    while (team < lanes) team <<= 1;
+// Launches the bulk-copy kernel over problems [first, last) of `probs`
+// (all taking this path, all with MR activation rows).
+template <int MR, int NP>
+cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev, cudaStream_t stream) {
+  constexpr int kThreads = MR == 1 ? kThreads1 : kThreads2;
+  const int consumers = consumers_for(MR);
+  const int grid = dev.sm_count;
+  static_assert(sizeof(GemvLaunch<NP>) <= 32000, "kernel parameters exceed the launch limit");
+  thread_local GemvLaunch<NP> L;  // copied into the launch parameters by cudaLaunchKernelEx
+  uint32_t stage_bytes = 128, xslot = 128, red_floats = 1;
+  for (int i = 0; i < count; ++i) {
+    const GemvProblem& P = probs[i];
+    const Geometry geo = geometry_of(P.K, consumers);
+    const uint32_t tile = static_cast<uint32_t>(geo.rt) * (P.K / 2) +
+                          2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
+    stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
+    xslot = std::max(xslot, (static_cast<uint32_t>(MR) * P.K * 2 + 127u) & ~127u);
+    if (geo.wpt > 1) {
+      const int64_t rows = (P.N + grid - 1) / grid;
+      red_floats = std::max<uint32_t>(red_floats, static_cast<uint32_t>(rows * MR * geo.wpt));
+    }
   }
-  // Launch-bound instances: 384 and 640 threads, i.e. up to 170 and 102
-  // registers per thread; only one activation row fits the 640-thread one
-  // without spilling.
-  const int max_consumers = (mr == 1) ? 608 : 352;
-  if (team > max_consumers) return false;
-  int teams = static_cast<int>(std::max<int64_t>(1, (Q4_GEMV_TARGET_THREADS + team / 2) / team));
-  teams = std::min<int>(teams, static_cast<int>(max_consumers / team));
-  if (team < 32) teams = std::max(teams, static_cast<int>(32 / team));
-  if ((teams * team) % 32) return false;
-  const int rpt = rpt_for(mr);
-  const int rt = teams * rpt;
-  const uint32_t codes_tile = static_cast<uint32_t>(rt * (K / 2));
-  const uint32_t sb_tile = static_cast<uint32_t>((rt * G * 2 + 15) / 16 * 16);
-  const uint32_t stage_bytes = (codes_tile + 2 * sb_tile + 127) / 128 * 128;
-  const int wpt = (team >= 32) ? static_cast<int>(team / 32) : 0;
-  grid = static_cast<int>(std::min<int64_t>(a.N, int64_t(dev.sm_count) * Q4_GEMV_CTAS_PER_SM));
-  const int64_t cta_rows = (a.N + grid - 1) / grid;
-  const int64_t cta_tiles = (cta_rows + rt - 1) / rt;
-  // Cross-warp partials: one float per (row, activation row, warp), at most 16 KB.
-  int chunk_tiles = static_cast<int>(cta_tiles);
-  size_t red_bytes = 0;
-  if (wpt > 1) {
-    const size_t per_tile = static_cast<size_t>(rt) * mr * wpt * sizeof(float);
-    chunk_tiles = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cta_tiles, (16 * 1024) / per_tile)));
-    red_bytes = per_tile * chunk_tiles;
-  }
+  red_floats = (red_floats + 31u) & ~31u;
+  const size_t fixed = 2 * static_cast<size_t>(xslot) + 2 * sizeof(float) * red_floats + 8 * 8;
   const size_t budget = std::min<size_t>(Q4_GEMV_SMEM_BUDGET, dev.smem_optin);
-  int stages = static_cast<int>((budget - red_bytes) / (stage_bytes + 16));
-  stages = std::min<int64_t>(std::min(stages, 8), std::max<int64_t>(2, cta_tiles));
-  if (stages < 2) stages = 2;
-  smem = static_cast<size_t>(stages) * stage_bytes + 16 * stages + red_bytes;
-  if (smem > dev.smem_optin) return false;
-  p.N = a.N;
-  p.y_ld = a.N;
-  p.K = static_cast<int>(K);
-  p.G = static_cast<int>(G);
-  p.codes = a.codes;
-  p.scales = a.scales;
-  p.biases = a.biases;
-  p.team = static_cast<int>(team);
-  p.teams = teams;
-  p.rt = rt;
-  p.stages = stages;
-  p.consumer_threads = static_cast<int>(team) * teams;
-  p.chunk_tiles = chunk_tiles;
-  p.codes_tile_bytes = codes_tile;
-  p.sb_tile_bytes = sb_tile;
-  p.stage_bytes = stage_bytes;
-  return true;
+  if (fixed + 2 * (stage_bytes + 16) > dev.smem_optin) return cudaErrorInvalidConfiguration;
+  int stages = static_cast<int>((budget > fixed ? budget - fixed : 0) / (stage_bytes + 16));
+  stages = std::max(2, std::min(stages, 8));
+  const size_t smem = static_cast<size_t>(stages) * stage_bytes + fixed + 16 * stages;
+  L.count = count;
+  L.consumer_threads = consumers;
+  L.stages = stages;
+  L.stage_bytes = stage_bytes;
+  L.xslot_bytes = xslot;
+  L.red_floats = red_floats;
+  for (int i = 0; i < count; ++i) L.prob[i] = probs[i];
+  auto kern = gemv_kernel<MR, kThreads, NP>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, L);
 }
 
+// Splits problems whose per-CTA reduction buffer would be too large into row
+// ranges, then launches in groups of at most kMaxProblems.
 template <int MR>
-cudaError_t run_chunk(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, cudaStream_t stream) {
-  TmaGemvParams p;
-  size_t smem;
-  int grid;
-  if (plan_tma(a, MR, dev, p, smem, grid)) {
-    const int threads = p.consumer_threads + 32;
-    if (threads <= 384) return run_tma<MR, 384>(a, m0, p, smem, grid, stream);
-    if constexpr (MR == 1) return run_tma<1, 640>(a, m0, p, smem, grid, stream);
+cudaError_t run_problems(std::vector<GemvProblem>& probs, const DeviceInfo& dev, cudaStream_t stream) {
+  const int consumers = consumers_for(MR);
+  std::vector<GemvProblem> split;
+  split.reserve(probs.size());
+  for (const GemvProblem& P : probs) {
+    const Geometry geo = geometry_of(P.K, consumers);
+    const int64_t max_rows_per_cta = geo.wpt > 1 ? std::max<int64_t>(1, 2048 / (MR * geo.wpt)) : INT64_MAX / 4;
+    const int64_t max_rows = max_rows_per_cta * dev.sm_count;
+    for (int64_t r = 0; r < P.N; r += max_rows) {
+      GemvProblem Q = P;
+      Q.N = std::min<int64_t>(max_rows, P.N - r);
+      Q.codes = P.codes + r * (P.K / 2);
+      Q.scales = P.scales + r * (P.K / 32);
+      Q.biases = P.biases + r * (P.K / 32);
+      Q.y = P.y + r;
+      split.push_back(Q);
+    }
   }
-  return run_generic<MR>(a, m0, dev, stream);
+  for (size_t i = 0; i < split.size(); i += kMaxProblems) {
+    const int n = static_cast<int>(std::min<size_t>(kMaxProblems, split.size() - i));
+    cudaError_t e = (n <= kFewProblems) ? run_list<MR, kFewProblems>(split.data() + i, n, dev, stream)
+                                        : run_list<MR, kMaxProblems>(split.data() + i, n, dev, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -591,19 +680,40 @@ cudaError_t gemv_device_flags(unsigned int* flags, bool clear) {
   return e;
 }
 
-cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev) {
-  for (int64_t m0 = 0; m0 < a.M; m0 += kMaxRows) {
-    const int mr = static_cast<int>(std::min<int64_t>(kMaxRows, a.M - m0));
-    cudaError_t e;
-    switch (mr) {
-      case 1: e = run_chunk<1>(a, m0, dev, stream); break;
-      case 2: e = run_chunk<2>(a, m0, dev, stream); break;
-      case 3: e = run_chunk<3>(a, m0, dev, stream); break;
-      default: e = run_chunk<4>(a, m0, dev, stream); break;
+cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev) {
+  // Activation rows in chunks of at most two; every chunk of every problem
+  // that fits the bulk-copy kernel joins one list per chunk size.
+  std::vector<GemvProblem> one, two;
+  for (int i = 0; i < count; ++i) {
+    const MatmulArgs& a = list[i];
+    for (int64_t m0 = 0; m0 < a.M; m0 += 2) {
+      const int mr = static_cast<int>(std::min<int64_t>(2, a.M - m0));
+      if (!tma_ok(a, mr)) {
+        cudaError_t e = (mr == 1) ? run_generic<1>(a, m0, dev, stream) : run_generic<2>(a, m0, dev, stream);
+        if (e != cudaSuccess) return e;
+        continue;
+      }
+      GemvProblem P;
+      P.x = a.x + m0 * a.K;
+      P.codes = a.codes;
+      P.scales = a.scales;
+      P.biases = a.biases;
+      P.y = a.y + m0 * a.N;
+      P.N = a.N;
+      P.y_ld = a.N;
+      P.K = static_cast<int32_t>(a.K);
+      P.pad_ = 0;
+      (mr == 1 ? one : two).push_back(P);
     }
-    if (e != cudaSuccess) return e;
   }
-  return cudaSuccess;
+  cudaError_t e = cudaSuccess;
+  if (!one.empty()) e = run_problems<1>(one, dev, stream);
+  if (e == cudaSuccess && !two.empty()) e = run_problems<2>(two, dev, stream);
+  return e;
+}
+
+cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev) {
+  return launch_gemv_batch(&a, 1, stream, dev);
 }
 
 }  // namespace q4

@@ -34,8 +34,12 @@ struct MatmulArgs {
   uint16_t* y;  // [M, N]
   int64_t M, N, K;
 };
-// CUDA-core GEMV family, any M (processed in chunks of at most 4 rows).
+// CUDA-core GEMV family, any M (activation rows in chunks of at most two;
+// every chunk re-reads the weights).
 cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev);
+// Several independent matmuls; those the bulk-copy kernel takes share one
+// launch (per chunk size).
+cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
 
 // Counts every kernel launch libq4 enqueues (host side).
 void count_launch();
