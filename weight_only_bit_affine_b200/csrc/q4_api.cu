@@ -82,6 +82,7 @@ q4_status matmul_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* co
   const DeviceInfo* dev;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   MatmulArgs a{x, codes, scales, biases, y, M, N, K};
+  if (M >= kTensorCoreMinRows && tc_supported(a)) return from_cuda(launch_tc(a, stream, *dev), "q4_matmul launch");
   return from_cuda(launch_gemv(a, stream, *dev), "q4_matmul launch");
 }
 
@@ -199,8 +200,17 @@ q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int
   const DeviceInfo* dev;
   q4_status st;
   if ((st = check_device(&dev)) != Q4_OK) return st;
-  return from_cuda(launch_gemv_batch(list.data(), static_cast<int>(list.size()), reinterpret_cast<cudaStream_t>(stream), *dev),
-                   "q4_matmul_batch launch");
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<MatmulArgs> gemv;
+  for (const MatmulArgs& a : list) {
+    if (a.M >= kTensorCoreMinRows && tc_supported(a)) {
+      if ((st = from_cuda(launch_tc(a, cs, *dev), "q4_matmul_batch launch")) != Q4_OK) return st;
+    } else {
+      gemv.push_back(a);
+    }
+  }
+  if (gemv.empty()) return Q4_OK;
+  return from_cuda(launch_gemv_batch(gemv.data(), static_cast<int>(gemv.size()), cs, *dev), "q4_matmul_batch launch");
 }
 
 const char* q4_last_error(void) { return t_last_error; }

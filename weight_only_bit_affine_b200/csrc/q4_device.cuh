@@ -60,14 +60,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
+// As mbar_try_wait, but a thread whose phase is not complete is suspended
+// (not spinning, so it takes no issue slots from working warps) until the
+// phase completes or about `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises the device flag) if it has not completed within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       atomicOr(&g_device_flags, kFlagWaitTimeout);
       return false;
@@ -141,6 +151,28 @@ __device__ __forceinline__ void word_dot_bf16(uint32_t w, uint32_t x0, uint32_t 
       "fma.rn.f32.bf16 %0, xl2, l2, %0;\n\tfma.rn.f32.bf16 %1, xh2, h2, %1;\n\t"
       "fma.rn.f32.bf16 %0, xl3, l3, %0;\n\tfma.rn.f32.bf16 %1, xh3, h3, %1;\n\t}"
       : "+f"(c0), "+f"(c1)
+      : "r"(w), "r"(x0), "r"(x1), "r"(x2), "r"(x3));
+}
+
+// As word_dot_bf16, with all eight products into one accumulator.
+__device__ __forceinline__ void word_dot_bf16_acc(uint32_t w, uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3,
+                                                  float& c) {
+  asm("{\n\t.reg .b32 s1, s2, s3, v0, v1, v2, v3;\n\t"
+      ".reg .b16 l0, h0, l1, h1, l2, h2, l3, h3, xl0, xh0, xl1, xh1, xl2, xh2, xl3, xh3;\n\t"
+      "shr.b32 s1, %1, 4;\n\t"
+      "shr.b32 s2, %1, 8;\n\t"
+      "shr.b32 s3, %1, 12;\n\t"
+      "lop3.b32 v0, %1, 0x000F000F, 0x43004300, 0xEA;\n\t"
+      "lop3.b32 v1, s1, 0x000F000F, 0x43004300, 0xEA;\n\t"
+      "lop3.b32 v2, s2, 0x000F000F, 0x43004300, 0xEA;\n\t"
+      "lop3.b32 v3, s3, 0x000F000F, 0x43004300, 0xEA;\n\t"
+      "mov.b32 {l0, h0}, v0;\n\tmov.b32 {l1, h1}, v1;\n\tmov.b32 {l2, h2}, v2;\n\tmov.b32 {l3, h3}, v3;\n\t"
+      "mov.b32 {xl0, xh0}, %2;\n\tmov.b32 {xl1, xh1}, %3;\n\tmov.b32 {xl2, xh2}, %4;\n\tmov.b32 {xl3, xh3}, %5;\n\t"
+      "fma.rn.f32.bf16 %0, xl0, l0, %0;\n\tfma.rn.f32.bf16 %0, xh0, h0, %0;\n\t"
+      "fma.rn.f32.bf16 %0, xl1, l1, %0;\n\tfma.rn.f32.bf16 %0, xh1, h1, %0;\n\t"
+      "fma.rn.f32.bf16 %0, xl2, l2, %0;\n\tfma.rn.f32.bf16 %0, xh2, h2, %0;\n\t"
+      "fma.rn.f32.bf16 %0, xl3, l3, %0;\n\tfma.rn.f32.bf16 %0, xh3, h3, %0;\n\t}"
+      : "+f"(c)
       : "r"(w), "r"(x0), "r"(x1), "r"(x2), "r"(x3));
 }
 

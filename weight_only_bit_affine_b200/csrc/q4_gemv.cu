@@ -14,8 +14,9 @@
 //  * One persistent CTA per SM takes a balanced contiguous share of the rows
 //    of every problem in turn.  A producer warp streams those rows (codes,
 //    scales, biases: contiguous byte ranges) through a ring of shared-memory
-//    stages with 1-D bulk (TMA) copies, and each problem's activations into
-//    one of two shared-memory slots; the ring never drains between problems.
+//    stages with 1-D bulk (TMA) copies; each problem's activations travel
+//    through the same ring just ahead of its tiles, so the ring never drains
+//    between problems and the next problem's inputs arrive early.
 //  * Consumer threads form "teams" of K/32 lanes; a team owns one weight row
 //    at a time and lane j always covers input group j, so its slice of x sits
 //    in registers for the whole problem.  Each warp sums its lanes with a
@@ -37,7 +38,7 @@
 #include <vector>
 
 #ifndef Q4_GEMV_SMEM_BUDGET
-#define Q4_GEMV_SMEM_BUDGET (200 * 1024)
+#define Q4_GEMV_SMEM_BUDGET (227 * 1024)
 #endif
 #ifndef Q4_GEMV_MAC
 #define Q4_GEMV_MAC 0
@@ -137,8 +138,7 @@ __device__ __forceinline__ void dot_plus128(const uint32_t (&words)[WORDS], cons
       for (int m = 0; m < MR; ++m)
         word_dot_bf16(words[w], xs[m].v[w][0][0], xs[m].v[w][1][0], xs[m].v[w][2][0], xs[m].v[w][3][0], a0[m],
                       a1[m]);
-    return;
-  }
+  } else {
 #pragma unroll
   for (int w = 0; w < WORDS; ++w) {
 #pragma unroll
@@ -153,6 +153,7 @@ __device__ __forceinline__ void dot_plus128(const uint32_t (&words)[WORDS], cons
           ffma2(a0[m], a1[m], __uint_as_float(xs[m].v[w][t][0]), __uint_as_float(xs[m].v[w][t][1]), lo, hi);
       }
     }
+  }
   }
 }
 
@@ -203,7 +204,10 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float v) { return __bfloat16_as
 // (a small instance for single calls, a large one for batches).
 constexpr int kMaxProblems = 256;
 constexpr int kFewProblems = 4;
-constexpr int kRpt = 4;            // weight rows per team per tile
+#ifndef Q4_GEMV_RPT
+#define Q4_GEMV_RPT 4
+#endif
+constexpr int kRpt = Q4_GEMV_RPT;  // weight rows per team per tile
 
 struct GemvProblem {
   const uint16_t* x;       // [MR, K]
@@ -220,8 +224,7 @@ struct GemvLaunch {
   int count;
   int consumer_threads;  // a multiple of 32
   int stages;
-  uint32_t stage_bytes;  // >= every problem's tile, 128-byte multiple
-  uint32_t xslot_bytes;  // >= MR * K * 2 for every problem, 128-byte multiple
+  uint32_t stage_bytes;  // >= every problem's tile and activation block, 128-byte multiple
   uint32_t red_floats;   // per reduction buffer
   GemvProblem prob[NP];
 };
@@ -262,13 +265,10 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   const int warp = tid >> 5, lane = tid & 31;
   const int consumer_warps = L.consumer_threads >> 5;
 
-  uint8_t* xslots = smem + static_cast<size_t>(L.stages) * L.stage_bytes;
-  float* red = reinterpret_cast<float*>(xslots + 2 * static_cast<size_t>(L.xslot_bytes));
+  float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(L.stages) * L.stage_bytes);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(red + 2 * static_cast<size_t>(L.red_floats));
   uint64_t* empty_bar = full_bar + L.stages;
-  uint64_t* xfull_bar = empty_bar + L.stages;  // [2]
-  uint64_t* xempty_bar = xfull_bar + 2;        // [2]
-  uint64_t* rfull_bar = xempty_bar + 2;        // [2]
+  uint64_t* rfull_bar = empty_bar + L.stages;  // [2]
   uint64_t* rempty_bar = rfull_bar + 2;        // [2]
 
   if (tid == 0) {
@@ -277,8 +277,6 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       mbar_init(&empty_bar[s], consumer_warps);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&xfull_bar[s], 1);
-      mbar_init(&xempty_bar[s], consumer_warps);
       mbar_init(&rfull_bar[s], consumer_warps);
       mbar_init(&rempty_bar[s], 1);
     }
@@ -307,31 +305,32 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         }
       }
       pdl_wait_predecessors();
-      int stage = 0, xs = 0, issued = 0, xissued = 0;
-      uint32_t phase = 0, xphase = 0;
+      // Ring order per problem: its activation block [MR, K], then its tiles.
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
       bool dead = false;
       for (int pi = 0; pi < L.count && !dead; ++pi) {
         const GemvProblem& P = L.prob[pi];
         const Geometry geo = geometry_of(P.K, L.consumer_threads);
         const int half_k = P.K >> 1;
-        const uint32_t xbytes = static_cast<uint32_t>(MR) * P.K * 2;
-        if (!mbar_wait(&xempty_bar[xs], xphase ^ 1u)) { dead = true; break; }
-        mbar_arrive_expect_tx(&xfull_bar[xs], xbytes);
-        bulk_g2s(xslots + static_cast<size_t>(xs) * L.xslot_bytes, P.x, xbytes, &xfull_bar[xs]);
-        ++xissued;
-        if (++xs == 2) { xs = 0; xphase ^= 1u; }
         const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
-        for (int64_t row0 = r_begin; row0 < r_end; row0 += geo.rt) {
+        for (int64_t row0 = r_begin - geo.rt; row0 < r_end; row0 += geo.rt) {  // first pass: x
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; break; }
-          const uint32_t rows = tile_rows(r_end, row0, geo.rt);
-          const uint32_t cb = rows * half_k, sb = rows * geo.G * 2;
-          const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
-          const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
           uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
-          mbar_arrive_expect_tx(&full_bar[stage], cb + 2 * sb);
-          bulk_g2s(st, P.codes + row0 * half_k, cb, &full_bar[stage]);
-          bulk_g2s(st + sb_off, P.scales + row0 * geo.G, sb, &full_bar[stage]);
-          bulk_g2s(st + sb_off + sb_tile, P.biases + row0 * geo.G, sb, &full_bar[stage]);
+          if (row0 < r_begin) {
+            const uint32_t xbytes = static_cast<uint32_t>(MR) * P.K * 2;
+            mbar_arrive_expect_tx(&full_bar[stage], xbytes);
+            bulk_g2s(st, P.x, xbytes, &full_bar[stage]);
+          } else {
+            const uint32_t rows = tile_rows(r_end, row0, geo.rt);
+            const uint32_t cb = rows * half_k, sb = rows * geo.G * 2;
+            const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
+            const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
+            mbar_arrive_expect_tx(&full_bar[stage], cb + 2 * sb);
+            bulk_g2s(st, P.codes + row0 * half_k, cb, &full_bar[stage]);
+            bulk_g2s(st + sb_off, P.scales + row0 * geo.G, sb, &full_bar[stage]);
+            bulk_g2s(st + sb_off + sb_tile, P.biases + row0 * geo.G, sb, &full_bar[stage]);
+          }
           ++issued;
           if (++stage == L.stages) { stage = 0; phase ^= 1u; }
         }
@@ -342,12 +341,6 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         uint32_t ph = phase;
         if (s < 0) { s += L.stages; ph ^= 1u; }
         mbar_wait(&full_bar[s], ph);
-      }
-      for (int i = 0; i < min(xissued, 2); ++i) {
-        int s = xs - 1 - i;
-        uint32_t ph = xphase;
-        if (s < 0) { s += 2; ph ^= 1u; }
-        mbar_wait(&xfull_bar[s], ph);
       }
     }
     return;
@@ -382,8 +375,8 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   }
 
   // ---------------- consumer threads ----------------
-  int stage = 0, xs = 0, rb = 0;
-  uint32_t phase = 0, xphase = 0, rph = 0;
+  int stage = 0, rb = 0;
+  uint32_t phase = 0, rph = 0;
   bool dead = false;
   for (int pi = 0; pi < L.count; ++pi) {
     const GemvProblem& P = L.prob[pi];
@@ -396,12 +389,19 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
     const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
     const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
+    // Byte offsets inside a stage of this lane's first row (row team_idx) and
+    // the step to its next row (teams rows further).
+    const uint32_t code_off0 = static_cast<uint32_t>(team_idx) * half_k + j * 16;
+    const uint32_t code_step = static_cast<uint32_t>(geo.teams) * half_k;
+    const uint32_t sc_off0 = sb_off + (static_cast<uint32_t>(team_idx) * geo.G + j) * 2;
+    const uint32_t sc_step = static_cast<uint32_t>(geo.teams) * geo.G * 2;
 
-    // Activations: this lane's 32 inputs of each row, from the staged slot.
-    if (!dead && !mbar_wait(&xfull_bar[xs], xphase)) dead = true;
+    // Activations: this lane's 32 inputs of each row, from the ring stage
+    // that precedes the problem's tiles.
+    if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
     XSlice<4, Q4_GEMV_MAC> xsl[MR];
     {
-      const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(xslots + static_cast<size_t>(xs) * L.xslot_bytes);
+      const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(smem + static_cast<size_t>(stage) * L.stage_bytes);
 #pragma unroll
       for (int m = 0; m < MR; ++m) {
         if (active)
@@ -411,8 +411,8 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&xempty_bar[xs]);
-    if (++xs == 2) { xs = 0; xphase ^= 1u; }
+    if (lane == 0) mbar_arrive(&empty_bar[stage]);
+    if (++stage == L.stages) { stage = 0; phase ^= 1u; }
 
     const bool use_red = geo.wpt > 1;
     if (use_red && !dead && !mbar_wait(&rempty_bar[rb], rph ^ 1u)) dead = true;
@@ -422,68 +422,116 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     for (int64_t row0 = r_begin; row0 < r_end; row0 += geo.rt) {
       if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
       const uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
-      const uint16_t* ssc = reinterpret_cast<const uint16_t*>(st + sb_off);
-      const uint16_t* sbi = reinterpret_cast<const uint16_t*>(st + sb_off + sb_tile);
-      const int r_first = team_idx * kRpt;
-      const int64_t grow0 = row0 + r_first;
-
-      uint32_t words[kRpt][4];
-      float sc[kRpt], bi[kRpt];
-#pragma unroll
-      for (int rr = 0; rr < kRpt; ++rr) {  // all shared-memory loads first
-        const int r = r_first + rr;
-        if (active && grow0 + rr < r_end) {
-          load_words_smem<4>(st + static_cast<size_t>(r) * half_k + j * 16, words[rr]);
-          sc[rr] = bf16_bits_to_float(ssc[r * geo.G + j]);
-          bi[rr] = bf16_bits_to_float(sbi[r * geo.G + j]);
-        } else {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) words[rr][w] = 0u;
-          sc[rr] = bi[rr] = 0.f;
-        }
-      }
-      // The stage's bytes are in registers now: hand it back to the producer.
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[stage]);
-      if (++stage == L.stages) { stage = 0; phase ^= 1u; }
-
+      // Rows of this tile are dealt to the teams round-robin (row r goes to
+      // team r % teams), so a short last tile stays balanced; when a team
+      // spans whole warps the row count below is warp-uniform and idle warps
+      // skip the arithmetic entirely.
+      const int tile_n = static_cast<int>((r_end - row0 < geo.rt) ? (r_end - row0) : geo.rt);
+      const int nv = (team_idx < geo.teams && team_idx < tile_n) ? (tile_n - team_idx + geo.teams - 1) / geo.teams : 0;
       float vals[VP];
 #pragma unroll
       for (int i = 0; i < VP; ++i) vals[i] = 0.f;
+
+      if (geo.team >= 32 && nv == kRpt) {
+        // Fast path: every row of this team is present (warp-uniform).
+        // Lanes past G (padding) read in-stage bytes but take s = b = 0 and
+        // a zero x slice, so they add exactly nothing.
+        uint32_t words[kRpt][4];
+        float sc[kRpt], bi[kRpt];
+        const uint8_t* cp = st + code_off0;
+        const uint8_t* sp = st + sc_off0;
 #pragma unroll
-      for (int rr = 0; rr < kRpt; ++rr) {
-        float a0[MR], a1[MR];
+        for (int rr = 0; rr < kRpt; ++rr) {
+          load_words_smem<4>(cp + rr * code_step, words[rr]);
+          const uint16_t sh = *reinterpret_cast<const uint16_t*>(sp + rr * sc_step);
+          const uint16_t bh = *reinterpret_cast<const uint16_t*>(sp + rr * sc_step + sb_tile);
+          sc[rr] = active ? bf16_bits_to_float(sh) : 0.f;
+          bi[rr] = active ? bf16_bits_to_float(bh) : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[stage]);
+        if (++stage == L.stages) { stage = 0; phase ^= 1u; }
 #pragma unroll
-        for (int m = 0; m < MR; ++m) a0[m] = a1[m] = 0.f;
-        dot_plus128<MR, 4, Q4_GEMV_MAC>(words[rr], xsl, a0, a1);
-        const float c = fmaf(-kOffset, sc[rr], bi[rr]);
+        for (int rr = 0; rr < kRpt; ++rr) {
+          const float c = fmaf(-kOffset, sc[rr], bi[rr]);
 #pragma unroll
-        for (int m = 0; m < MR; ++m) vals[rr * MR + m] = fmaf(sc[rr], a0[m] + a1[m], c * xsl[m].sum);
+          for (int m = 0; m < MR; ++m) {
+            float a = 0.f;
+            if constexpr (Q4_GEMV_MAC == kMacMixedBf16) {
+#pragma unroll
+              for (int w = 0; w < 4; ++w)
+                word_dot_bf16_acc(words[rr][w], xsl[m].v[w][0][0], xsl[m].v[w][1][0], xsl[m].v[w][2][0],
+                                  xsl[m].v[w][3][0], a);
+            } else {
+              float a0[1] = {0.f}, a1[1] = {0.f};
+              dot_plus128<1, 4, Q4_GEMV_MAC>(words[rr], *reinterpret_cast<const XSlice<4, Q4_GEMV_MAC>(*)[1]>(&xsl[m]),
+                                             a0, a1);
+              a = a0[0] + a1[0];
+            }
+            vals[rr * MR + m] = fmaf(sc[rr], a, c * xsl[m].sum);
+          }
+        }
+      } else {
+        uint32_t words[kRpt][4];
+        float sc[kRpt], bi[kRpt];
+        const bool lane_on = active && nv > 0;
+#pragma unroll
+        for (int rr = 0; rr < kRpt; ++rr) {  // all shared-memory loads first
+          if (lane_on && rr < nv) {
+            load_words_smem<4>(st + code_off0 + rr * code_step, words[rr]);
+            sc[rr] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + sc_off0 + rr * sc_step));
+            bi[rr] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + sc_off0 + rr * sc_step + sb_tile));
+          } else {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) words[rr][w] = 0u;
+            sc[rr] = bi[rr] = 0.f;
+          }
+        }
+        // The stage's bytes are in registers now: hand it back to the producer.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[stage]);
+        if (++stage == L.stages) { stage = 0; phase ^= 1u; }
+
+        if (geo.team >= 32 && nv == 0) continue;  // a whole idle warp
+
+#pragma unroll
+        for (int rr = 0; rr < kRpt; ++rr) {
+          if (geo.team >= 32 && rr >= nv) break;  // warp-uniform
+          float a0[MR], a1[MR];
+#pragma unroll
+          for (int m = 0; m < MR; ++m) a0[m] = a1[m] = 0.f;
+          dot_plus128<MR, 4, Q4_GEMV_MAC>(words[rr], xsl, a0, a1);
+          const float c = fmaf(-kOffset, sc[rr], bi[rr]);
+#pragma unroll
+          for (int m = 0; m < MR; ++m) vals[rr * MR + m] = fmaf(sc[rr], a0[m] + a1[m], c * xsl[m].sum);
+        }
       }
 
       if (geo.team >= 32) {
         const float tot = transpose_reduce<VP>(vals, lane);
         const int idx = lane >> (5 - ilog2(VP));
-        const bool holder = (lane & ((32 / VP) - 1)) == 0 && idx < V && team_idx < geo.teams;
         const int rr = idx / MR, m = idx % MR;
-        if (holder && grow0 + rr < r_end) {
+        const bool holder = (lane & ((32 / VP) - 1)) == 0 && idx < V && rr < nv;
+        if (holder) {
+          const int64_t row = row0 + team_idx + rr * geo.teams;
           if (!use_red) {
-            P.y[static_cast<int64_t>(m) * P.y_ld + grow0 + rr] = to_bf16_bits(tot);
+            P.y[static_cast<int64_t>(m) * P.y_ld + row] = to_bf16_bits(tot);
           } else {
-            const int lr = static_cast<int>(grow0 + rr - r_begin);  // row within this CTA's share
+            const int lr = static_cast<int>(row - r_begin);  // row within this CTA's share
             rbuf[(lr * MR + m) * geo.wpt + warp_in_team] = tot;
           }
         }
       } else {
 #pragma unroll
         for (int i = 0; i < V; ++i) vals[i] = seg_allreduce_dyn(vals[i], geo.team);
-        if (j == 0 && team_idx < geo.teams) {
+        if (j == 0) {
 #pragma unroll
           for (int rr = 0; rr < kRpt; ++rr)
-            if (grow0 + rr < r_end) {
+            if (rr < nv) {
+              const int64_t row = row0 + team_idx + rr * geo.teams;
 #pragma unroll
               for (int m = 0; m < MR; ++m)
-                P.y[static_cast<int64_t>(m) * P.y_ld + grow0 + rr] = to_bf16_bits(vals[rr * MR + m]);
+                P.y[static_cast<int64_t>(m) * P.y_ld + row] = to_bf16_bits(vals[rr * MR + m]);
             }
         }
       }
@@ -602,31 +650,30 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   const int grid = dev.sm_count;
   static_assert(sizeof(GemvLaunch<NP>) <= 32000, "kernel parameters exceed the launch limit");
   thread_local GemvLaunch<NP> L;  // copied into the launch parameters by cudaLaunchKernelEx
-  uint32_t stage_bytes = 128, xslot = 128, red_floats = 1;
+  uint32_t stage_bytes = 128, red_floats = 1;
   for (int i = 0; i < count; ++i) {
     const GemvProblem& P = probs[i];
     const Geometry geo = geometry_of(P.K, consumers);
     const uint32_t tile = static_cast<uint32_t>(geo.rt) * (P.K / 2) +
                           2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
     stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
-    xslot = std::max(xslot, (static_cast<uint32_t>(MR) * P.K * 2 + 127u) & ~127u);
+    stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(MR) * P.K * 2 + 127u) & ~127u);
     if (geo.wpt > 1) {
       const int64_t rows = (P.N + grid - 1) / grid;
       red_floats = std::max<uint32_t>(red_floats, static_cast<uint32_t>(rows * MR * geo.wpt));
     }
   }
   red_floats = (red_floats + 31u) & ~31u;
-  const size_t fixed = 2 * static_cast<size_t>(xslot) + 2 * sizeof(float) * red_floats + 8 * 8;
+  const size_t fixed = 2 * sizeof(float) * red_floats + 4 * 8;
   const size_t budget = std::min<size_t>(Q4_GEMV_SMEM_BUDGET, dev.smem_optin);
   if (fixed + 2 * (stage_bytes + 16) > dev.smem_optin) return cudaErrorInvalidConfiguration;
   int stages = static_cast<int>((budget > fixed ? budget - fixed : 0) / (stage_bytes + 16));
-  stages = std::max(2, std::min(stages, 8));
+  stages = std::max(2, std::min(stages, 12));
   const size_t smem = static_cast<size_t>(stages) * stage_bytes + fixed + 16 * stages;
   L.count = count;
   L.consumer_threads = consumers;
   L.stages = stages;
   L.stage_bytes = stage_bytes;
-  L.xslot_bytes = xslot;
   L.red_floats = red_floats;
   for (int i = 0; i < count; ++i) L.prob[i] = probs[i];
   auto kern = gemv_kernel<MR, kThreads, NP>;

@@ -41,6 +41,11 @@ cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceIn
 // launch (per chunk size).
 cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
 
+// Tensor-core path (tcgen05) for many activation rows.
+constexpr int64_t kTensorCoreMinRows = 16;
+bool tc_supported(const MatmulArgs& a);
+cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev);
+
 // Counts every kernel launch libq4 enqueues (host side).
 void count_launch();
 
