@@ -173,6 +173,14 @@ def _traffic_per_launch(kernel_hash: str):
     return ent.get("dram_bytes_per_launch_avg")
 
 
+def _bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except (OSError, ValueError, KeyError):
+        return 1590.0
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -180,6 +188,135 @@ def _peaks():
         return float(d["hbm_gbs"]), "measured"
     except (OSError, ValueError, KeyError):
         return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------- other workloads
+
+
+def _graph_ms(dev, fn, reps):
+    """Capture fn() once in a CUDA graph; median-free mean of `reps` replays (CUDA events)."""
+    import torch
+
+    fn()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            fn()
+    torch.cuda.synchronize(dev)
+    st = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(st)
+    for _ in range(reps):
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / reps
+    del g
+    return ms
+
+
+def workload_rows(dev, packed, x, x_down, bf16_peak):
+    """The other workloads, as informational rows (not the metric).
+
+    temporal_layer: one layer's 7 projections at M = 1 (four different layers
+    rotate so the 514 MB exceed L2); depformer_steps: 16 codebook steps x 43
+    step-sliced projections of stacked weights (792 MB per frame); batched
+    layer at M = 4, 64, 256 (tensor cores from M = 16).
+    """
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    rows = {}
+    layer = [packed[i * 7:(i + 1) * 7] for i in range(4)]
+    lbytes = sum(c.numel() + 2 * s.numel() + 2 * b.numel() for _, c, s, b in layer[0])
+
+    def y_for(M, items):
+        return [torch.empty((M, p.N), dtype=torch.bfloat16, device=dev) for p, _, _, _ in items]
+
+    ys1 = [y_for(1, l) for l in layer]
+
+    def layer_batch():
+        for l, ys in zip(layer, ys1):
+            q4.q4_matmul_batch([(x_down if p.K == 11264 else x, c, s, b, y) for (p, c, s, b), y in zip(l, ys)])
+
+    ms = _graph_ms(dev, layer_batch, 50) / 4
+    rows["temporal_layer_M1"] = {"us_per_layer": round(ms * 1e3, 2), "GBps": round(lbytes / (ms * 1e-3) / 1e9, 1),
+                                 "launches_per_layer": 1, "bytes": lbytes}
+    per_proj = {}
+    for i, (p, c, s, b) in enumerate(layer[0]):
+        items = [l[i] for l in layer]
+        yy = [ys1[j][i] for j in range(4)]
+
+        def one(items=items, yy=yy):
+            for (pp, cc, ss, bb), y in zip(items, yy):
+                q4.q4_matmul(x_down if pp.K == 11264 else x, cc, ss, bb, out=y)
+
+        t = _graph_ms(dev, one, 100) / 4
+        nb = c.numel() + 2 * s.numel() + 2 * b.numel()
+        per_proj[p.name.split(".")[1]] = {"us": round(t * 1e3, 2), "GBps": round(nb / (t * 1e-3) / 1e9, 1)}
+    rows["temporal_layer_M1"]["per_projection_single_call"] = per_proj
+
+    # depformer: stacked [16 N, K] weights per projection, drawn and quantized on the GPU
+    seed = workloads.seed_of("depformer_steps")
+    steps = workloads.DEPFORMER_STEPS
+    dep = []
+    for t, p in enumerate(workloads.depformer_projs()):
+        W = workloads.weight(steps * p.N, p.K, seed, t, device=dev)
+        dep.append((p,) + tuple(q4.q4_quantize(W)))
+        del W
+    xd = {K: workloads.activation(1, K, seed, 500 + K, device=dev) for K in (1024, 2816)}
+    ysd = [torch.empty((1, p.N), dtype=torch.bfloat16, device=dev) for p, _, _, _ in dep]
+    fbytes = sum(c.numel() + 2 * s.numel() + 2 * b.numel() for _, c, s, b in dep)
+
+    def frame_step_calls():
+        for st in range(steps):
+            for (p, c, s, b), y in zip(dep, ysd):
+                q4.q4_matmul_step(xd[p.K], c, s, b, steps, st, out=y)
+
+    def frame_batched():
+        for st in range(steps):
+            sl = lambda t: t[st * (t.shape[0] // steps):(st + 1) * (t.shape[0] // steps)]
+            q4.q4_matmul_batch([(xd[p.K], sl(c), sl(s), sl(b), y) for (p, c, s, b), y in zip(dep, ysd)])
+
+    ms_calls = _graph_ms(dev, frame_step_calls, 10)
+    ms_batch = _graph_ms(dev, frame_batched, 20)
+    rows["depformer_steps_M1"] = {
+        "bytes_per_frame": fbytes,
+        "step_calls_us_per_step": round(ms_calls * 1e3 / steps, 2), "step_calls_ms_per_frame": round(ms_calls, 4),
+        "batched_us_per_step": round(ms_batch * 1e3 / steps, 2), "batched_ms_per_frame": round(ms_batch, 4),
+        "batched_GBps": round(fbytes / (ms_batch * 1e-3) / 1e9, 1),
+        "note": "43 step-sliced projections per codebook step; 'step_calls' = 43 q4_matmul_step launches per step, "
+                "'batched' = one q4_matmul_batch launch per step",
+    }
+    del dep
+
+    # batched layer for concurrent conversations / prefill
+    flops_layer = 2 * sum(p.N * p.K for p, _, _, _ in layer[0])
+    for M in workloads.BATCHED_M:
+        xb = workloads.activation(M, 4096, seed, 100 + M, device=dev)
+        xbd = workloads.activation(M, 11264, seed, 200 + M, device=dev)
+        ysm = [y_for(M, l) for l in layer]
+
+        def run_layers(xb=xb, xbd=xbd, ysm=ysm, M=M):
+            for l, ys in zip(layer, ysm):
+                for (p, c, s, b), y in zip(l, ys):
+                    q4.q4_matmul(xbd if p.K == 11264 else xb, c, s, b, out=y)
+
+        t = _graph_ms(dev, run_layers, 20) / 4
+        tf = flops_layer * M / (t * 1e-3) / 1e12
+        rows[f"batched_layer_M{M}"] = {
+            "us_per_layer": round(t * 1e3, 2), "TFLOPs": round(tf, 1),
+            "frac_of_bf16_peak": round(tf / bf16_peak, 4), "packed_GBps": round(lbytes / (t * 1e-3) / 1e9, 1),
+            "path": "tcgen05 tensor cores" if M >= 16 else "CUDA-core GEMV (activation rows in pairs)",
+        }
+    return rows
 
 
 # --------------------------------------------------------------------- CPU oracle
@@ -407,6 +544,10 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms, ms_e2e = float(t[0]), float(t[1])
 
+    extra = {}
+    if not args.no_rows:
+        extra = workload_rows(dev, packed, x, x_down, _bf16_peak())
+
     flags = q4.q4_debug_device_flags()
     peak, peak_kind = _peaks()
     kh = _kernel_source_hash()
@@ -455,6 +596,7 @@ def run_ours(args):
             "stream_GBps_225_calls_graph": round(nbytes / (ms_calls_graph * 1e-3) / 1e9, 1),
             "stream_ms_225_calls_plain": round(ms_plain, 4),
             "per_shape_single_call_events": shapes,
+            **extra,
         },
         "device_flags": flags,
     }
@@ -478,6 +620,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the informational rows of the other workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

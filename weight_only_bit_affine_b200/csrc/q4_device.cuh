@@ -70,14 +70,25 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
   return ok != 0;
 }
+#ifndef Q4_WAIT_SLEEP_NS
+#define Q4_WAIT_SLEEP_NS 20000u
+#endif
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises the device flag) if it has not completed within kWaitLimitNs.
+// kSleep selects the suspend-hinted form (for waits that are usually long,
+// so the waiting warp leaves its issue slots to the others).
+template <bool kSleep = true>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    for (int i = 0; i < 16; ++i)
-      if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    for (int i = 0; i < 16; ++i) {
+      if constexpr (kSleep) {
+        if (mbar_try_wait_sleep(bar, parity, Q4_WAIT_SLEEP_NS)) return true;
+      } else {
+        if (mbar_try_wait(bar, parity)) return true;
+      }
+    }
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       atomicOr(&g_device_flags, kFlagWaitTimeout);
       return false;

@@ -38,6 +38,10 @@
 #include <algorithm>
 #include <mutex>
 
+#ifndef Q4_TC_WAIT_SLEEP
+#define Q4_TC_WAIT_SLEEP 0
+#endif
+
 namespace q4 {
 namespace {
 
@@ -117,11 +121,15 @@ __device__ __forceinline__ void tc_ld_x8(uint32_t taddr, float (&v)[8]) {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t local_addr, uint32_t rank) {
   uint32_t remote;
-  float v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  return remote;
+}
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t remote_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(remote_addr));
   return v;
 }
 
@@ -193,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % p.stages;
         const uint32_t ph = static_cast<uint32_t>(c / p.stages) & 1u;
-        if (!dead && !mbar_wait(&stage_free[s], ph ^ 1u)) dead = true;
+        if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&stage_free[s], ph ^ 1u)) dead = true;
         const int k0 = (chunk_begin + c) * kChunkK;
         mbar_arrive_expect_tx(&tma_full[s], p.b_tile_bytes + kCodeTileBytes);
         tma_load_2d(b_tile(s), &tmap_x, k0, static_cast<int>(m0), &tma_full[s]);
@@ -207,8 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % p.stages;
         const uint32_t ph = static_cast<uint32_t>(c / p.stages) & 1u;
-        if (!dead && !mbar_wait(&tma_full[s], ph)) dead = true;
-        if (!dead && !mbar_wait(&a_full[s], ph)) dead = true;
+        if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&tma_full[s], ph)) dead = true;
+        if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&a_full[s], ph)) dead = true;
         tc_fence_after();
         const uint64_t ad = sw128_desc(smem_u32(a_tile(s)));
         const uint64_t bd = sw128_desc(smem_u32(b_tile(s)));
@@ -260,8 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t s2 = __byte_perm(sw, 0, sel);
       const uint32_t b2 = __byte_perm(bw, 0, sel);
 
-      if (!dead && !mbar_wait(&stage_free[s], ph ^ 1u)) dead = true;  // A buffer no longer read
-      if (!dead && !mbar_wait(&tma_full[s], ph)) dead = true;         // codes arrived
+      if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&stage_free[s], ph ^ 1u)) dead = true;  // A buffer no longer read
+      if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&tma_full[s], ph)) dead = true;         // codes arrived
       const uint4 cw = *reinterpret_cast<const uint4*>(c_tile(s) + row * 32 + half * 16);
       const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
       uint8_t* arow = a_tile(s) + row * 128;
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cols = p.bn / 2;
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lane_base) << 16) + col_half * cols;
     float* red = reinterpret_cast<float*>(smem);  // reuses the stage area (all MMAs are done)
-    const int red_ld = p.bn + 1;
+    const int red_ld = p.bn + 4;                  // 16-byte rows; row r and r + 1 four banks apart
     for (int c0 = 0; c0 < cols; c0 += 8) {
       float v[8];
       tc_ld_x8(taddr + c0, v);
@@ -305,8 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
         }
       } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) red[trow * red_ld + col_half * cols + c0 + i] = v[i];
+        float4* dst = reinterpret_cast<float4*>(red + trow * red_ld + col_half * cols + c0);
+        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
       }
     }
   }
@@ -318,15 +327,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp >= 2) {
       const int t = tid - 64;
       const int trow = t & (kTileN - 1);
-      const int cbeg = split * p.bn / p.splits, cend = (split + 1) * p.bn / p.splits;
-      const uint32_t red_base = smem_u32(smem);
-      const int red_ld = p.bn + 1;
-      for (int col = cbeg + (t >> 7); col < cend; col += 2) {
-        float acc = 0.f;
-        for (int r = 0; r < p.splits; ++r)
-          acc += ld_dsmem_f32(red_base + static_cast<uint32_t>(trow * red_ld + col) * 4u, static_cast<uint32_t>(r));
-        const int64_t m = m0 + col;
-        if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+      // Column slice of this CTA, in float4 units (bn and the slice are multiples of 4).
+      const int q_beg = split * (p.bn / 4) / p.splits, q_end = (split + 1) * (p.bn / 4) / p.splits;
+      const uint32_t row_addr = smem_u32(smem) + static_cast<uint32_t>(trow * (p.bn + 4)) * 4u;
+      uint32_t peer[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) peer[r] = dsmem_map(row_addr, static_cast<uint32_t>(r < p.splits ? r : 0));
+      for (int q = q_beg + (t >> 7); q < q_end; q += 2) {
+        // all peers' loads first, then the sums
+        float4 v[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          if (r < p.splits) v[r] = ld_dsmem_v4(peer[r] + static_cast<uint32_t>(q) * 16u);
+        float4 acc = v[0];
+#pragma unroll
+        for (int r = 1; r < 8; ++r)
+          if (r < p.splits) {
+            acc.x += v[r].x;
+            acc.y += v[r].y;
+            acc.z += v[r].z;
+            acc.w += v[r].w;
+          }
+        const float out[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int64_t m = m0 + 4 * q + i;
+          if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
+        }
       }
     }
     cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
@@ -424,7 +451,7 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
   p.splits = splits;
   p.b_tile_bytes = static_cast<uint32_t>(bn) * kChunkK * 2;
   p.stage_bytes = (kATileBytes + p.b_tile_bytes + kCodeTileBytes + 1023u) & ~1023u;
-  const size_t red_bytes = static_cast<size_t>(kTileN) * (bn + 1) * 4;
+  const size_t red_bytes = static_cast<size_t>(kTileN) * (bn + 4) * 4;
   const size_t barrier_bytes = 8 * (3 * 8 + 1) + 16;
   const size_t avail = dev.smem_optin - 1024 - barrier_bytes;
   p.stages = static_cast<int>(std::min<size_t>(6, avail / p.stage_bytes));
