@@ -216,6 +216,7 @@ struct GemvProblem {
   const uint16_t* biases;  // [N, K/32]
   uint16_t* y;             // [MR, y_ld]
   int64_t N, y_ld;
+  int64_t byte_begin;      // packed bytes of all earlier problems in the list
   int32_t K, pad_;
 };
 
@@ -225,9 +226,12 @@ struct GemvLaunch {
   int consumer_threads;  // a multiple of 32
   int stages;
   uint32_t stage_bytes;  // >= every problem's tile and activation block, 128-byte multiple
-  uint32_t red_floats;   // per reduction buffer
+  int64_t total_bytes;   // packed bytes of the whole list
   GemvProblem prob[NP];
 };
+
+constexpr int kRedSlots = 8;    // tiles of cross-warp partial sums in flight to the epilogue warp
+constexpr int kRedSlotFloats = 64 * 2;  // >= rt * MR * warps-per-team (rt * wpt <= 4 * 16)
 
 // Shape of one problem for a given consumer count (host and device agree).
 struct Geometry {
@@ -251,9 +255,35 @@ __host__ __device__ inline Geometry geometry_of(int K, int consumer_threads) {
   g.rt = g.teams * kRpt;
   return g;
 }
+__host__ __device__ inline int64_t packed_row_bytes(int K) { return K / 2 + (K / 32) * 4; }
 
 __device__ __forceinline__ uint32_t tile_rows(int64_t r_end, int64_t row0, int rt) {
   return static_cast<uint32_t>((r_end - row0 < rt) ? (r_end - row0) : rt);
+}
+
+// The rows of problem `pi` that belong to this CTA's byte range [lo, hi) of
+// the concatenated list: [*r0, *r1).  A row belongs to the CTA whose range
+// holds its first packed byte, with segment boundaries rounded up to whole
+// tiles of the problem, so every row has the same place in its tile however
+// the list is split (results do not depend on batching) and each row of the
+// list belongs to exactly one CTA.  Returns false when the problem lies
+// entirely after the range (the caller stops scanning).
+template <int NP>
+__device__ __forceinline__ bool segment_of(const GemvLaunch<NP>& L, int pi, int64_t lo, int64_t hi, int64_t* r0,
+                                           int64_t* r1) {
+  const GemvProblem& P = L.prob[pi];
+  const int64_t rb = packed_row_bytes(P.K);
+  const int64_t pb = P.byte_begin, pe = pb + P.N * rb;
+  *r0 = *r1 = 0;
+  if (pb >= hi) return false;
+  if (pe <= lo) return true;
+  const int64_t rt = geometry_of(P.K, L.consumer_threads).rt;
+  const int64_t a = (lo > pb ? lo : pb) - pb, b = (hi < pe ? hi : pe) - pb;
+  *r0 = ((a + rb - 1) / rb + rt - 1) / rt * rt;
+  *r1 = ((b + rb - 1) / rb + rt - 1) / rt * rt;
+  if (*r0 > P.N) *r0 = P.N;
+  if (*r1 > P.N) *r1 = P.N;
+  return true;
 }
 
 template <int MR, int MAXT, int NP>
@@ -266,17 +296,17 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   const int consumer_warps = L.consumer_threads >> 5;
 
   float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(L.stages) * L.stage_bytes);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(red + 2 * static_cast<size_t>(L.red_floats));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(red + kRedSlots * kRedSlotFloats);
   uint64_t* empty_bar = full_bar + L.stages;
-  uint64_t* rfull_bar = empty_bar + L.stages;  // [2]
-  uint64_t* rempty_bar = rfull_bar + 2;        // [2]
+  uint64_t* rfull_bar = empty_bar + L.stages;   // [kRedSlots]
+  uint64_t* rempty_bar = rfull_bar + kRedSlots;  // [kRedSlots]
 
   if (tid == 0) {
     for (int s = 0; s < L.stages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], consumer_warps);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kRedSlots; ++s) {
       mbar_init(&rfull_bar[s], consumer_warps);
       mbar_init(&rempty_bar[s], 1);
     }
@@ -285,44 +315,50 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   __syncthreads();
   pdl_launch_dependents();
 
-  const int64_t cta = blockIdx.x, grid = gridDim.x;
+  // This CTA's share of the list: a contiguous, balanced range of packed bytes.
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * L.total_bytes / gridDim.x;
+  const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * L.total_bytes / gridDim.x;
 
   if (warp == consumer_warps) {
     // ---------------- producer warp ----------------
     if (lane == 0) {
-      {  // warm L2 with the first problem's first tiles (a hint; changes no value)
-        const GemvProblem& P = L.prob[0];
-        const Geometry geo = geometry_of(P.K, L.consumer_threads);
-        const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
-        const int half_k = P.K >> 1;
-        for (int i = 0; i < L.stages; ++i) {
-          const int64_t row0 = r_begin + static_cast<int64_t>(i) * geo.rt;
-          if (row0 >= r_end) break;
-          const uint32_t rows = tile_rows(r_end, row0, geo.rt);
-          bulk_prefetch_l2(P.codes + row0 * half_k, rows * half_k);
-          bulk_prefetch_l2(P.scales + row0 * geo.G, rows * geo.G * 2);
-          bulk_prefetch_l2(P.biases + row0 * geo.G, rows * geo.G * 2);
+      {  // warm L2 with the first tiles of the range (a hint; changes no value)
+        int64_t r0, r1;
+        int issued = 0;
+        for (int pi = 0; pi < L.count && issued < L.stages; ++pi) {
+          if (!segment_of(L, pi, lo, hi, &r0, &r1)) break;
+          const GemvProblem& P = L.prob[pi];
+          const Geometry geo = geometry_of(P.K, L.consumer_threads);
+          const int half_k = P.K >> 1;
+          for (int64_t row0 = r0; row0 < r1 && issued < L.stages; row0 += geo.rt, ++issued) {
+            const uint32_t rows = tile_rows(r1, row0, geo.rt);
+            bulk_prefetch_l2(P.codes + row0 * half_k, rows * half_k);
+            bulk_prefetch_l2(P.scales + row0 * geo.G, rows * geo.G * 2);
+            bulk_prefetch_l2(P.biases + row0 * geo.G, rows * geo.G * 2);
+          }
         }
       }
       pdl_wait_predecessors();
-      // Ring order per problem: its activation block [MR, K], then its tiles.
+      // Ring order per segment: its activation block [MR, K], then its tiles.
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool dead = false;
       for (int pi = 0; pi < L.count && !dead; ++pi) {
+        int64_t r0, r1;
+        if (!segment_of(L, pi, lo, hi, &r0, &r1)) break;
+        if (r0 >= r1) continue;
         const GemvProblem& P = L.prob[pi];
         const Geometry geo = geometry_of(P.K, L.consumer_threads);
         const int half_k = P.K >> 1;
-        const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
-        for (int64_t row0 = r_begin - geo.rt; row0 < r_end; row0 += geo.rt) {  // first pass: x
+        for (int64_t row0 = r0 - geo.rt; row0 < r1; row0 += geo.rt) {  // first pass: x
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; break; }
           uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
-          if (row0 < r_begin) {
+          if (row0 < r0) {
             const uint32_t xbytes = static_cast<uint32_t>(MR) * P.K * 2;
             mbar_arrive_expect_tx(&full_bar[stage], xbytes);
             bulk_g2s(st, P.x, xbytes, &full_bar[stage]);
           } else {
-            const uint32_t rows = tile_rows(r_end, row0, geo.rt);
+            const uint32_t rows = tile_rows(r1, row0, geo.rt);
             const uint32_t cb = rows * half_k, sb = rows * geo.G * 2;
             const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
             const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
@@ -349,36 +385,50 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   pdl_wait_predecessors();  // consumers and epilogue read x and write y
 
   if (warp == consumer_warps + 1) {
-    // ---------------- epilogue warp: sums across a team's warps ----------------
-    int rb = 0;
-    uint32_t rph = 0;
+    // ---------------- epilogue warp: sums across a team's warps, per tile ----------------
+    int slot = 0;
+    uint32_t sph = 0;
     bool dead = false;
     for (int pi = 0; pi < L.count; ++pi) {
+      int64_t r0, r1;
+      if (!segment_of(L, pi, lo, hi, &r0, &r1)) break;
       const GemvProblem& P = L.prob[pi];
       const Geometry geo = geometry_of(P.K, L.consumer_threads);
       if (geo.wpt <= 1) continue;
-      if (!dead && !mbar_wait(&rfull_bar[rb], rph)) dead = true;
-      const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
-      const int n_out = static_cast<int>(r_end - r_begin) * MR;
-      const float* rbuf = red + static_cast<size_t>(rb) * L.red_floats;
-      for (int i = lane; i < n_out; i += 32) {
-        float v = 0.f;
-        for (int w = 0; w < geo.wpt; ++w) v += rbuf[i * geo.wpt + w];
-        const int lr = i / MR, m = i - lr * MR;
-        P.y[static_cast<int64_t>(m) * P.y_ld + r_begin + lr] = to_bf16_bits(v);
+      for (int64_t row0 = r0; row0 < r1; row0 += geo.rt) {
+        if (!dead && !mbar_wait(&rfull_bar[slot], sph)) dead = true;
+        const int n_out = static_cast<int>(tile_rows(r1, row0, geo.rt)) * MR;
+        const float* rs = red + slot * kRedSlotFloats;
+        if (lane < n_out) {
+          float v = 0.f;
+          for (int w = 0; w < geo.wpt; ++w) v += rs[lane * geo.wpt + w];
+          const int lr = lane / MR, m = lane - lr * MR;
+          P.y[static_cast<int64_t>(m) * P.y_ld + row0 + lr] = to_bf16_bits(v);
+        }
+        if (n_out > 32) {  // MR * rt rows beyond one per lane
+          for (int i = lane + 32; i < n_out; i += 32) {
+            float v = 0.f;
+            for (int w = 0; w < geo.wpt; ++w) v += rs[i * geo.wpt + w];
+            const int lr = i / MR, m = i - lr * MR;
+            P.y[static_cast<int64_t>(m) * P.y_ld + row0 + lr] = to_bf16_bits(v);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rempty_bar[slot]);
+        if (++slot == kRedSlots) { slot = 0; sph ^= 1u; }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&rempty_bar[rb]);
-      if (++rb == 2) { rb = 0; rph ^= 1u; }
     }
     return;
   }
 
   // ---------------- consumer threads ----------------
-  int stage = 0, rb = 0;
-  uint32_t phase = 0, rph = 0;
+  int stage = 0, slot = 0;
+  uint32_t phase = 0, sph = 0;
   bool dead = false;
   for (int pi = 0; pi < L.count; ++pi) {
+    int64_t r_begin, r_end;
+    if (!segment_of(L, pi, lo, hi, &r_begin, &r_end)) break;
+    if (r_begin >= r_end) continue;
     const GemvProblem& P = L.prob[pi];
     const Geometry geo = geometry_of(P.K, L.consumer_threads);
     const int half_k = P.K >> 1;
@@ -386,7 +436,6 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     const int j = tid - team_idx * geo.team;
     const bool active = team_idx < geo.teams && j < geo.G;
     const int warp_in_team = (geo.team >= 32) ? (j >> 5) : 0;
-    const int64_t r_begin = cta * P.N / grid, r_end = (cta + 1) * P.N / grid;
     const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
     const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
     // Byte offsets inside a stage of this lane's first row (row team_idx) and
@@ -397,7 +446,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     const uint32_t sc_step = static_cast<uint32_t>(geo.teams) * geo.G * 2;
 
     // Activations: this lane's 32 inputs of each row, from the ring stage
-    // that precedes the problem's tiles.
+    // that precedes the segment's tiles.
     if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
     XSlice<4, Q4_GEMV_MAC> xsl[MR];
     {
@@ -415,8 +464,6 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     if (++stage == L.stages) { stage = 0; phase ^= 1u; }
 
     const bool use_red = geo.wpt > 1;
-    if (use_red && !dead && !mbar_wait(&rempty_bar[rb], rph ^ 1u)) dead = true;
-    float* rbuf = red + static_cast<size_t>(rb) * L.red_floats;
     constexpr float kOffset = mac_offset<Q4_GEMV_MAC>();
 
     for (int64_t row0 = r_begin; row0 < r_end; row0 += geo.rt) {
@@ -427,10 +474,13 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       // spans whole warps the row count below is warp-uniform and idle warps
       // skip the arithmetic entirely.
       const int tile_n = static_cast<int>((r_end - row0 < geo.rt) ? (r_end - row0) : geo.rt);
-      const int nv = (team_idx < geo.teams && team_idx < tile_n) ? (tile_n - team_idx + geo.teams - 1) / geo.teams : 0;
+      const int nv = (team_idx >= geo.teams || team_idx >= tile_n) ? 0
+                     : (tile_n == geo.rt)                          ? kRpt
+                                                                   : (tile_n - team_idx + geo.teams - 1) / geo.teams;
       float vals[VP];
 #pragma unroll
       for (int i = 0; i < VP; ++i) vals[i] = 0.f;
+      bool compute = true;
 
       if (geo.team >= 32 && nv == kRpt) {
         // Fast path: every row of this team is present (warp-uniform).
@@ -456,19 +506,19 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
           const float c = fmaf(-kOffset, sc[rr], bi[rr]);
 #pragma unroll
           for (int m = 0; m < MR; ++m) {
-            float a = 0.f;
+            float acc = 0.f;
             if constexpr (Q4_GEMV_MAC == kMacMixedBf16) {
 #pragma unroll
               for (int w = 0; w < 4; ++w)
                 word_dot_bf16_acc(words[rr][w], xsl[m].v[w][0][0], xsl[m].v[w][1][0], xsl[m].v[w][2][0],
-                                  xsl[m].v[w][3][0], a);
+                                  xsl[m].v[w][3][0], acc);
             } else {
               float a0[1] = {0.f}, a1[1] = {0.f};
               dot_plus128<1, 4, Q4_GEMV_MAC>(words[rr], *reinterpret_cast<const XSlice<4, Q4_GEMV_MAC>(*)[1]>(&xsl[m]),
                                              a0, a1);
-              a = a0[0] + a1[0];
+              acc = a0[0] + a1[0];
             }
-            vals[rr * MR + m] = fmaf(sc[rr], a, c * xsl[m].sum);
+            vals[rr * MR + m] = fmaf(sc[rr], acc, c * xsl[m].sum);
           }
         }
       } else {
@@ -492,34 +542,44 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         if (lane == 0) mbar_arrive(&empty_bar[stage]);
         if (++stage == L.stages) { stage = 0; phase ^= 1u; }
 
-        if (geo.team >= 32 && nv == 0) continue;  // a whole idle warp
-
+        if (geo.team >= 32 && nv == 0) {
+          compute = false;  // a whole idle warp
+        } else {
 #pragma unroll
-        for (int rr = 0; rr < kRpt; ++rr) {
-          if (geo.team >= 32 && rr >= nv) break;  // warp-uniform
-          float a0[MR], a1[MR];
+          for (int rr = 0; rr < kRpt; ++rr) {
+            if (geo.team >= 32 && rr >= nv) break;  // warp-uniform
+            float a0[MR], a1[MR];
 #pragma unroll
-          for (int m = 0; m < MR; ++m) a0[m] = a1[m] = 0.f;
-          dot_plus128<MR, 4, Q4_GEMV_MAC>(words[rr], xsl, a0, a1);
-          const float c = fmaf(-kOffset, sc[rr], bi[rr]);
+            for (int m = 0; m < MR; ++m) a0[m] = a1[m] = 0.f;
+            dot_plus128<MR, 4, Q4_GEMV_MAC>(words[rr], xsl, a0, a1);
+            const float c = fmaf(-kOffset, sc[rr], bi[rr]);
 #pragma unroll
-          for (int m = 0; m < MR; ++m) vals[rr * MR + m] = fmaf(sc[rr], a0[m] + a1[m], c * xsl[m].sum);
+            for (int m = 0; m < MR; ++m) vals[rr * MR + m] = fmaf(sc[rr], a0[m] + a1[m], c * xsl[m].sum);
+          }
         }
       }
 
       if (geo.team >= 32) {
-        const float tot = transpose_reduce<VP>(vals, lane);
-        const int idx = lane >> (5 - ilog2(VP));
-        const int rr = idx / MR, m = idx % MR;
-        const bool holder = (lane & ((32 / VP) - 1)) == 0 && idx < V && rr < nv;
-        if (holder) {
-          const int64_t row = row0 + team_idx + rr * geo.teams;
-          if (!use_red) {
-            P.y[static_cast<int64_t>(m) * P.y_ld + row] = to_bf16_bits(tot);
-          } else {
-            const int lr = static_cast<int>(row - r_begin);  // row within this CTA's share
-            rbuf[(lr * MR + m) * geo.wpt + warp_in_team] = tot;
+        float* rs = red + slot * kRedSlotFloats;
+        if (use_red && !dead && !mbar_wait(&rempty_bar[slot], sph ^ 1u)) dead = true;
+        if (compute) {
+          const float tot = transpose_reduce<VP>(vals, lane);
+          const int idx = lane >> (5 - ilog2(VP));
+          const int rr = idx / MR, m = idx % MR;
+          const bool holder = (lane & ((32 / VP) - 1)) == 0 && idx < V && rr < nv;
+          if (holder) {
+            const int lr = team_idx + rr * geo.teams;  // row within the tile
+            if (!use_red) {
+              P.y[static_cast<int64_t>(m) * P.y_ld + row0 + lr] = to_bf16_bits(tot);
+            } else {
+              rs[(lr * MR + m) * geo.wpt + warp_in_team] = tot;
+            }
           }
+        }
+        if (use_red) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&rfull_bar[slot]);
+          if (++slot == kRedSlots) { slot = 0; sph ^= 1u; }
         }
       } else {
 #pragma unroll
@@ -535,11 +595,6 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
             }
         }
       }
-    }
-    if (use_red) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&rfull_bar[rb]);
-      if (++rb == 2) { rb = 0; rph ^= 1u; }
     }
   }
 }
@@ -641,16 +696,16 @@ cudaError_t run_generic(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, 
   return launch_pdl(gemv_generic_kernel<MR>, dim3(grid), dim3(256), 0, stream, p);
 }
 
-// Launches the bulk-copy kernel over problems [first, last) of `probs`
-// (all taking this path, all with MR activation rows).
+// Launches the bulk-copy kernel over `count` problems of `probs` (all taking
+// this path, all with MR activation rows).
 template <int MR, int NP>
 cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev, cudaStream_t stream) {
   constexpr int kThreads = MR == 1 ? kThreads1 : kThreads2;
   const int consumers = consumers_for(MR);
-  const int grid = dev.sm_count;
   static_assert(sizeof(GemvLaunch<NP>) <= 32000, "kernel parameters exceed the launch limit");
   thread_local GemvLaunch<NP> L;  // copied into the launch parameters by cudaLaunchKernelEx
-  uint32_t stage_bytes = 128, red_floats = 1;
+  uint32_t stage_bytes = 128;
+  int64_t total = 0;
   for (int i = 0; i < count; ++i) {
     const GemvProblem& P = probs[i];
     const Geometry geo = geometry_of(P.K, consumers);
@@ -658,24 +713,24 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
                           2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
     stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
     stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(MR) * P.K * 2 + 127u) & ~127u);
-    if (geo.wpt > 1) {
-      const int64_t rows = (P.N + grid - 1) / grid;
-      red_floats = std::max<uint32_t>(red_floats, static_cast<uint32_t>(rows * MR * geo.wpt));
-    }
+    L.prob[i] = P;
+    L.prob[i].byte_begin = total;
+    total += P.N * packed_row_bytes(P.K);
   }
-  red_floats = (red_floats + 31u) & ~31u;
-  const size_t fixed = 2 * sizeof(float) * red_floats + 4 * 8;
+  const size_t fixed = sizeof(float) * kRedSlots * kRedSlotFloats + 16 * kRedSlots;
   const size_t budget = std::min<size_t>(Q4_GEMV_SMEM_BUDGET, dev.smem_optin);
   if (fixed + 2 * (stage_bytes + 16) > dev.smem_optin) return cudaErrorInvalidConfiguration;
-  int stages = static_cast<int>((budget > fixed ? budget - fixed : 0) / (stage_bytes + 16));
+  int stages = static_cast<int>((budget - fixed) / (stage_bytes + 16));
   stages = std::max(2, std::min(stages, 12));
   const size_t smem = static_cast<size_t>(stages) * stage_bytes + fixed + 16 * stages;
   L.count = count;
   L.consumer_threads = consumers;
   L.stages = stages;
   L.stage_bytes = stage_bytes;
-  L.red_floats = red_floats;
-  for (int i = 0; i < count; ++i) L.prob[i] = probs[i];
+  L.total_bytes = total;
+  // Enough CTAs that every one has work; one per SM.
+  const int64_t rows = [&] { int64_t r = 0; for (int i = 0; i < count; ++i) r += probs[i].N; return r; }();
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, rows)));
   auto kern = gemv_kernel<MR, kThreads, NP>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -686,31 +741,13 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, L);
 }
 
-// Splits problems whose per-CTA reduction buffer would be too large into row
-// ranges, then launches in groups of at most kMaxProblems.
+// Launches in groups of at most kMaxProblems problems.
 template <int MR>
 cudaError_t run_problems(std::vector<GemvProblem>& probs, const DeviceInfo& dev, cudaStream_t stream) {
-  const int consumers = consumers_for(MR);
-  std::vector<GemvProblem> split;
-  split.reserve(probs.size());
-  for (const GemvProblem& P : probs) {
-    const Geometry geo = geometry_of(P.K, consumers);
-    const int64_t max_rows_per_cta = geo.wpt > 1 ? std::max<int64_t>(1, 2048 / (MR * geo.wpt)) : INT64_MAX / 4;
-    const int64_t max_rows = max_rows_per_cta * dev.sm_count;
-    for (int64_t r = 0; r < P.N; r += max_rows) {
-      GemvProblem Q = P;
-      Q.N = std::min<int64_t>(max_rows, P.N - r);
-      Q.codes = P.codes + r * (P.K / 2);
-      Q.scales = P.scales + r * (P.K / 32);
-      Q.biases = P.biases + r * (P.K / 32);
-      Q.y = P.y + r;
-      split.push_back(Q);
-    }
-  }
-  for (size_t i = 0; i < split.size(); i += kMaxProblems) {
-    const int n = static_cast<int>(std::min<size_t>(kMaxProblems, split.size() - i));
-    cudaError_t e = (n <= kFewProblems) ? run_list<MR, kFewProblems>(split.data() + i, n, dev, stream)
-                                        : run_list<MR, kMaxProblems>(split.data() + i, n, dev, stream);
+  for (size_t i = 0; i < probs.size(); i += kMaxProblems) {
+    const int n = static_cast<int>(std::min<size_t>(kMaxProblems, probs.size() - i));
+    cudaError_t e = (n <= kFewProblems) ? run_list<MR, kFewProblems>(probs.data() + i, n, dev, stream)
+                                        : run_list<MR, kMaxProblems>(probs.data() + i, n, dev, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -750,6 +787,7 @@ cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t st
       P.y_ld = a.N;
       P.K = static_cast<int32_t>(a.K);
       P.pad_ = 0;
+      P.byte_begin = 0;
       (mr == 1 ? one : two).push_back(P);
     }
   }

@@ -1,0 +1,105 @@
+"""Small, named workloads for profiling libq4 under ncu.
+
+    python -m weight_only_bit_affine_b200.profile_case <case> [reps]
+
+Cases (seeded synthetic inputs of the workload shapes; each rep runs the
+whole case once, after one warm-up rep):
+
+  stream_small   3 temporal layers + the text head (553 MB packed) as one
+                 q4_matmul_batch per rep: the benchmark's kernel on a case
+                 small enough for a full ncu capture.
+  tc_layer       one temporal layer (7 projections, 128 MB) through q4_matmul
+                 at M = 64 and then M = 256: the tensor-core kernel.
+  depformer_step one depformer codebook step (43 step-sliced projections) as
+                 one q4_matmul_batch.
+
+Every case checks the library's bounded-wait flag at the end.
+"""
+from __future__ import annotations
+
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def _stream_small(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    projs = workloads.stream_projs()
+    sel = [(t, p) for t, p in enumerate(projs) if p.name.startswith(("L0.", "L1.", "L2."))] + [(len(projs) - 1, projs[-1])]
+    seed = workloads.seed_of("temporal_stream")
+    x = workloads.activation(1, 4096, seed, 10000, device=dev)
+    xd = workloads.activation(1, 11264, seed, 10001, device=dev)
+    probs = []
+    for t, p in sel:
+        c, s, b = q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+        probs.append((xd if p.K == 11264 else x, c, s, b, torch.empty((1, p.N), dtype=torch.bfloat16, device=dev)))
+    return lambda: q4.q4_matmul_batch(probs)
+
+
+def _tc_layer(dev):
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    packed = [(p,) + tuple(q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev)))
+              for t, p in enumerate(workloads.TEMPORAL_LAYER)]
+    xs = {M: (workloads.activation(M, 4096, seed, 100 + M, device=dev),
+              workloads.activation(M, 11264, seed, 200 + M, device=dev)) for M in (64, 256)}
+
+    def run():
+        for M in (64, 256):
+            for p, c, s, b in packed:
+                q4.q4_matmul(xs[M][1] if p.K == 11264 else xs[M][0], c, s, b)
+
+    return run
+
+
+def _depformer_step(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("depformer_steps")
+    steps = workloads.DEPFORMER_STEPS
+    xs = {K: workloads.activation(1, K, seed, 500 + K, device=dev) for K in (1024, 2816)}
+    probs = []
+    for t, p in enumerate(workloads.depformer_projs()):
+        c, s, b = q4.q4_quantize(workloads.weight(steps * p.N, p.K, seed, t, device=dev))
+        probs.append((xs[p.K], c[:p.N], s[:p.N], b[:p.N], torch.empty((1, p.N), dtype=torch.bfloat16, device=dev)))
+    return lambda: q4.q4_matmul_batch(probs)
+
+
+CASES = {"stream_small": _stream_small, "tc_layer": _tc_layer, "depformer_step": _depformer_step}
+
+
+def main(argv=None):
+    import torch
+
+    import weight_only_bit_affine_b200 as q4
+
+    argv = sys.argv[1:] if argv is None else argv
+    if not argv or argv[0] not in CASES:
+        raise SystemExit(f"usage: profile_case <{'|'.join(CASES)}> [reps]")
+    reps = int(argv[1]) if len(argv) > 1 else 3
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    run = CASES[argv[0]](dev)
+    torch.cuda.synchronize(dev)
+    for _ in range(1 + reps):
+        run()
+    torch.cuda.synchronize(dev)
+    if q4.q4_debug_device_flags() != 0:
+        raise SystemExit("a bounded wait gave up inside a kernel")
+    print(f"{argv[0]}: {reps} reps ok")
+
+
+if __name__ == "__main__":
+    main()
