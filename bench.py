@@ -40,6 +40,27 @@ def _dist_env():
     return world, rank, local
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity on one rank).
+
+    The benchmark's only collective besides the barrier: each replica times its
+    own stream, and the job's time is the slowest replica's.
+    """
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_gbps(world: int, bytes_per_replica: int, ms_max: float) -> float:
+    """Whole-job GB/s: every replica streams its bytes; time is the slowest rank's."""
+    return world * bytes_per_replica / (ms_max * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------------- clocks
 
 
@@ -149,13 +170,16 @@ def enqueue_stream_batched(packed, x, x_down, ys):
     q4.q4_matmul_batch([(x_down if p.K == 11264 else x, c, s, b, y) for (p, c, s, b), y in zip(packed, ys)])
 
 
-def _kernel_source_hash() -> str:
+GEMV_SOURCES = ("q4_gemv.cu", "q4_device.cuh", "q4_internal.h")
+
+
+def _kernel_source_hash(files=GEMV_SOURCES) -> str:
+    """Hash of the sources the M=1 kernel is built from (keys the committed DRAM traffic)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_only_bit_affine_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+    for f in sorted(files):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -538,11 +562,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     ms_e2e = max(ev0.elapsed_time(ev1), (time.perf_counter() - t_wall0) * 1e3) / e2e_steps
 
-    # max over ranks
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], device=dev)
 
     extra = {}
     if not args.no_rows:
@@ -554,7 +574,7 @@ def run_ours(args):
     traffic = _traffic_per_launch(kh)
     line = {
         "metric": METRIC,
-        "value": round(world * nbytes / (ms * 1e-3) / 1e9, 2),
+        "value": round(job_gbps(world, nbytes, ms), 2),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -584,7 +604,7 @@ def run_ours(args):
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback",
             "kernel": "gemv_kernel<MR=1> (one launch per step, all 225 problems); CUDA events on its stream",
         },
-        "e2e": {"value": round(world * nbytes / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(job_gbps(world, nbytes, ms_e2e), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "how": "pinned x H2D + graph replay of the public q4_matmul_batch call + y D2H, per step"},
         "gpu_launches": int(launches_per_step) * args.steps,

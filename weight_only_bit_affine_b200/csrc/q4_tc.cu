@@ -146,10 +146,18 @@ __device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t 
 }
 
 // ---- the kernel ------------------------------------------------------------
+//
+// A pipeline stage covers ATOMS x 64 inputs k (one or two 128-byte swizzle
+// spans): fewer, larger stages cut the fixed per-stage cost of every role
+// (barrier waits, TMA issue, MMA issue and commit) when shared memory allows
+// at least three of them.
 
+template <int ATOMS>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
               const __grid_constant__ TcParams p) {
+  constexpr int kStageK = kChunkK * ATOMS;
+  constexpr int kStagesPerSuper = kSuperK / kStageK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled operand tiles.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -165,8 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t m0 = static_cast<int64_t>(blockIdx.z) * p.bn;
   const int supers = p.K / kSuperK;
   const int sc_begin = split * supers / p.splits, sc_end = (split + 1) * supers / p.splits;
-  const int chunk_begin = sc_begin * (kSuperK / kChunkK);
-  const int nchunks = (sc_end - sc_begin) * (kSuperK / kChunkK);
+  const int stage_begin = sc_begin * kStagesPerSuper;
+  const int nstages = (sc_end - sc_begin) * kStagesPerSuper;
 
   if (tid == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -190,40 +198,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   pdl_wait_predecessors();
 
+  // Stage layout: ATOMS A tiles (128 rows x 128 B each, 16 KB apart), then
+  // ATOMS x tiles (bn rows x 128 B each), then the code tile (128 rows x
+  // 32*ATOMS bytes).
+  const uint32_t b_atom = static_cast<uint32_t>(p.bn) * 128u;
   auto a_tile = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
-  auto b_tile = [&](int s) { return a_tile(s) + kATileBytes; };
-  auto c_tile = [&](int s) { return a_tile(s) + kATileBytes + p.b_tile_bytes; };
+  auto b_tile = [&](int s) { return a_tile(s) + ATOMS * kATileBytes; };
+  auto c_tile = [&](int s) { return b_tile(s) + ATOMS * b_atom; };
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       bool dead = false;
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % p.stages;
-        const uint32_t ph = static_cast<uint32_t>(c / p.stages) & 1u;
+      int s = 0;
+      uint32_t ph = 0;
+      for (int c = 0; c < nstages; ++c) {
         if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&stage_free[s], ph ^ 1u)) dead = true;
-        const int k0 = (chunk_begin + c) * kChunkK;
-        mbar_arrive_expect_tx(&tma_full[s], p.b_tile_bytes + kCodeTileBytes);
-        tma_load_2d(b_tile(s), &tmap_x, k0, static_cast<int>(m0), &tma_full[s]);
+        const int k0 = (stage_begin + c) * kStageK;
+        mbar_arrive_expect_tx(&tma_full[s], ATOMS * b_atom + kTileN * kStageK / 2);
+#pragma unroll
+        for (int at = 0; at < ATOMS; ++at)
+          tma_load_2d(b_tile(s) + at * b_atom, &tmap_x, k0 + at * kChunkK, static_cast<int>(m0), &tma_full[s]);
         tma_load_2d(c_tile(s), &tmap_codes, k0 / 2, static_cast<int>(n0), &tma_full[s]);
+        if (++s == p.stages) { s = 0; ph ^= 1u; }
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // Waits only for the dequantizing warps: they arrive after having waited
+    // for this stage's TMA themselves, so the x tile is in place too.
     if (lane == 0) {
       bool dead = false;
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % p.stages;
-        const uint32_t ph = static_cast<uint32_t>(c / p.stages) & 1u;
-        if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&tma_full[s], ph)) dead = true;
+      int s = 0;
+      uint32_t ph = 0;
+      for (int c = 0; c < nstages; ++c) {
         if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&a_full[s], ph)) dead = true;
         tc_fence_after();
         const uint64_t ad = sw128_desc(smem_u32(a_tile(s)));
         const uint64_t bd = sw128_desc(smem_u32(b_tile(s)));
 #pragma unroll
-        for (int kk = 0; kk < kChunkK / 16; ++kk)  // 16 bf16 = 32 bytes per MMA step
-          tc_mma_f16(tmem_base, ad + 2 * kk, bd + 2 * kk, p.idesc, (c > 0 || kk > 0) ? 1u : 0u);
+        for (int at = 0; at < ATOMS; ++at)
+#pragma unroll
+          for (int kk = 0; kk < kChunkK / 16; ++kk)  // 16 bf16 = 32 bytes per MMA step
+            tc_mma_f16(tmem_base, ad + at * (kATileBytes >> 4) + 2 * kk, bd + at * (b_atom >> 4) + 2 * kk, p.idesc,
+                       (c > 0 || at > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&stage_free[s]);
+        if (++s == p.stages) { s = 0; ph ^= 1u; }
       }
       tc_commit(accum_full);
     }
@@ -231,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- dequantize, then epilogue ----------------
     const int t = tid - 64;
     const int row = t & (kTileN - 1);  // weight row within the tile
-    const int half = t >> 7;           // which group of the 64-wide chunk
+    const int half = t >> 7;           // which group of each 64-wide atom
     const int64_t grow = n0 + row;
     const bool row_ok = grow < p.N;
     const int G = p.K / 32;
@@ -251,46 +271,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     load_sb(sc_begin, s_cur, b_cur);
     load_sb(sc_begin + 1, s_nxt, b_nxt);
     bool dead = false;
-    for (int c = 0; c < nchunks; ++c) {
-      const int s = c % p.stages;
-      const uint32_t ph = static_cast<uint32_t>(c / p.stages) & 1u;
-      const int sub = c & 3;  // chunk within the super-chunk
+    int s = 0, sub = 0, sc_next = sc_begin + 2;
+    uint32_t ph = 0;
+    for (int c = 0; c < nstages; ++c) {
       if (c > 0 && sub == 0) {
         s_cur = s_nxt;
         b_cur = b_nxt;
-        load_sb(sc_begin + c / 4 + 1, s_nxt, b_nxt);
+        load_sb(sc_next++, s_nxt, b_nxt);
       }
-      // group (2*sub + half) of the current super-chunk: 16-bit lane of s_cur/b_cur
-      const int gi = 2 * sub + half;
-      const uint32_t sw = (gi < 2) ? s_cur.x : (gi < 4) ? s_cur.y : (gi < 6) ? s_cur.z : s_cur.w;
-      const uint32_t bw = (gi < 2) ? b_cur.x : (gi < 4) ? b_cur.y : (gi < 6) ? b_cur.z : b_cur.w;
-      const uint32_t sel = (gi & 1) ? 0x3232u : 0x1010u;  // broadcast one bf16 to both halves
-      const uint32_t s2 = __byte_perm(sw, 0, sel);
-      const uint32_t b2 = __byte_perm(bw, 0, sel);
-
       if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&stage_free[s], ph ^ 1u)) dead = true;  // A buffer no longer read
       if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&tma_full[s], ph)) dead = true;         // codes arrived
-      const uint4 cw = *reinterpret_cast<const uint4*>(c_tile(s) + row * 32 + half * 16);
-      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-      uint8_t* arow = a_tile(s) + row * 128;
+      const uint8_t* crow = c_tile(s) + row * (32 * ATOMS);
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint32_t wd = words[w], w4 = wd >> 4;
-        uint32_t o[4];
+      for (int at = 0; at < ATOMS; ++at) {
+        // group (2*(sub*ATOMS + at) + half) of the current super-chunk
+        const int gi = 2 * (sub * ATOMS + at) + half;
+        const uint32_t sw = (gi < 2) ? s_cur.x : (gi < 4) ? s_cur.y : (gi < 6) ? s_cur.z : s_cur.w;
+        const uint32_t bw = (gi < 2) ? b_cur.x : (gi < 4) ? b_cur.y : (gi < 6) ? b_cur.z : b_cur.w;
+        const uint32_t sel = (gi & 1) ? 0x3232u : 0x1010u;  // broadcast one bf16 to both halves
+        const uint32_t s2 = __byte_perm(sw, 0, sel);
+        const uint32_t b2 = __byte_perm(bw, 0, sel);
+        const uint4 cw = *reinterpret_cast<const uint4*>(crow + at * 32 + half * 16);
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        uint8_t* arow = a_tile(s) + at * kATileBytes + row * 128;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          // bytes: [wd.byte_i, -, w4.byte_i, -] -> nibbles q[2i] at bits 0..3, q[2i+1] at 16..19
-          const uint32_t pr = __byte_perm(wd, w4, (i) | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-          const uint32_t v = (pr & 0x000F000Fu) | 0x43004300u;  // (128 + q, 128 + q') exactly
-          const uint32_t q = bf16x2_sub(v, 0x43004300u);          // (q, q') exactly
-          o[i] = bf16x2_fma(q, s2, b2);                           // bf16(s*q + b), one rounding
+        for (int w = 0; w < 4; ++w) {
+          const uint32_t wd = words[w], w4 = wd >> 4;
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            // bytes: [wd.byte_i, -, w4.byte_i, -] -> nibbles q[2i] at bits 0..3, q[2i+1] at 16..19
+            const uint32_t pr = __byte_perm(wd, w4, (i) | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
+            const uint32_t v = (pr & 0x000F000Fu) | 0x43004300u;  // (128 + q, 128 + q') exactly
+            const uint32_t q = bf16x2_sub(v, 0x43004300u);          // (q, q') exactly
+            o[i] = bf16x2_fma(q, s2, b2);                           // bf16(s*q + b), one rounding
+          }
+          const int chunk16 = 4 * half + w;  // 16-byte chunk (8 k) within the 128-byte row
+          *reinterpret_cast<uint4*>(arow + ((chunk16 ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        const int chunk16 = 4 * half + w;  // 16-byte chunk (8 k) within the 128-byte row
-        *reinterpret_cast<uint4*>(arow + ((chunk16 ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       fence_proxy_async_smem();  // make the generic stores visible to the tensor core
       __syncwarp();
       if (lane == 0) mbar_arrive(&a_full[s]);
+      if (++s == p.stages) { s = 0; ph ^= 1u; }
+      if (++sub == kStagesPerSuper) sub = 0;
     }
 
     // ---- epilogue: tensor memory -> y (or partial sums for the cluster) ----
@@ -418,6 +442,15 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
     if (want > splits && want <= supers && tiles * want <= dev.sm_count * 1.05) splits = want;
   }
 
+  // Two 64-wide atoms per stage when at least three such stages fit.
+  const uint32_t b_atom = static_cast<uint32_t>(bn) * kChunkK * 2;
+  auto stage_size = [&](int atoms) {
+    return (static_cast<uint32_t>(atoms) * (kATileBytes + b_atom + kCodeTileBytes) + 1023u) & ~1023u;
+  };
+  const size_t barrier_bytes = 8 * (3 * 12 + 1) + 16;
+  const size_t avail = dev.smem_optin - 1024 - barrier_bytes;
+  const int atoms = (avail / stage_size(2) >= 3) ? 2 : 1;
+
   CUtensorMap tmap_x, tmap_codes;
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
@@ -432,7 +465,7 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 2), static_cast<cuuint64_t>(a.N)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 2)};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunkK / 2), static_cast<cuuint32_t>(kTileN)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunkK / 2 * atoms), static_cast<cuuint32_t>(kTileN)};
     cuuint32_t estr[2] = {1, 1};
     if (encode(&tmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.codes), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -449,12 +482,10 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
   p.K = static_cast<int>(a.K);
   p.bn = bn;
   p.splits = splits;
-  p.b_tile_bytes = static_cast<uint32_t>(bn) * kChunkK * 2;
-  p.stage_bytes = (kATileBytes + p.b_tile_bytes + kCodeTileBytes + 1023u) & ~1023u;
+  p.b_tile_bytes = b_atom;
+  p.stage_bytes = stage_size(atoms);
   const size_t red_bytes = static_cast<size_t>(kTileN) * (bn + 4) * 4;
-  const size_t barrier_bytes = 8 * (3 * 8 + 1) + 16;
-  const size_t avail = dev.smem_optin - 1024 - barrier_bytes;
-  p.stages = static_cast<int>(std::min<size_t>(6, avail / p.stage_bytes));
+  p.stages = static_cast<int>(std::min<size_t>(12, avail / p.stage_bytes));
   while (p.stages > 2 && static_cast<size_t>(p.stages) * p.stage_bytes < red_bytes) ++p.stages;
   if (p.stages < 2 || static_cast<size_t>(p.stages) * p.stage_bytes < red_bytes ||
       static_cast<size_t>(p.stages) * p.stage_bytes > avail)
@@ -467,10 +498,12 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
 
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(dev.smem_optin));
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-    if (e != cudaSuccess) return e;
+    for (auto kern : {tc_kernel<1>, tc_kernel<2>}) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(dev.smem_optin));
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+      if (e != cudaSuccess) return e;
+    }
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
@@ -488,7 +521,8 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   count_launch();
-  return cudaLaunchKernelEx(&cfg, tc_kernel, tmap_x, tmap_codes, p);
+  return atoms == 2 ? cudaLaunchKernelEx(&cfg, tc_kernel<2>, tmap_x, tmap_codes, p)
+                    : cudaLaunchKernelEx(&cfg, tc_kernel<1>, tmap_x, tmap_codes, p);
 }
 
 }  // namespace q4
