@@ -82,6 +82,7 @@ q4_status matmul_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* co
   const DeviceInfo* dev;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   MatmulArgs a{x, codes, scales, biases, y, M, N, K};
+  if (stream_supported(a, *dev)) return from_cuda(launch_stream_batch(&a, 1, stream, *dev), "q4_matmul launch");
   if (M >= kTensorCoreMinRows && tc_supported(a)) return from_cuda(launch_tc(a, stream, *dev), "q4_matmul launch");
   return from_cuda(launch_gemv(a, stream, *dev), "q4_matmul launch");
 }
@@ -201,14 +202,22 @@ q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int
   q4_status st;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  std::vector<MatmulArgs> gemv;
+  // Each problem takes the path it would take alone, so a batched result is
+  // bit-identical to the single call.
+  std::vector<MatmulArgs> gemv, streamed;
   for (const MatmulArgs& a : list) {
-    if (a.M >= kTensorCoreMinRows && tc_supported(a)) {
+    if (stream_supported(a, *dev)) {
+      streamed.push_back(a);
+    } else if (a.M >= kTensorCoreMinRows && tc_supported(a)) {
       if ((st = from_cuda(launch_tc(a, cs, *dev), "q4_matmul_batch launch")) != Q4_OK) return st;
     } else {
       gemv.push_back(a);
     }
   }
+  if (!streamed.empty() &&
+      (st = from_cuda(launch_stream_batch(streamed.data(), static_cast<int>(streamed.size()), cs, *dev),
+                      "q4_matmul_batch launch")) != Q4_OK)
+    return st;
   if (gemv.empty()) return Q4_OK;
   return from_cuda(launch_gemv_batch(gemv.data(), static_cast<int>(gemv.size()), cs, *dev), "q4_matmul_batch launch");
 }
@@ -218,8 +227,11 @@ const char* q4_last_error(void) { return t_last_error; }
 unsigned long long q4_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int q4_debug_device_flags(int clear) {
-  unsigned int f = 0;
-  if (gemv_device_flags(&f, clear != 0) != cudaSuccess) return -1;
+  unsigned int f = 0, t = 0, s = 0;
+  if (gemv_device_flags(&f, clear != 0) != cudaSuccess || tc_device_flags(&t, clear != 0) != cudaSuccess ||
+      stream_device_flags(&s, clear != 0) != cudaSuccess)
+    return -1;
+  f |= t | s;
   return static_cast<int>(f);
 }
 

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 #include <cstdint>
 
 namespace q4 {
@@ -13,6 +14,16 @@ namespace q4 {
 // q4_debug_device_flags().
 enum : unsigned int { kFlagWaitTimeout = 1u };
 static __device__ unsigned int g_device_flags = 0;
+
+// Host side: read (and optionally clear) this translation unit's flag word.
+static inline cudaError_t tu_device_flags(unsigned int* flags, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(flags, g_device_flags, sizeof(unsigned int));
+  if (e == cudaSuccess && clear) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_flags, &zero, sizeof(unsigned int));
+  }
+  return e;
+}
 
 // A wait gives up after this many nanoseconds of %globaltimer (1 s): far
 // beyond any legitimate wait in these kernels.
@@ -144,17 +155,26 @@ __device__ __forceinline__ void fma_bf16x2_f32(float& c0, float& c1, uint32_t a2
 // whose last significand bit weighs 1), and fma.rn.f32.bf16 multiplies the
 // bf16 halves exactly and accumulates in fp32 with one rounding.  Written as
 // one PTX block so the 16-bit halves are used in place (no extraction moves).
+// The LOP3 constants (mask 0x000F000F, magic 0x43004300) come in registers
+// that the caller holds across its loop (see q4_lop3_constants): given as two
+// immediates, each LOP3 would rebuild one of them first.
+__device__ __forceinline__ void q4_lop3_constants(uint32_t& mask, uint32_t& magic) {
+  mask = 0x000F000Fu;
+  magic = 0x43004300u;
+  asm volatile("" : "+r"(mask), "+r"(magic));  // opaque: kept in registers, not rebuilt per use
+}
+
 __device__ __forceinline__ void word_dot_bf16(uint32_t w, uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3,
-                                              float& c0, float& c1) {
+                                              float& c0, float& c1, uint32_t mask, uint32_t magic) {
   asm("{\n\t.reg .b32 s1, s2, s3, v0, v1, v2, v3;\n\t"
       ".reg .b16 l0, h0, l1, h1, l2, h2, l3, h3, xl0, xh0, xl1, xh1, xl2, xh2, xl3, xh3;\n\t"
       "shr.b32 s1, %2, 4;\n\t"
       "shr.b32 s2, %2, 8;\n\t"
       "shr.b32 s3, %2, 12;\n\t"
-      "lop3.b32 v0, %2, 0x000F000F, 0x43004300, 0xEA;\n\t"
-      "lop3.b32 v1, s1, 0x000F000F, 0x43004300, 0xEA;\n\t"
-      "lop3.b32 v2, s2, 0x000F000F, 0x43004300, 0xEA;\n\t"
-      "lop3.b32 v3, s3, 0x000F000F, 0x43004300, 0xEA;\n\t"
+      "lop3.b32 v0, %2, %7, %8, 0xEA;\n\t"
+      "lop3.b32 v1, s1, %7, %8, 0xEA;\n\t"
+      "lop3.b32 v2, s2, %7, %8, 0xEA;\n\t"
+      "lop3.b32 v3, s3, %7, %8, 0xEA;\n\t"
       "mov.b32 {l0, h0}, v0;\n\tmov.b32 {l1, h1}, v1;\n\tmov.b32 {l2, h2}, v2;\n\tmov.b32 {l3, h3}, v3;\n\t"
       "mov.b32 {xl0, xh0}, %3;\n\tmov.b32 {xl1, xh1}, %4;\n\tmov.b32 {xl2, xh2}, %5;\n\tmov.b32 {xl3, xh3}, %6;\n\t"
       "fma.rn.f32.bf16 %0, xl0, l0, %0;\n\tfma.rn.f32.bf16 %1, xh0, h0, %1;\n\t"
@@ -162,21 +182,21 @@ __device__ __forceinline__ void word_dot_bf16(uint32_t w, uint32_t x0, uint32_t 
       "fma.rn.f32.bf16 %0, xl2, l2, %0;\n\tfma.rn.f32.bf16 %1, xh2, h2, %1;\n\t"
       "fma.rn.f32.bf16 %0, xl3, l3, %0;\n\tfma.rn.f32.bf16 %1, xh3, h3, %1;\n\t}"
       : "+f"(c0), "+f"(c1)
-      : "r"(w), "r"(x0), "r"(x1), "r"(x2), "r"(x3));
+      : "r"(w), "r"(x0), "r"(x1), "r"(x2), "r"(x3), "r"(mask), "r"(magic));
 }
 
 // As word_dot_bf16, with all eight products into one accumulator.
 __device__ __forceinline__ void word_dot_bf16_acc(uint32_t w, uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3,
-                                                  float& c) {
+                                                  float& c, uint32_t mask, uint32_t magic) {
   asm("{\n\t.reg .b32 s1, s2, s3, v0, v1, v2, v3;\n\t"
       ".reg .b16 l0, h0, l1, h1, l2, h2, l3, h3, xl0, xh0, xl1, xh1, xl2, xh2, xl3, xh3;\n\t"
       "shr.b32 s1, %1, 4;\n\t"
       "shr.b32 s2, %1, 8;\n\t"
       "shr.b32 s3, %1, 12;\n\t"
-      "lop3.b32 v0, %1, 0x000F000F, 0x43004300, 0xEA;\n\t"
-      "lop3.b32 v1, s1, 0x000F000F, 0x43004300, 0xEA;\n\t"
-      "lop3.b32 v2, s2, 0x000F000F, 0x43004300, 0xEA;\n\t"
-      "lop3.b32 v3, s3, 0x000F000F, 0x43004300, 0xEA;\n\t"
+      "lop3.b32 v0, %1, %6, %7, 0xEA;\n\t"
+      "lop3.b32 v1, s1, %6, %7, 0xEA;\n\t"
+      "lop3.b32 v2, s2, %6, %7, 0xEA;\n\t"
+      "lop3.b32 v3, s3, %6, %7, 0xEA;\n\t"
       "mov.b32 {l0, h0}, v0;\n\tmov.b32 {l1, h1}, v1;\n\tmov.b32 {l2, h2}, v2;\n\tmov.b32 {l3, h3}, v3;\n\t"
       "mov.b32 {xl0, xh0}, %2;\n\tmov.b32 {xl1, xh1}, %3;\n\tmov.b32 {xl2, xh2}, %4;\n\tmov.b32 {xl3, xh3}, %5;\n\t"
       "fma.rn.f32.bf16 %0, xl0, l0, %0;\n\tfma.rn.f32.bf16 %0, xh0, h0, %0;\n\t"
@@ -184,7 +204,7 @@ __device__ __forceinline__ void word_dot_bf16_acc(uint32_t w, uint32_t x0, uint3
       "fma.rn.f32.bf16 %0, xl2, l2, %0;\n\tfma.rn.f32.bf16 %0, xh2, h2, %0;\n\t"
       "fma.rn.f32.bf16 %0, xl3, l3, %0;\n\tfma.rn.f32.bf16 %0, xh3, h3, %0;\n\t}"
       : "+f"(c)
-      : "r"(w), "r"(x0), "r"(x1), "r"(x2), "r"(x3));
+      : "r"(w), "r"(x0), "r"(x1), "r"(x2), "r"(x3), "r"(mask), "r"(magic));
 }
 
 // Packed fp32x2 fused multiply-add: (c0, c1) += (a0, a1) * (b0, b1).
@@ -227,6 +247,18 @@ __device__ __forceinline__ void unpack_codes_f32(uint32_t w, float (&q)[8]) {
   fadd2(q[2], q[3], -32768.f, -2048.f);
   fadd2(q[4], q[5], -128.f, -32768.f);
   fadd2(q[6], q[7], -2048.f, -128.f);
+}
+
+// bf16x2 arithmetic (packed, one rounding per lane).
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {

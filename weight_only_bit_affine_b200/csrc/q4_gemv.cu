@@ -132,12 +132,14 @@ __device__ __forceinline__ void dot_plus128(const uint32_t (&words)[WORDS], cons
     return;
   }
   if constexpr (MAC == kMacMixedBf16) {
+    uint32_t kmask, kmagic;
+    q4_lop3_constants(kmask, kmagic);
 #pragma unroll
     for (int w = 0; w < WORDS; ++w)
 #pragma unroll
       for (int m = 0; m < MR; ++m)
         word_dot_bf16(words[w], xs[m].v[w][0][0], xs[m].v[w][1][0], xs[m].v[w][2][0], xs[m].v[w][3][0], a0[m],
-                      a1[m]);
+                      a1[m], kmask, kmagic);
   } else {
 #pragma unroll
   for (int w = 0; w < WORDS; ++w) {
@@ -422,6 +424,8 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   }
 
   // ---------------- consumer threads ----------------
+  uint32_t kmask, kmagic;  // the dot product's LOP3 constants, held in registers
+  q4_lop3_constants(kmask, kmagic);
   int stage = 0, slot = 0;
   uint32_t phase = 0, sph = 0;
   bool dead = false;
@@ -511,7 +515,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 #pragma unroll
               for (int w = 0; w < 4; ++w)
                 word_dot_bf16_acc(words[rr][w], xsl[m].v[w][0][0], xsl[m].v[w][1][0], xsl[m].v[w][2][0],
-                                  xsl[m].v[w][3][0], acc);
+                                  xsl[m].v[w][3][0], acc, kmask, kmagic);
             } else {
               float a0[1] = {0.f}, a1[1] = {0.f};
               dot_plus128<1, 4, Q4_GEMV_MAC>(words[rr], *reinterpret_cast<const XSlice<4, Q4_GEMV_MAC>(*)[1]>(&xsl[m]),
@@ -755,14 +759,7 @@ cudaError_t run_problems(std::vector<GemvProblem>& probs, const DeviceInfo& dev,
 
 }  // namespace
 
-cudaError_t gemv_device_flags(unsigned int* flags, bool clear) {
-  cudaError_t e = cudaMemcpyFromSymbol(flags, g_device_flags, sizeof(unsigned int));
-  if (e == cudaSuccess && clear) {
-    const unsigned int zero = 0;
-    e = cudaMemcpyToSymbol(g_device_flags, &zero, sizeof(unsigned int));
-  }
-  return e;
-}
+cudaError_t gemv_device_flags(unsigned int* flags, bool clear) { return tu_device_flags(flags, clear); }
 
 cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev) {
   // Activation rows in chunks of at most two; every chunk of every problem

@@ -46,10 +46,17 @@ constexpr int64_t kTensorCoreMinRows = 16;
 bool tc_supported(const MatmulArgs& a);
 cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev);
 
+// Tensor-core weight streaming (tcgen05, A operand in tensor memory) for
+// three or four activation rows; several problems share one launch.
+bool stream_supported(const MatmulArgs& a, const DeviceInfo& dev);
+cudaError_t launch_stream_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
+
 // Counts every kernel launch libq4 enqueues (host side).
 void count_launch();
 
-// Diagnostic: the bounded-wait flags of the GEMV kernels (synchronous copy).
+// Diagnostics: the bounded-wait flags of each kernel family (synchronous copies).
 cudaError_t gemv_device_flags(unsigned int* flags, bool clear);
+cudaError_t tc_device_flags(unsigned int* flags, bool clear);
+cudaError_t stream_device_flags(unsigned int* flags, bool clear);
 
 }  // namespace q4

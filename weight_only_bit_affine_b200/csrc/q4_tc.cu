@@ -133,18 +133,6 @@ __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t remote_addr) {
   return v;
 }
 
-// bf16x2 helpers (packed, one rounding each).
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
 // ---- the kernel ------------------------------------------------------------
 //
 // A pipeline stage covers ATOMS x 64 inputs k (one or two 128-byte swizzle
@@ -418,6 +406,8 @@ uint32_t make_idesc(int bn) {
 }
 
 }  // namespace
+
+cudaError_t tc_device_flags(unsigned int* flags, bool clear) { return tu_device_flags(flags, clear); }
 
 bool tc_supported(const MatmulArgs& a) {
   if (a.K % kSuperK != 0) return false;
