@@ -329,16 +329,17 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
         ysm = [y_for(M, l) for l in layer]
 
         def run_layers(xb=xb, xbd=xbd, ysm=ysm, M=M):
-            for l, ys in zip(layer, ysm):
-                for (p, c, s, b), y in zip(l, ys):
-                    q4.q4_matmul(xbd if p.K == 11264 else xb, c, s, b, out=y)
+            for l, ys in zip(layer, ysm):  # one q4_matmul_batch per layer (7 projections)
+                q4.q4_matmul_batch([(xbd if p.K == 11264 else xb, c, s, b, y) for (p, c, s, b), y in zip(l, ys)])
 
         t = _graph_ms(dev, run_layers, 20) / 4
         tf = flops_layer * M / (t * 1e-3) / 1e12
         rows[f"batched_layer_M{M}"] = {
             "us_per_layer": round(t * 1e3, 2), "TFLOPs": round(tf, 1),
             "frac_of_bf16_peak": round(tf / bf16_peak, 4), "packed_GBps": round(lbytes / (t * 1e-3) / 1e9, 1),
-            "path": "tcgen05 tensor cores" if M >= 16 else "CUDA-core GEMV (activation rows in pairs)",
+            "path": ("tc_kernel: tcgen05, dequantized tile in shared memory" if M >= 16 else
+                     "stream_kernel: tcgen05, dequantized weights in tensor memory" if M >= 3 else
+                     "gemv_kernel: CUDA cores"),
         }
     return rows
 

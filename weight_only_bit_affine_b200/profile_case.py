@@ -12,6 +12,8 @@ whole case once, after one warm-up rep):
                  at M = 64 and then M = 256: the tensor-core kernel.
   depformer_step one depformer codebook step (43 step-sliced projections) as
                  one q4_matmul_batch.
+  layer_m4       one temporal layer (7 projections) at M = 4 as one
+                 q4_matmul_batch: the tensor-core streaming kernel.
 
 Every case checks the library's bounded-wait flag at the end.
 """
@@ -77,7 +79,25 @@ def _depformer_step(dev):
     return lambda: q4.q4_matmul_batch(probs)
 
 
-CASES = {"stream_small": _stream_small, "tc_layer": _tc_layer, "depformer_step": _depformer_step}
+def _layer_m4(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    M = 4
+    x = workloads.activation(M, 4096, seed, 100 + M, device=dev)
+    xd = workloads.activation(M, 11264, seed, 200 + M, device=dev)
+    probs = []
+    for t, p in enumerate(workloads.TEMPORAL_LAYER):
+        c, s, b = q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+        probs.append((xd if p.K == 11264 else x, c, s, b, torch.empty((M, p.N), dtype=torch.bfloat16, device=dev)))
+    return lambda: q4.q4_matmul_batch(probs)
+
+
+CASES = {"stream_small": _stream_small, "tc_layer": _tc_layer, "depformer_step": _depformer_step,
+         "layer_m4": _layer_m4}
 
 
 def main(argv=None):
