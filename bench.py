@@ -374,7 +374,7 @@ class OracleSample:
             self.items.append((p, c, s, b))
             spent += self._run_one(self.items[-1])
         self.nbytes = sum(c.size + 2 * s.size + 2 * b.size for _, c, s, b in self.items)
-        self.threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+        self.threads = oracle.max_threads()
         names = [p.name for p, _, _, _ in self.items]
         self.desc = (f"oracle dequantize+matmul (C, binary64, OpenMP, {self.threads} threads) on the first "
                      f"{len(names)} of 225 stream projections ({names[0]}..{names[-1]}, {self.nbytes} packed bytes)")
@@ -390,6 +390,25 @@ class OracleSample:
     def time(self):
         spent = sum(self._run_one(it) for it in self.items)
         return self.nbytes / spent / 1e9, spent
+
+    def time_one_thread(self, budget_s: float):
+        """The same oracle on one host thread, over the first projections of
+        the sample until about `budget_s` seconds: GB/s, projections, seconds."""
+        import oracle
+
+        oracle.set_threads(1)
+        try:
+            spent, nbytes, n = 0.0, 0, 0
+            for it in self.items:
+                if spent >= budget_s:
+                    break
+                spent += self._run_one(it)
+                _, c, s, b = it
+                nbytes += c.size + 2 * s.size + 2 * b.size
+                n += 1
+        finally:
+            oracle.set_threads(self.threads)
+        return nbytes / spent / 1e9, n, spent
 
 
 # --------------------------------------------------------------------- arms
@@ -626,6 +645,9 @@ def run_ours(args):
         gbs, spent = sample.time()
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": sample.threads, "kind": "oracle",
                                 "sample": sample.desc, "seconds": round(spent, 2)}
+        gbs1, n1, spent1 = sample.time_one_thread(float(os.environ.get("Q4_CPU_BASELINE_1T_SECONDS", "8")))
+        line["rows"]["cpu_oracle_one_thread"] = {"GBps": round(gbs1, 4), "projections": n1, "seconds": round(spent1, 2),
+                                                 "note": "the same oracle on 1 host thread, first projections"}
     del graph, graph_calls
     if world > 1:
         dist.barrier()

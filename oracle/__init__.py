@@ -64,6 +64,10 @@ def _load():
         lib.oq4_matmul_ref.argtypes = [p, i64, i64, p, p, p, i64, p, i64, p, p]
         lib.oq4_matmul_ref_factored.restype = ctypes.c_int
         lib.oq4_matmul_ref_factored.argtypes = [p, i64, i64, p, p, p, i64, p]
+        lib.oq4_set_threads.restype = None
+        lib.oq4_set_threads.argtypes = [ctypes.c_int]
+        lib.oq4_max_threads.restype = ctypes.c_int
+        lib.oq4_max_threads.argtypes = []
         _lib = lib
     return _lib
 
@@ -182,6 +186,15 @@ def matmul_ref_factored(x_bits, codes, scales, biases) -> np.ndarray:
     _check(_load().oq4_matmul_ref_factored(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases),
                                            N, _ptr(y)), "matmul_ref_factored")
     return y
+
+
+def set_threads(n: int) -> None:
+    """Threads of the oracle's OpenMP loops (timing only: results do not depend on it)."""
+    _load().oq4_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(_load().oq4_max_threads())
 
 
 def nrmse(W_ref: np.ndarray, W_hat: np.ndarray) -> float:

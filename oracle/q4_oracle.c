@@ -36,6 +36,9 @@
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define OQ4_GROUP 32
 
@@ -245,4 +248,22 @@ int oq4_matmul_ref_factored(const uint16_t* x, int64_t M, int64_t K, const uint8
     }
   }
   return OQ4_OK;
+}
+
+/* Threads used by the OpenMP loops above (timing only; results do not depend
+ * on it: every output element is computed by one thread in a fixed order). */
+void oq4_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+int oq4_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
 }

@@ -335,3 +335,22 @@ def test_tolerance_helper(oracle):
     ref = np.array([[1.0, 2.01]])
     ad = np.array([[10.0, 1.0]])
     assert oracle.tolerance_ok(y, ref, ad).tolist() == [[True, False]]
+
+
+def test_oracle_results_independent_of_thread_count(oracle):
+    """Timing knob only: every output element is computed by one thread in a fixed order."""
+    rng = np.random.default_rng(77)
+    W = workloads.bf16_bits(torch.from_numpy(rng.standard_normal((96, 512)).astype(np.float32) * 0.02))
+    x = workloads.bf16_bits(torch.from_numpy(rng.standard_normal((2, 512)).astype(np.float32)))
+    n0 = oracle.max_threads()
+    try:
+        oracle.set_threads(1)
+        c1, s1, b1 = oracle.quantize(W)
+        y1, a1 = oracle.matmul_ref(x, c1, s1, b1)
+        oracle.set_threads(4)
+        c4, s4, b4 = oracle.quantize(W)
+        y4, a4 = oracle.matmul_ref(x, c4, s4, b4)
+    finally:
+        oracle.set_threads(n0)
+    assert np.array_equal(c1, c4) and np.array_equal(s1, s4) and np.array_equal(b1, b4)
+    assert np.array_equal(y1, y4) and np.array_equal(a1, a4)
