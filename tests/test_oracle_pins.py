@@ -340,8 +340,8 @@ def test_tolerance_helper(oracle):
 def test_oracle_results_independent_of_thread_count(oracle):
     """Timing knob only: every output element is computed by one thread in a fixed order."""
     rng = np.random.default_rng(77)
-    W = workloads.bf16_bits(torch.from_numpy(rng.standard_normal((96, 512)).astype(np.float32) * 0.02))
-    x = workloads.bf16_bits(torch.from_numpy(rng.standard_normal((2, 512)).astype(np.float32)))
+    W = workloads.bf16_bits(torch.from_numpy(rng.standard_normal((96, 512)).astype(np.float32) * 0.02).to(torch.bfloat16))
+    x = workloads.bf16_bits(torch.from_numpy(rng.standard_normal((2, 512)).astype(np.float32)).to(torch.bfloat16))
     n0 = oracle.max_threads()
     try:
         oracle.set_threads(1)
