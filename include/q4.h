@@ -104,7 +104,13 @@ Q4_API q4_status q4_dequantize(const uint8_t* codes, const q4_bf16* scales,
  * are not expanded back to BF16).
  * In:  x [M, K] bf16 (row-major), codes [N, K/2], scales, biases [N, K/32].
  * Out: y [M, N] bf16 (row-major).
- * M < 16 runs the CUDA-core GEMV family; M >= 16 the tensor-core path.
+ * Kernel by M (the same for every problem, alone or batched, so a batched
+ * result is bit-identical to the single call): M = 1, 2 the CUDA-core GEMV;
+ * M = 3, 4 (K % 256 == 0, 16-byte aligned scale and bias rows) tensor-core
+ * weight streaming, dequantized weights in tensor memory; M >= 16 (K % 256
+ * == 0, same alignment) tensor-core tiles; otherwise the GEMV on pairs of
+ * activation rows.  Results of the tensor-core kernels use w_hat rounded to
+ * bf16 (exactly q4_dequantize's values); the GEMV uses the exact s*q + b.
  * Launch-order contract: the kernels may be launched with programmatic
  * dependent launch; they read nothing written by an earlier kernel in the
  * stream before that kernel has completed.
@@ -141,7 +147,8 @@ typedef struct {
  * q4_matmul_batch -- `count` independent matmuls sharing the number of
  * activation rows M, each computing exactly what q4_matmul computes, enqueued
  * as few kernel launches as possible: one for up to 256 problems that take
- * the bulk-copy GEMV path.  The Swift/MLX blog ("Performance optimizations":
+ * the bulk-copy GEMV path (or the weight-streaming path), one per problem on
+ * the tensor-core tile path.  The Swift/MLX blog ("Performance optimizations":
  * compiling the temporal transformer fuses its ~450 per-step kernel
  * dispatches) and the ONNX README ("All four variants": CUDA Graph capture)
  * both cut per-call launch overhead; this is that fusion for a whole weight
