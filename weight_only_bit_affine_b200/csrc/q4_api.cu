@@ -79,7 +79,7 @@ q4_status matmul_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* co
   bool empty = false;
   q4_status st = check_matmul("q4_matmul", x, M, K, codes, scales, biases, N, group, y, &empty);
   if (st != Q4_OK || empty) return st;
-  const DeviceInfo* dev;
+  const DeviceInfo* dev = nullptr;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   MatmulArgs a{x, codes, scales, biases, y, M, N, K};
   if (stream_supported(a, *dev)) return from_cuda(launch_stream_batch(&a, 1, stream, *dev), "q4_matmul launch");
@@ -139,7 +139,7 @@ q4_status q4_quantize(const q4_bf16* W, int64_t N, int64_t K, int group, uint8_t
     return fail(Q4_ERR_ALIGN, "q4_quantize: W and codes must be 16-byte aligned");
   if (!aligned(scales, 2) || !aligned(biases, 2))
     return fail(Q4_ERR_ALIGN, "q4_quantize: scales and biases must be 2-byte aligned");
-  const DeviceInfo* dev;
+  const DeviceInfo* dev = nullptr;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   return from_cuda(launch_quantize(W, N, K, codes, scales, biases, reinterpret_cast<cudaStream_t>(stream), *dev),
                    "q4_quantize launch");
@@ -156,7 +156,7 @@ q4_status q4_dequantize(const uint8_t* codes, const q4_bf16* scales, const q4_bf
     return fail(Q4_ERR_ALIGN, "q4_dequantize: W_out and codes must be 16-byte aligned");
   if (!aligned(scales, 2) || !aligned(biases, 2))
     return fail(Q4_ERR_ALIGN, "q4_dequantize: scales and biases must be 2-byte aligned");
-  const DeviceInfo* dev;
+  const DeviceInfo* dev = nullptr;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   return from_cuda(
       launch_dequantize(codes, scales, biases, N, K, W_out, reinterpret_cast<cudaStream_t>(stream), *dev),
@@ -198,7 +198,7 @@ q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int
     if (!empty) list.push_back(MatmulArgs{d.x, d.codes, d.scales, d.biases, d.y, M, d.N, d.K});
   }
   if (list.empty()) return Q4_OK;
-  const DeviceInfo* dev;
+  const DeviceInfo* dev = nullptr;
   q4_status st;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
