@@ -319,6 +319,23 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
         "note": "43 step-sliced projections per codebook step; 'step_calls' = 43 q4_matmul_step launches per step, "
                 "'batched' = one q4_matmul_batch launch per step",
     }
+
+    # the same frame for four concurrent conversations (M = 4 rows per step slice)
+    x4 = {K: workloads.activation(4, K, seed, 600 + K, device=dev) for K in (1024, 2816)}
+    ys4 = [torch.empty((4, p.N), dtype=torch.bfloat16, device=dev) for p, _, _, _ in dep]
+
+    def frame_batched_m4():
+        for st in range(steps):
+            sl = lambda t: t[st * (t.shape[0] // steps):(st + 1) * (t.shape[0] // steps)]
+            q4.q4_matmul_batch([(x4[p.K], sl(c), sl(s), sl(b), y) for (p, c, s, b), y in zip(dep, ys4)])
+
+    ms_m4 = _graph_ms(dev, frame_batched_m4, 20)
+    rows["depformer_steps_M4"] = {
+        "batched_us_per_step": round(ms_m4 * 1e3 / steps, 2), "batched_ms_per_frame": round(ms_m4, 4),
+        "packed_GBps": round(fbytes / (ms_m4 * 1e-3) / 1e9, 1),
+        "path": "stream_kernel: tcgen05, dequantized weights in tensor memory",
+        "note": "four conversations' rows per step slice, one q4_matmul_batch launch per codebook step",
+    }
     del dep
 
     # batched layer for concurrent conversations / prefill

@@ -108,3 +108,18 @@ def test_stream_large_problem_sampled():
         x = workloads.activation(4, K, 54, 1, device=DEV)
         y = q4.q4_matmul(x, c, s, b)
         check_matmul(x, c, s, b, y, rows=sample_rows(N, 256, seed=7), what=f"{N}x{K}")
+
+
+@pytest.mark.parametrize("N,K", [(1024, 1024), (2816, 1024), (1024, 2816)])
+def test_stream_step_slices(N, K):
+    """Depformer step slices for four concurrent conversations: q4_matmul_step
+    equals q4_matmul on the slice bit for bit, and the oracle within the bound."""
+    steps = workloads.DEPFORMER_STEPS
+    c, s, b = _packed(steps * N, K, 55, N + K)
+    x = workloads.activation(4, K, 55, 7, device=DEV)
+    for step in (0, 9, steps - 1):
+        y1 = q4.q4_matmul_step(x, c, s, b, steps, step)
+        sl = slice(step * N, (step + 1) * N)
+        y2 = q4.q4_matmul(x, c[sl].contiguous(), s[sl].contiguous(), b[sl].contiguous())
+        assert torch.equal(y1, y2), step
+        check_matmul(x, c[sl], s[sl], b[sl], y1, rows=sample_rows(N, 64, seed=step), what=f"step {step} {N}x{K}")

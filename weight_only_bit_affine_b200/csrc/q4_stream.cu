@@ -5,10 +5,12 @@
 //
 // with the products and the fp32 accumulation done by the 5th-generation
 // tensor cores (tcgen05.mma, kind::f16) and the CUDA cores doing nothing but
-// the dequantization.  At one activation row the matmul is a weight stream
-// (about 1.6 flop per packed byte); the CUDA-core GEMV spends most of its
-// issue slots widening codes to fp32 and reducing across lanes, while here
-// every weight costs about two instructions and the accumulation is free.
+// the dequantization (about two instructions per weight, whatever the number
+// of activation rows).  At three or four rows the CUDA-core GEMV, which works
+// on pairs of rows, reads the weights twice and multiplies every weight by
+// every row on the CUDA cores; this kernel reads them once and the rows cost
+// tensor-core time only.  (At one or two rows the GEMV is faster: measured
+// 4.7 TB/s at one row against this kernel's 2.7.)
 //
 // Segmented-K tiles.  The MMA's 128 rows (tensor-memory lanes) are not 128
 // weight rows: a tile is R weight rows x `segs` segments of K (R * segs =
