@@ -746,11 +746,11 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   const int64_t rows = [&] { int64_t r = 0; for (int i = 0; i < count; ++i) r += probs[i].N; return r; }();
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, rows)));
   auto kern = gemv_kernel<MR, kThreads, NP>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static PerDeviceOnce attr_once;
+  if (attr_once.needed(dev.device)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_once.mark(dev.device);
   }
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, L);
 }

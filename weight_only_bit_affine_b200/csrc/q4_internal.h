@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 namespace q4 {
@@ -16,6 +17,15 @@ struct DeviceInfo {
 // Returns nullptr (and sets the error message) if the current device cannot
 // be queried.
 const DeviceInfo* current_device_info();
+
+// One bit per device ordinal (< 64) for settings that are made once per
+// kernel and device (cudaFuncSetAttribute applies to the current device).
+// Two threads may both make the setting; it is idempotent.
+struct PerDeviceOnce {
+  std::atomic<uint64_t> done{0};
+  bool needed(int device) const { return ((done.load(std::memory_order_acquire) >> device) & 1u) == 0; }
+  void mark(int device) { done.fetch_or(uint64_t(1) << device, std::memory_order_release); }
+};
 
 // Launchers return cudaSuccess or the launch error.  Arguments are already
 // validated by the ABI layer.

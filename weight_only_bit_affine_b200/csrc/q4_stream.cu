@@ -675,12 +675,12 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
   const size_t smem = kFixedSmem + b_bytes + static_cast<size_t>(stages) * stage_bytes;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, tiles)));
   auto kern = stream_kernel<NP>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static PerDeviceOnce attr_once;
+  if (attr_once.needed(dev.device)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(dev.smem_optin));
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_once.mark(dev.device);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));

@@ -486,15 +486,15 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
   p.idesc = make_idesc(bn);
   const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + barrier_bytes + 1024;
 
-  static bool attr_set = false;
-  if (!attr_set) {
+  static PerDeviceOnce attr_once;
+  if (attr_once.needed(dev.device)) {
     for (auto kern : {tc_kernel<1>, tc_kernel<2>}) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(dev.smem_optin));
       if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
       if (e != cudaSuccess) return e;
     }
-    attr_set = true;
+    attr_once.mark(dev.device);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(n_tiles), static_cast<unsigned>(m_tiles));
