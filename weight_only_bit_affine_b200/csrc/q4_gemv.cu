@@ -233,7 +233,7 @@ struct GemvLaunch {
 };
 
 constexpr int kRedSlots = 8;    // tiles of cross-warp partial sums in flight to the epilogue warp
-constexpr int kRedSlotFloats = 64 * 2;  // >= rt * MR * warps-per-team (rt * wpt <= 4 * 22)
+constexpr int kRedSlotFloats = 64 * 2;  // >= rt * MR * warps-per-team (<= 4 * 22 at MR = 1, 4 * 2 * 12 at MR = 2)
 
 // Shape of one problem for a given consumer count (host and device agree).
 struct Geometry {
@@ -668,17 +668,22 @@ cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStre
 }
 
 // Block shapes: consumers + producer warp + epilogue warp.  The thread
-// counts bound the registers (768 threads: 80 per thread; 416: 157).  One
-// activation row: 22 consumer warps -- teams of 4 warps for K = 4096 (five
-// teams), of 11 for K = 11264 (two teams), and enough warps in flight to hide
-// the shared-memory and dependency latencies of the dot products (measured:
-// 704 consumers stream the temporal step 30% faster than 512).
+// counts bound the registers (768 threads: 80 per thread; 448: 128 -- the
+// registers are split evenly over the SM's four schedulers, each holding at
+// most ceil(warps / 4) of the block's warps).  One activation row: 22
+// consumer warps -- teams of 4 warps for K = 4096 (five teams), of 11 for
+// K = 11264 (two teams), and enough warps in flight to hide the
+// shared-memory and dependency latencies of the dot products (measured: 704
+// consumers stream the temporal step 30% faster than 512; 24 consumer warps,
+// which need 72 registers, or a reduction by the team's last warp in place
+// of the epilogue warp, were 12-15% slower).  Two rows: 12 consumer warps,
+// three teams for K = 4096 (7% faster on a layer than 11 warps, two teams).
 #ifndef Q4_GEMV_CONSUMERS1
 #define Q4_GEMV_CONSUMERS1 704
 #endif
 constexpr int kConsumers1 = Q4_GEMV_CONSUMERS1, kThreads1 = kConsumers1 + 64;  // one activation row
 #ifndef Q4_GEMV_CONSUMERS2
-#define Q4_GEMV_CONSUMERS2 352
+#define Q4_GEMV_CONSUMERS2 384
 #endif
 constexpr int kConsumers2 = Q4_GEMV_CONSUMERS2, kThreads2 = kConsumers2 + 64;  // two activation rows
 
