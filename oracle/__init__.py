@@ -188,6 +188,63 @@ def matmul_ref_factored(x_bits, codes, scales, biases) -> np.ndarray:
     return y
 
 
+# --------------------------------------------------------------- output epilogues
+#
+# The projections feed the blocks the pages name as reused components of the
+# model (Swift/MLX blog, section "Reusing the Mimi codec": KV cache, RoPE,
+# SwiGLU, RMSNorm; GeekNews summary, "Arsitektur model dan konversi"): the
+# attention output and down projections add into the residual stream, and the
+# MLP's gate and up projections meet in SwiGLU, h = silu(gate) * up with
+# silu(z) = z * sigmoid(z).  The fused forms below take the exact products
+# from matmul_ref (the pinned product) as their step.
+
+SILU_LIPSCHITZ = 1.1  # bound on |d silu / dz| = |s(z) (1 + z (1 - s(z)))|, max 1.0998 near z = 2.40
+
+
+def silu(z) -> np.ndarray:
+    """silu(z) = z / (1 + e^-z) in binary64, elementwise (e^-z -> inf gives -0)."""
+    z = np.asarray(z, np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def matmul_residual_ref(x_bits, codes, scales, biases, r_bits, rows=None):
+    """y = r + x . W_hat^T in binary64 (r [M, N] bf16 bits, the residual stream).
+
+    Returns (y, bound): the per-element acceptance bound extends the product's
+    4e-3 * sum|x w_hat| + 1e-6 to the magnitude of the sum, 4e-3 * (sum|x w_hat|
+    + |r|) + 1e-6, since the one bf16 rounding of r + acc is relative to it.
+    """
+    y, ad = matmul_ref(x_bits, codes, scales, biases, rows=rows)
+    r = bf16_bits_to_f64(_c(r_bits, np.uint16))
+    if r.ndim == 1:
+        r = r[None, :]
+    if rows is not None:
+        r = r[:, np.asarray(rows, dtype=np.int64)]
+    return y + r, 4e-3 * (ad + np.abs(r)) + 1e-6
+
+
+def matmul_swiglu_ref(x_bits, gate, up, rows=None):
+    """h = silu(g) * u in binary64, g and u the exact products x . W_hat^T of
+    the gate and up weights ((codes, scales, biases) triples).
+
+    Returns (h, bound).  The bound carries the product bounds
+    T = 4e-3 * sum|x w_hat| + 1e-6 of g and u through h to first order:
+    |silu(g') u' - silu(g) u| <= L (|dg|) (|u| + Tu) + |silu(g)| Tu with
+    L = SILU_LIPSCHITZ, where |dg| <= Tg + 2^-8 (|g| + Tg) also covers a gate
+    stored as bf16 between two passes; then one bf16 rounding of h, relative
+    2^-8 of its magnitude (with margin over the 2^-9 of round-to-nearest).
+    """
+    g, adg = matmul_ref(x_bits, *gate, rows=rows)
+    u, adu = matmul_ref(x_bits, *up, rows=rows)
+    tg, tu = 4e-3 * adg + 1e-6, 4e-3 * adu + 1e-6
+    sg = silu(g)
+    dg = SILU_LIPSCHITZ * (tg + 2.0 ** -8 * (np.abs(g) + tg))
+    mag_u = np.abs(u) + tu
+    bound = dg * mag_u + np.abs(sg) * tu + 2.0 ** -8 * (np.abs(sg) + dg) * mag_u + 1e-6
+    return sg * u, bound
+
+
 def set_threads(n: int) -> None:
     """Threads of the oracle's OpenMP loops (timing only: results do not depend on it)."""
     _load().oq4_set_threads(int(n))
