@@ -287,6 +287,36 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
         per_proj[p.name.split(".")[1]] = {"us": round(t * 1e3, 2), "GBps": round(nb / (t * 1e-3) / 1e9, 1)}
     rows["temporal_layer_M1"]["per_projection_single_call"] = per_proj
 
+    # The same four layers with the block's element-wise steps fused into the
+    # matmuls: o and down each add into a residual stream in place (two
+    # streams: problems of one launch may not share an output), gate and up
+    # are one SwiGLU problem -- 6 problems, one launch per layer, same bytes.
+    resid = [[torch.zeros((1, 4096), dtype=torch.bfloat16, device=dev) for _ in range(2)] for _ in range(4)]
+    hs = [torch.empty((1, 11264), dtype=torch.bfloat16, device=dev) for _ in range(4)]
+
+    def fused_problems(l, ys, r, h):
+        byname = {p.name.split(".")[1]: (p, c, s, b, y) for (p, c, s, b), y in zip(l, ys)}
+        probs = [(x, *byname[n][1:4], byname[n][4]) for n in ("q", "k", "v")]
+        probs.append((x, *byname["o"][1:4], r[0], q4.Residual(r[0])))
+        _, gc, gs, gb, _ = byname["gate"]
+        _, uc, us, ub, _ = byname["up"]
+        probs.append((x, gc, gs, gb, h, q4.SwiGLU(uc, us, ub)))
+        probs.append((x_down, *byname["down"][1:4], r[1], q4.Residual(r[1])))
+        return probs
+
+    fused = [fused_problems(l, ys, r, h) for l, ys, r, h in zip(layer, ys1, resid, hs)]
+    n0 = q4.q4_debug_launch_count()
+    for probs in fused:
+        q4.q4_matmul_batch(probs)
+    fused_launches = (q4.q4_debug_launch_count() - n0) / 4
+    ms_f = _graph_ms(dev, lambda: [q4.q4_matmul_batch(p) for p in fused], 50) / 4
+    rows["temporal_layer_fused_M1"] = {
+        "us_per_layer": round(ms_f * 1e3, 2), "GBps": round(lbytes / (ms_f * 1e-3) / 1e9, 1),
+        "launches_per_layer": fused_launches, "bytes": lbytes,
+        "note": "q, k, v plain; o and down with the residual add (in place); gate and up as one SwiGLU problem "
+                "(silu(gate) * up in the GEMV epilogue); compare temporal_layer_M1, the 7 plain projections",
+    }
+
     # depformer: stacked [16 N, K] weights per projection, drawn and quantized on the GPU
     seed = workloads.seed_of("depformer_steps")
     steps = workloads.DEPFORMER_STEPS

@@ -33,7 +33,8 @@
  *    biases and y 2-byte aligned.  Row strides are implied by K (dense).
  *  - Sizes: 0 <= M, N; 32 <= K, K % 32 == 0.  M == 0 or N == 0 is a no-op.
  *    `group` must be 32.  K <= 2^24, N <= 2^40, M <= 2^31.
- *  - Output buffers must not overlap inputs.
+ *  - Output buffers must not overlap inputs (the one exception: a residual
+ *    operand may be the output buffer itself, see q4_matmul_residual).
  *  - Device: compute capability 10.0 (B200, sm_100a) only; any other device
  *    returns Q4_ERR_UNSUPPORTED.
  */
@@ -132,16 +133,74 @@ Q4_API q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K,
                          const q4_bf16* biases, int64_t N, int64_t num_steps,
                          int64_t step, int group, q4_bf16* y, q4_stream_t stream);
 
-/* One problem of q4_matmul_batch: pointers and sizes as for q4_matmul. */
+/*
+ * Output epilogues: a step of the feed-forward block that follows the
+ * matmul, fused into it so that the fp32 accumulator is rounded to bf16 once.
+ * The pages name the blocks these projections belong to (Swift/MLX blog,
+ * section "Reusing the Mimi codec": KV cache, RoPE, SwiGLU and RMSNorm are
+ * shared with the earlier ports; GeekNews summary, section "Arsitektur model
+ * dan konversi", likewise) and fuse per-step kernel dispatches (Swift/MLX
+ * blog, "Performance optimizations"); the fused forms are defined here.
+ *   Q4_EPI_NONE      y = acc
+ *   Q4_EPI_RESIDUAL  y = bf16(r + acc), r [M, N] bf16 (the residual stream;
+ *                    r may be y itself, an in-place update)
+ *   Q4_EPI_SWIGLU    y = bf16(silu(acc) * acc_up), silu(z) = z / (1 + e^-z),
+ *                    acc the gate projection's and acc_up the up
+ *                    projection's fp32 accumulators (weights of the same
+ *                    shape).  Where q4_matmul would run the CUDA-core GEMV
+ *                    both come from one pass that reads x and the two
+ *                    weights once per pair of activation rows; where it
+ *                    would run a tensor-core kernel, the gate result is
+ *                    stored in y as bf16 and the up pass reads it back, so
+ *                    silu sees the bf16-rounded gate.
+ */
+typedef enum { Q4_EPI_NONE = 0, Q4_EPI_RESIDUAL = 1, Q4_EPI_SWIGLU = 2 } q4_epilogue;
+
+/* One problem of q4_matmul_batch: pointers and sizes as for q4_matmul, plus
+ * an optional epilogue (all-zero fields mean Q4_EPI_NONE). */
 typedef struct {
   const q4_bf16* x;       /* [M, K] activations, 16-byte aligned   */
-  const uint8_t* codes;   /* [N, K/2], 16-byte aligned               */
+  const uint8_t* codes;   /* [N, K/2], 16-byte aligned (the gate for SWIGLU) */
   const q4_bf16* scales;  /* [N, K/32]                               */
   const q4_bf16* biases;  /* [N, K/32]                               */
   q4_bf16* y;             /* [M, N] output                           */
   int64_t N;
   int64_t K;
+  int32_t epilogue;       /* q4_epilogue                              */
+  int32_t reserved;       /* must be 0                                */
+  const q4_bf16* r;       /* RESIDUAL: [M, N], 2-byte aligned; else NULL */
+  const uint8_t* up_codes;   /* SWIGLU: up projection, as codes/scales/biases */
+  const q4_bf16* up_scales;
+  const q4_bf16* up_biases;
 } q4_matmul_desc;
+
+/*
+ * q4_matmul_residual -- y = bf16(r + x . w_hat^T), the sum taken in fp32
+ * before the one rounding: the attention output and down projections
+ * adding their result to the residual stream.  r [M, N] bf16, 2-byte
+ * aligned; r == y updates the stream in place; any other overlap of r and y
+ * is an error (Q4_ERR_SHAPE).  Same kernels, alignment and status codes as
+ * q4_matmul.
+ */
+Q4_API q4_status q4_matmul_residual(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes,
+                                    const q4_bf16* scales, const q4_bf16* biases, int64_t N, int group,
+                                    const q4_bf16* r, q4_bf16* y, q4_stream_t stream);
+
+/*
+ * q4_matmul_swiglu -- h = bf16(silu(x . w_hat_gate^T) * (x . w_hat_up^T)):
+ * the gate and up projections of the SwiGLU MLP and its activation in one
+ * call (Q4_EPI_SWIGLU above).  Both weights are [N, K] in the packed format
+ * with the same alignment rules as q4_matmul; h [M, N] must not overlap any
+ * input.  Kernels as q4_matmul chooses them for M: on the GEMV one pass
+ * (M = 1, 2: one launch reading each weight once); on a tensor-core kernel
+ * two passes (gate into h, then up with the silu-multiply epilogue reading
+ * h), one launch each.
+ */
+Q4_API q4_status q4_matmul_swiglu(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* gate_codes,
+                                  const q4_bf16* gate_scales, const q4_bf16* gate_biases,
+                                  const uint8_t* up_codes, const q4_bf16* up_scales,
+                                  const q4_bf16* up_biases, int64_t N, int group, q4_bf16* h,
+                                  q4_stream_t stream);
 
 /*
  * q4_matmul_batch -- `count` independent matmuls sharing the number of
@@ -155,8 +214,12 @@ typedef struct {
  * stream (every projection of a decode step) in one launch.
  * `descs` is a HOST array of `count` entries, read before the call returns.
  * The problems run concurrently: no output may overlap any input of any
- * problem in the list.  Validation covers every entry before anything is
- * enqueued; count == 0 is a no-op; count < 0 is Q4_ERR_SHAPE.
+ * problem in the list (a residual operand may be its own problem's output).
+ * Each entry's epilogue applies as in q4_matmul_residual / q4_matmul_swiglu;
+ * a SwiGLU entry on the two-pass path adds one launch for the up passes.
+ * Validation covers every entry before anything is enqueued; count == 0 is
+ * a no-op; count < 0 is Q4_ERR_SHAPE; an unknown epilogue or a nonzero
+ * `reserved` is Q4_ERR_UNSUPPORTED.
  */
 Q4_API q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int group,
                                  q4_stream_t stream);

@@ -36,7 +36,8 @@ def declared_symbols():
 
 def test_header_declares_the_entry_points():
     names = declared_symbols()
-    for n in ["q4_quantize", "q4_dequantize", "q4_matmul", "q4_matmul_step", "q4_last_error"]:
+    for n in ["q4_quantize", "q4_dequantize", "q4_matmul", "q4_matmul_step", "q4_matmul_residual",
+              "q4_matmul_swiglu", "q4_matmul_batch", "q4_last_error"]:
         assert n in names
 
 
@@ -97,6 +98,58 @@ def test_quantize_dequantize_validation(lib):
     assert lib.q4_dequantize(P, P, P, 4, 64, 8, P, None) == UNSUP
     assert lib.q4_dequantize(P, P, P, -1, 64, 32, P, None) == SHAPE
     assert lib.q4_dequantize(P, P + 1, P, 4, 64, 32, P, None) == ALIGN
+
+
+def test_residual_validation(lib):
+    res = lambda r=P, y=P, M=1, N=8: lib.q4_matmul_residual(P, M, 64, P, P, P, N, 32, r, y, None)
+    assert res(r=None) == NULL
+    assert b"residual" in lib.q4_last_error()
+    assert res(r=P + 1) == ALIGN
+    # r may be y itself, but no other overlap: [P + 2, P + 18) against [P, P + 16)
+    assert res(r=P + 2, y=P) == SHAPE
+    assert res(r=P, y=P + 2) == SHAPE
+    assert res(M=0) == OK
+
+
+def test_swiglu_validation(lib):
+    sw = lambda uc=P, us=P, ub=P, h=P: lib.q4_matmul_swiglu(P, 1, 64, P, P, P, uc, us, ub, 8, 32, h, None)
+    assert sw(uc=None) == NULL
+    assert sw(us=None) == NULL
+    assert sw(uc=P + 8) == ALIGN
+    assert sw(ub=P + 1) == ALIGN
+    assert sw(h=None) == NULL
+    assert lib.q4_matmul_swiglu(P, 1, 64, P, P, P, P, P, P, 8, 16, P, None) == UNSUP
+
+
+def test_batch_descriptor_validation(lib):
+    def one(**kw):
+        d = q4.MatmulDesc(P, P, P, P, P, 8, 64)
+        for k, v in kw.items():
+            setattr(d, k, v)
+        arr = (q4.MatmulDesc * 1)(d)
+        return lib.q4_matmul_batch(ctypes.cast(arr, ctypes.c_void_p), 1, 1, 32, None)
+
+    assert ctypes.sizeof(q4.MatmulDesc) == 96  # the C struct (include/q4.h) on LP64
+    assert one(epilogue=7) == UNSUP
+    assert b"epilogue" in lib.q4_last_error()
+    assert one(reserved=1) == UNSUP
+    assert one(epilogue=q4.EPI_RESIDUAL) == NULL  # r missing
+    assert one(epilogue=q4.EPI_RESIDUAL, r=P + 1) == ALIGN
+    assert one(epilogue=q4.EPI_SWIGLU, up_codes=P, up_scales=P) == NULL
+    assert one(epilogue=q4.EPI_SWIGLU, up_codes=P + 4, up_scales=P, up_biases=P) == ALIGN
+
+
+def test_descriptor_layout_matches_c(tmp_path):
+    src = tmp_path / "l.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "q4.h"\n'
+                   'int main(void){ printf("%zu %zu %zu %zu %zu", sizeof(q4_matmul_desc), '
+                   'offsetof(q4_matmul_desc, epilogue), offsetof(q4_matmul_desc, r), '
+                   'offsetof(q4_matmul_desc, up_codes), offsetof(q4_matmul_desc, up_biases)); return 0; }\n')
+    exe = tmp_path / "l"
+    subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
+    D = q4.MatmulDesc
+    assert got == [ctypes.sizeof(D), D.epilogue.offset, D.r.offset, D.up_codes.offset, D.up_biases.offset]
 
 
 def test_valid_call_without_gpu_reports_cuda_error(lib):

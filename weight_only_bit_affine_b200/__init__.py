@@ -12,6 +12,9 @@ come from PyTorch) and have the same names as the C entry points:
     W_hat = q4_dequantize(codes, scales, biases)        # [N, K] bf16
     y = q4_matmul(x, codes, scales, biases)             # x [M, K] -> y [M, N]
     y = q4_matmul_step(x, codes, scales, biases, num_steps, step)
+    y = q4_matmul_residual(x, codes, scales, biases, r)   # r + x . w_hat^T
+    h = q4_matmul_swiglu(x, (gc, gs, gb), (uc, us, ub))   # silu(gate) * up
+    q4_matmul_batch([(x, codes, scales, biases, y), ...]) # one launch per kernel path
 
 Layout (model card "personaplex-edge-q4", "Release details": affine Q4,
 group size 32, BF16): codes [N, K/2] uint8 (low nibble = even k), scales
@@ -21,7 +24,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Optional, Tuple
+from typing import NamedTuple, Optional, Tuple
 
 import torch
 
@@ -34,7 +37,11 @@ __all__ = [
     "q4_dequantize",
     "q4_matmul",
     "q4_matmul_step",
+    "q4_matmul_residual",
+    "q4_matmul_swiglu",
     "q4_matmul_batch",
+    "Residual",
+    "SwiGLU",
     "q4_debug_device_flags",
     "q4_debug_launch_count",
 ]
@@ -60,6 +67,8 @@ SIGNATURES = {
     "q4_dequantize": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),
     "q4_matmul": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P]),
     "q4_matmul_step": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P, _P]),
+    "q4_matmul_residual": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P, _P]),
+    "q4_matmul_swiglu": (_INT, [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I64, _INT, _P, _P]),
     "q4_matmul_batch": (_INT, [_P, _INT, _I64, _INT, _P]),
     "q4_last_error": (ctypes.c_char_p, []),
     "q4_debug_device_flags": (_INT, [_INT]),
@@ -67,10 +76,30 @@ SIGNATURES = {
 }
 
 
+EPI_NONE, EPI_RESIDUAL, EPI_SWIGLU = 0, 1, 2  # q4_epilogue
+
+
 class MatmulDesc(ctypes.Structure):
     """Mirror of q4_matmul_desc (include/q4.h)."""
 
-    _fields_ = [("x", _P), ("codes", _P), ("scales", _P), ("biases", _P), ("y", _P), ("N", _I64), ("K", _I64)]
+    _fields_ = [("x", _P), ("codes", _P), ("scales", _P), ("biases", _P), ("y", _P), ("N", _I64), ("K", _I64),
+                ("epilogue", ctypes.c_int32), ("reserved", ctypes.c_int32), ("r", _P), ("up_codes", _P),
+                ("up_scales", _P), ("up_biases", _P)]
+
+
+class Residual(NamedTuple):
+    """Batch epilogue: out = r + x . w_hat^T (r [M, N] bf16; may be out itself)."""
+
+    r: torch.Tensor
+
+
+class SwiGLU(NamedTuple):
+    """Batch epilogue: out = silu(x . w_hat^T) * (x . w_hat_up^T), the problem's
+    weights being the gate and these the up projection's."""
+
+    up_codes: torch.Tensor
+    up_scales: torch.Tensor
+    up_biases: torch.Tensor
 
 
 class Q4Error(RuntimeError):
@@ -219,12 +248,70 @@ def q4_matmul_step(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, b
     return out
 
 
+def _out(out, M, N, dev):
+    if out is None:
+        return torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _want(out, "out", torch.bfloat16, 2)
+    if out.shape != (M, N) or out.device != dev:
+        raise ValueError(f"out must be [{M}, {N}] on {dev}")
+    return out
+
+
+def _same_weights(codes, scales, biases, up, what):
+    uc, us, ub = up
+    _matmul_shapes_w(uc, us, ub, codes.shape[1] * 2, what)
+    if uc.shape != codes.shape or not (uc.device == us.device == ub.device == codes.device):
+        raise ValueError(f"{what}: the up weights must match the gate's shape and device")
+
+
+def _matmul_shapes_w(codes, scales, biases, K, what):
+    _want(codes, f"{what} codes", torch.uint8, 2)
+    _want(scales, f"{what} scales", torch.bfloat16, 2)
+    _want(biases, f"{what} biases", torch.bfloat16, 2)
+    if codes.shape[1] * 2 != K or scales.shape != (codes.shape[0], K // GROUP) or biases.shape != scales.shape:
+        raise ValueError(f"{what}: codes [N, K/2], scales and biases [N, K/32] with K = {K}")
+
+
+def q4_matmul_residual(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+                       r: torch.Tensor, group: int = GROUP, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = bf16(r + x . w_hat^T), summed in fp32; out=r updates r in place."""
+    M, K = _matmul_shapes(x, codes, scales, biases, None)
+    N = codes.shape[0]
+    dev = x.device
+    _want(r, "r", torch.bfloat16, 2)
+    if r.shape != (M, N) or r.device != dev:
+        raise ValueError(f"r must be [{M}, {N}] on {dev}")
+    out = _out(out, M, N, dev)
+    with torch.cuda.device(dev):
+        _check(lib().q4_matmul_residual(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N, group, _ptr(r),
+                                        _ptr(out), _stream(dev)))
+    return out
+
+
+def q4_matmul_swiglu(x: torch.Tensor, gate, up, group: int = GROUP,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """h = bf16(silu(x . w_hat_gate^T) * (x . w_hat_up^T)); gate and up are
+    (codes, scales, biases) triples of the same [N, K] shape."""
+    gc, gs, gb = gate
+    M, K = _matmul_shapes(x, gc, gs, gb, None)
+    _same_weights(gc, gs, gb, up, "up")
+    N = gc.shape[0]
+    dev = x.device
+    out = _out(out, M, N, dev)
+    uc, us, ub = up
+    with torch.cuda.device(dev):
+        _check(lib().q4_matmul_swiglu(_ptr(x), M, K, _ptr(gc), _ptr(gs), _ptr(gb), _ptr(uc), _ptr(us), _ptr(ub), N,
+                                      group, _ptr(out), _stream(dev)))
+    return out
+
+
 def q4_matmul_batch(problems, group: int = GROUP):
     """Independent matmuls in as few launches as possible.
 
     `problems`: a sequence of (x, codes, scales, biases, out) tuples, every x
-    with the same number of rows M; `out` [M, N] bf16 is written.  Returns the
-    list of outputs.
+    with the same number of rows M; `out` [M, N] bf16 is written.  A sixth
+    element Residual(r) or SwiGLU(up_codes, up_scales, up_biases) adds that
+    epilogue.  Returns the list of outputs.
     """
     problems = list(problems)
     if not problems:
@@ -232,7 +319,11 @@ def q4_matmul_batch(problems, group: int = GROUP):
     descs = (MatmulDesc * len(problems))()
     M = None
     dev = None
-    for i, (x, codes, scales, biases, out) in enumerate(problems):
+    for i, prob in enumerate(problems):
+        if len(prob) not in (5, 6):
+            raise ValueError(f"problem {i}: (x, codes, scales, biases, out[, epilogue])")
+        x, codes, scales, biases, out = prob[:5]
+        epi = prob[5] if len(prob) == 6 else None
         Mi, K = _matmul_shapes(x, codes, scales, biases, None)
         if M is None:
             M, dev = Mi, x.device
@@ -241,8 +332,21 @@ def q4_matmul_batch(problems, group: int = GROUP):
         _want(out, "out", torch.bfloat16, 2)
         if out.shape != (M, codes.shape[0]) or out.device != dev:
             raise ValueError(f"out of problem {i} must be [{M}, {codes.shape[0]}] on {dev}")
-        descs[i] = MatmulDesc(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
-                              codes.shape[0], K)
+        d = MatmulDesc(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
+                       codes.shape[0], K)
+        if isinstance(epi, Residual):
+            _want(epi.r, "r", torch.bfloat16, 2)
+            if epi.r.shape != out.shape or epi.r.device != dev:
+                raise ValueError(f"problem {i}: r must be [{M}, {codes.shape[0]}] on {dev}")
+            d.epilogue, d.r = EPI_RESIDUAL, epi.r.data_ptr()
+        elif isinstance(epi, SwiGLU):
+            _same_weights(codes, scales, biases, epi, f"problem {i} up")
+            d.epilogue = EPI_SWIGLU
+            d.up_codes, d.up_scales, d.up_biases = (epi.up_codes.data_ptr(), epi.up_scales.data_ptr(),
+                                                    epi.up_biases.data_ptr())
+        elif epi is not None:
+            raise TypeError(f"problem {i}: epilogue must be Residual or SwiGLU")
+        descs[i] = d
     with torch.cuda.device(dev):
         _check(lib().q4_matmul_batch(ctypes.cast(descs, ctypes.c_void_p), len(problems), M, group, _stream(dev)))
     return [p[4] for p in problems]

@@ -74,17 +74,108 @@ q4_status check_matmul(const char* who, const uint16_t* x, int64_t M, int64_t K,
   return Q4_OK;
 }
 
-q4_status matmul_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* codes, const uint16_t* scales,
-                      const uint16_t* biases, int64_t N, int group, uint16_t* y, cudaStream_t stream) {
+// Host checks of a problem's epilogue fields (q4.h, q4_epilogue); fills the
+// epilogue part of *a.
+q4_status check_epilogue(const char* who, int32_t epi, int32_t reserved, const uint16_t* r,
+                         const uint8_t* up_codes, const uint16_t* up_scales, const uint16_t* up_biases,
+                         MatmulArgs* a) {
+  if (reserved != 0) return fail(Q4_ERR_UNSUPPORTED, "%s: reserved field must be 0", who);
+  if (epi == Q4_EPI_NONE) return Q4_OK;
+  if (epi == Q4_EPI_RESIDUAL) {
+    if (!r) return fail(Q4_ERR_NULL, "%s: residual epilogue without its operand r", who);
+    if (!aligned(r, 2)) return fail(Q4_ERR_ALIGN, "%s: r must be 2-byte aligned", who);
+    const uintptr_t rb = reinterpret_cast<uintptr_t>(r), yb = reinterpret_cast<uintptr_t>(a->y);
+    const uintptr_t bytes = static_cast<uintptr_t>(a->M) * static_cast<uintptr_t>(a->N) * 2u;
+    if (rb != yb && rb < yb + bytes && yb < rb + bytes)
+      return fail(Q4_ERR_SHAPE, "%s: r overlaps y without being y", who);
+    a->epi = kEpiResidual;
+    a->r = r;
+    return Q4_OK;
+  }
+  if (epi == Q4_EPI_SWIGLU) {
+    if (!up_codes || !up_scales || !up_biases) return fail(Q4_ERR_NULL, "%s: SwiGLU without its up weights", who);
+    if (!aligned(up_codes, 16)) return fail(Q4_ERR_ALIGN, "%s: up codes must be 16-byte aligned", who);
+    if (!aligned(up_scales, 2) || !aligned(up_biases, 2))
+      return fail(Q4_ERR_ALIGN, "%s: up scales and biases must be 2-byte aligned", who);
+    a->up_codes = up_codes;
+    a->up_scales = up_scales;
+    a->up_biases = up_biases;
+    return Q4_OK;
+  }
+  return fail(Q4_ERR_UNSUPPORTED, "%s: unknown epilogue %d", who, static_cast<int>(epi));
+}
+
+// Enqueues a validated, non-empty list.  Each problem takes the kernel it
+// would take alone (so a batched result is bit-identical to the single
+// call); problems on the bulk-copy GEMV and on the weight-streaming kernel
+// share a launch per path.  A SwiGLU problem bound for a tensor-core kernel
+// becomes two problems: the gate into y, then the up projection with the
+// silu-multiply epilogue reading y, enqueued after every first pass.
+q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& dev, cudaStream_t cs,
+                       const char* what) {
+  std::vector<MatmulArgs> gemv, streamed, tc, streamed_up, tc_up;
+  for (const MatmulArgs& a : list) {
+    if (a.fused()) {
+      MatmulArgs g = a, u = a;
+      g.up_codes = u.up_codes = nullptr;
+      g.up_scales = u.up_scales = nullptr;
+      g.up_biases = u.up_biases = nullptr;
+      u.codes = a.up_codes;
+      u.scales = a.up_scales;
+      u.biases = a.up_biases;
+      u.epi = kEpiSiluMul;
+      u.r = a.y;
+      if (stream_supported(g, dev) && stream_supported(u, dev)) {
+        streamed.push_back(g);
+        streamed_up.push_back(u);
+      } else if (a.M >= kTensorCoreMinRows && tc_supported(g) && tc_supported(u)) {
+        tc.push_back(g);
+        tc_up.push_back(u);
+      } else {
+        gemv.push_back(a);
+      }
+    } else if (stream_supported(a, dev)) {
+      streamed.push_back(a);
+    } else if (a.M >= kTensorCoreMinRows && tc_supported(a)) {
+      tc.push_back(a);
+    } else {
+      gemv.push_back(a);
+    }
+  }
+  q4_status st = Q4_OK;
+  for (const MatmulArgs& a : tc)
+    if ((st = from_cuda(launch_tc(a, cs, dev), what)) != Q4_OK) return st;
+  if (!streamed.empty() &&
+      (st = from_cuda(launch_stream_batch(streamed.data(), static_cast<int>(streamed.size()), cs, dev), what)) != Q4_OK)
+    return st;
+  if (!gemv.empty() &&
+      (st = from_cuda(launch_gemv_batch(gemv.data(), static_cast<int>(gemv.size()), cs, dev), what)) != Q4_OK)
+    return st;
+  if (!streamed_up.empty() &&
+      (st = from_cuda(launch_stream_batch(streamed_up.data(), static_cast<int>(streamed_up.size()), cs, dev), what)) !=
+          Q4_OK)
+    return st;
+  for (const MatmulArgs& a : tc_up)
+    if ((st = from_cuda(launch_tc(a, cs, dev), what)) != Q4_OK) return st;
+  return Q4_OK;
+}
+
+// One matmul with an epilogue (q4_matmul, q4_matmul_step, q4_matmul_residual,
+// q4_matmul_swiglu).
+q4_status matmul_impl(const char* who, const uint16_t* x, int64_t M, int64_t K, const uint8_t* codes,
+                      const uint16_t* scales, const uint16_t* biases, int64_t N, int group, uint16_t* y,
+                      int32_t epi, const uint16_t* r, const uint8_t* up_codes, const uint16_t* up_scales,
+                      const uint16_t* up_biases, cudaStream_t stream) {
   bool empty = false;
-  q4_status st = check_matmul("q4_matmul", x, M, K, codes, scales, biases, N, group, y, &empty);
+  q4_status st = check_matmul(who, x, M, K, codes, scales, biases, N, group, y, &empty);
   if (st != Q4_OK || empty) return st;
+  MatmulArgs a{x, codes, scales, biases, y, M, N, K};
+  if ((st = check_epilogue(who, epi, 0, r, up_codes, up_scales, up_biases, &a)) != Q4_OK) return st;
   const DeviceInfo* dev = nullptr;
   if ((st = check_device(&dev)) != Q4_OK) return st;
-  MatmulArgs a{x, codes, scales, biases, y, M, N, K};
-  if (stream_supported(a, *dev)) return from_cuda(launch_stream_batch(&a, 1, stream, *dev), "q4_matmul launch");
-  if (M >= kTensorCoreMinRows && tc_supported(a)) return from_cuda(launch_tc(a, stream, *dev), "q4_matmul launch");
-  return from_cuda(launch_gemv(a, stream, *dev), "q4_matmul launch");
+  char what[64];
+  snprintf(what, sizeof what, "%s launch", who);
+  return run_problems(std::vector<MatmulArgs>{a}, *dev, stream, what);
 }
 
 }  // namespace
@@ -165,7 +256,23 @@ q4_status q4_dequantize(const uint8_t* codes, const q4_bf16* scales, const q4_bf
 
 q4_status q4_matmul(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes, const q4_bf16* scales,
                     const q4_bf16* biases, int64_t N, int group, q4_bf16* y, q4_stream_t stream) {
-  return matmul_impl(x, M, K, codes, scales, biases, N, group, y, reinterpret_cast<cudaStream_t>(stream));
+  return matmul_impl("q4_matmul", x, M, K, codes, scales, biases, N, group, y, Q4_EPI_NONE, nullptr, nullptr,
+                     nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+q4_status q4_matmul_residual(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes, const q4_bf16* scales,
+                             const q4_bf16* biases, int64_t N, int group, const q4_bf16* r, q4_bf16* y,
+                             q4_stream_t stream) {
+  return matmul_impl("q4_matmul_residual", x, M, K, codes, scales, biases, N, group, y, Q4_EPI_RESIDUAL, r, nullptr,
+                     nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+q4_status q4_matmul_swiglu(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* gate_codes,
+                           const q4_bf16* gate_scales, const q4_bf16* gate_biases, const uint8_t* up_codes,
+                           const q4_bf16* up_scales, const q4_bf16* up_biases, int64_t N, int group, q4_bf16* h,
+                           q4_stream_t stream) {
+  return matmul_impl("q4_matmul_swiglu", x, M, K, gate_codes, gate_scales, gate_biases, N, group, h, Q4_EPI_SWIGLU,
+                     nullptr, up_codes, up_scales, up_biases, reinterpret_cast<cudaStream_t>(stream));
 }
 
 q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes, const q4_bf16* scales,
@@ -178,8 +285,9 @@ q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* 
   if (N < 0) return fail(Q4_ERR_SHAPE, "negative N = %lld", (long long)N);
   if (!codes || !scales || !biases) return fail(Q4_ERR_NULL, "q4_matmul_step: NULL pointer argument");
   const int64_t row0 = step * N;
-  return matmul_impl(x, M, K, codes + row0 * (K / 2), scales + row0 * (K / 32), biases + row0 * (K / 32), N, group,
-                     y, reinterpret_cast<cudaStream_t>(stream));
+  return matmul_impl("q4_matmul_step", x, M, K, codes + row0 * (K / 2), scales + row0 * (K / 32),
+                     biases + row0 * (K / 32), N, group, y, Q4_EPI_NONE, nullptr, nullptr, nullptr, nullptr,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int group, q4_stream_t stream) {
@@ -195,31 +303,16 @@ q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int
     snprintf(who, sizeof who, "q4_matmul_batch[%d]", i);
     q4_status st = check_matmul(who, d.x, M, d.K, d.codes, d.scales, d.biases, d.N, group, d.y, &empty);
     if (st != Q4_OK) return st;
-    if (!empty) list.push_back(MatmulArgs{d.x, d.codes, d.scales, d.biases, d.y, M, d.N, d.K});
+    MatmulArgs a{d.x, d.codes, d.scales, d.biases, d.y, M, d.N, d.K};
+    if ((st = check_epilogue(who, d.epilogue, d.reserved, d.r, d.up_codes, d.up_scales, d.up_biases, &a)) != Q4_OK)
+      return st;
+    if (!empty) list.push_back(a);
   }
   if (list.empty()) return Q4_OK;
   const DeviceInfo* dev = nullptr;
   q4_status st;
   if ((st = check_device(&dev)) != Q4_OK) return st;
-  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  // Each problem takes the path it would take alone, so a batched result is
-  // bit-identical to the single call.
-  std::vector<MatmulArgs> gemv, streamed;
-  for (const MatmulArgs& a : list) {
-    if (stream_supported(a, *dev)) {
-      streamed.push_back(a);
-    } else if (a.M >= kTensorCoreMinRows && tc_supported(a)) {
-      if ((st = from_cuda(launch_tc(a, cs, *dev), "q4_matmul_batch launch")) != Q4_OK) return st;
-    } else {
-      gemv.push_back(a);
-    }
-  }
-  if (!streamed.empty() &&
-      (st = from_cuda(launch_stream_batch(streamed.data(), static_cast<int>(streamed.size()), cs, *dev),
-                      "q4_matmul_batch launch")) != Q4_OK)
-    return st;
-  if (gemv.empty()) return Q4_OK;
-  return from_cuda(launch_gemv_batch(gemv.data(), static_cast<int>(gemv.size()), cs, *dev), "q4_matmul_batch launch");
+  return run_problems(list, *dev, reinterpret_cast<cudaStream_t>(stream), "q4_matmul_batch launch");
 }
 
 const char* q4_last_error(void) { return t_last_error; }

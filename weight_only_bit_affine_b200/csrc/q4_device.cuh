@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "q4_internal.h"
+
 namespace q4 {
 
 // Set (never cleared by kernels) when a bounded wait gives up.  Each
@@ -128,6 +130,18 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // ---- bf16 helpers -------------------------------------------------------------
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
   return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
+// ---- output epilogues (kEpi* in q4_internal.h) ----------------------------------
+// silu(z) = z * sigmoid(z) = z / (1 + e^-z); e^-z overflows to +inf for very
+// negative z, giving the correct limit -0.
+__device__ __forceinline__ float silu_f32(float z) { return z / (1.f + expf(-z)); }
+
+__device__ __forceinline__ uint16_t epilogue_bf16(float acc, int epi, const uint16_t* r, int64_t idx) {
+  if (epi == kEpiResidual) return float_to_bf16_bits(acc + bf16_bits_to_float(r[idx]));
+  if (epi == kEpiSiluMul) return float_to_bf16_bits(silu_f32(bf16_bits_to_float(r[idx])) * acc);
+  return float_to_bf16_bits(acc);
 }
 
 // Four codes of a packed word -> bf16x2 (128 + q[t], 128 + q[t + 4]).  0x4300

@@ -26,6 +26,10 @@
 //    codes) and multiplied with bf16 x by fma.rn.f32.bf16 (exact products,
 //    fp32 accumulation); the offset is removed per group exactly:
 //    s*sum x(128+q) + (b - 128 s)*sum x.
+//  * Output epilogues (residual add; SwiGLU, whose tiles carry the gate rows
+//    and then the same rows of the up weight, paired by the epilogue warp)
+//    are compiled into a separate instantiation that only launches holding
+//    such problems use.
 //  * Programmatic dependent launch: before waiting for the previous kernel a
 //    launch only prefetches its first weight tiles into L2 (a hint, no effect
 //    on values); everything that reads memory another kernel may write comes
@@ -199,7 +203,6 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[V], int lane) {
 constexpr int pow2_at_least(int v) { return v <= 1 ? 1 : 2 * pow2_at_least((v + 1) / 2); }
 constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
 
-__device__ __forceinline__ uint16_t to_bf16_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 
 
 // Problems per launch: their descriptors travel in the kernel parameters
@@ -217,9 +220,16 @@ struct GemvProblem {
   const uint16_t* scales;  // [N, K/32]
   const uint16_t* biases;  // [N, K/32]
   uint16_t* y;             // [MR, y_ld]
+  const uint16_t* r;       // residual [MR, y_ld] (kEpiResidual), else NULL
+  // SwiGLU in one pass: the up projection's weights (NULL otherwise).  A
+  // tile then carries rt/2 gate rows followed by the same rows of up, and
+  // the epilogue warp writes silu(gate) * up.
+  const uint8_t* up_codes;
+  const uint16_t* up_scales;
+  const uint16_t* up_biases;
   int64_t N, y_ld;
   int64_t byte_begin;      // packed bytes of all earlier problems in the list
-  int32_t K, pad_;
+  int32_t K, epi;
 };
 
 template <int NP>
@@ -258,6 +268,39 @@ __host__ __device__ inline Geometry geometry_of(int K, int consumer_threads) {
   return g;
 }
 __host__ __device__ inline int64_t packed_row_bytes(int K) { return K / 2 + (K / 32) * 4; }
+__host__ __device__ inline bool is_fused(const GemvProblem& P) { return P.up_codes != nullptr; }
+// Packed bytes per output row (gate + up when fused).
+__host__ __device__ inline int64_t problem_row_bytes(const GemvProblem& P) {
+  return packed_row_bytes(P.K) * (is_fused(P) ? 2 : 1);
+}
+// Does the problem's tile finish in the epilogue warp (sums across a team's
+// warps, or the pairing of gate and up rows)?
+__host__ __device__ inline bool uses_epilogue_warp(const GemvProblem& P, const Geometry& g) {
+  return g.wpt > 1 || (is_fused(P) && g.wpt >= 1);
+}
+
+// Kernel-side views of the above.  A launch whose problems have no epilogue
+// runs the EPI = false instantiation, where they fold to the plain matmul's
+// constants and the epilogue code is compiled out of the hot loop (keeping it
+// there cost the plain stream 4 %).
+template <bool EPI>
+__device__ __forceinline__ bool fused_k(const GemvProblem& P) {
+  if constexpr (EPI) return is_fused(P);
+  return false;
+}
+template <bool EPI>
+__device__ __forceinline__ int rtile_k(const GemvProblem& P, const Geometry& g) {
+  return fused_k<EPI>(P) ? g.rt / 2 : g.rt;
+}
+template <bool EPI>
+__device__ __forceinline__ bool epilogue_warp_k(const GemvProblem& P, const Geometry& g) {
+  return g.wpt > 1 || (fused_k<EPI>(P) && g.wpt >= 1);
+}
+template <bool EPI>
+__device__ __forceinline__ uint16_t store_k(float v, const GemvProblem& P, int64_t idx) {
+  if constexpr (EPI) return epilogue_bf16(v, P.epi, P.r, idx);
+  return float_to_bf16_bits(v);
+}
 
 __device__ __forceinline__ uint32_t tile_rows(int64_t r_end, int64_t row0, int rt) {
   return static_cast<uint32_t>((r_end - row0 < rt) ? (r_end - row0) : rt);
@@ -270,16 +313,16 @@ __device__ __forceinline__ uint32_t tile_rows(int64_t r_end, int64_t row0, int r
 // the list is split (results do not depend on batching) and each row of the
 // list belongs to exactly one CTA.  Returns false when the problem lies
 // entirely after the range (the caller stops scanning).
-template <int NP>
+template <bool EPI, int NP>
 __device__ __forceinline__ bool segment_of(const GemvLaunch<NP>& L, int pi, int64_t lo, int64_t hi, int64_t* r0,
                                            int64_t* r1) {
   const GemvProblem& P = L.prob[pi];
-  const int64_t rb = packed_row_bytes(P.K);
+  const int64_t rb = packed_row_bytes(P.K) * (fused_k<EPI>(P) ? 2 : 1);
   const int64_t pb = P.byte_begin, pe = pb + P.N * rb;
   *r0 = *r1 = 0;
   if (pb >= hi) return false;
   if (pe <= lo) return true;
-  const int64_t rt = geometry_of(P.K, L.consumer_threads).rt;
+  const int64_t rt = rtile_k<EPI>(P, geometry_of(P.K, L.consumer_threads));
   const int64_t a = (lo > pb ? lo : pb) - pb, b = (hi < pe ? hi : pe) - pb;
   *r0 = ((a + rb - 1) / rb + rt - 1) / rt * rt;
   *r1 = ((b + rb - 1) / rb + rt - 1) / rt * rt;
@@ -288,7 +331,7 @@ __device__ __forceinline__ bool segment_of(const GemvLaunch<NP>& L, int pi, int6
   return true;
 }
 
-template <int MR, int MAXT, int NP>
+template <int MR, int MAXT, int NP, bool EPI>
 __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ GemvLaunch<NP> L) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int V = kRpt * MR;
@@ -328,15 +371,21 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         int64_t r0, r1;
         int issued = 0;
         for (int pi = 0; pi < L.count && issued < L.stages; ++pi) {
-          if (!segment_of(L, pi, lo, hi, &r0, &r1)) break;
+          if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
           const GemvProblem& P = L.prob[pi];
           const Geometry geo = geometry_of(P.K, L.consumer_threads);
           const int half_k = P.K >> 1;
-          for (int64_t row0 = r0; row0 < r1 && issued < L.stages; row0 += geo.rt, ++issued) {
-            const uint32_t rows = tile_rows(r1, row0, geo.rt);
+          const int rtile = rtile_k<EPI>(P, geo);
+          for (int64_t row0 = r0; row0 < r1 && issued < L.stages; row0 += rtile, ++issued) {
+            const uint32_t rows = tile_rows(r1, row0, rtile);
             bulk_prefetch_l2(P.codes + row0 * half_k, rows * half_k);
             bulk_prefetch_l2(P.scales + row0 * geo.G, rows * geo.G * 2);
             bulk_prefetch_l2(P.biases + row0 * geo.G, rows * geo.G * 2);
+            if (fused_k<EPI>(P)) {
+              bulk_prefetch_l2(P.up_codes + row0 * half_k, rows * half_k);
+              bulk_prefetch_l2(P.up_scales + row0 * geo.G, rows * geo.G * 2);
+              bulk_prefetch_l2(P.up_biases + row0 * geo.G, rows * geo.G * 2);
+            }
           }
         }
       }
@@ -347,12 +396,13 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       bool dead = false;
       for (int pi = 0; pi < L.count && !dead; ++pi) {
         int64_t r0, r1;
-        if (!segment_of(L, pi, lo, hi, &r0, &r1)) break;
+        if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
         if (r0 >= r1) continue;
         const GemvProblem& P = L.prob[pi];
         const Geometry geo = geometry_of(P.K, L.consumer_threads);
         const int half_k = P.K >> 1;
-        for (int64_t row0 = r0 - geo.rt; row0 < r1; row0 += geo.rt) {  // first pass: x
+        const int rtile = rtile_k<EPI>(P, geo);
+        for (int64_t row0 = r0 - rtile; row0 < r1; row0 += rtile) {  // first pass: x
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; break; }
           uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
           if (row0 < r0) {
@@ -360,14 +410,24 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
             mbar_arrive_expect_tx(&full_bar[stage], xbytes);
             bulk_g2s(st, P.x, xbytes, &full_bar[stage]);
           } else {
-            const uint32_t rows = tile_rows(r1, row0, geo.rt);
+            // Stage layout: codes of the tile's rows from 0, scales from
+            // sb_off, biases from sb_off + sb_tile; a fused tile puts the up
+            // rows right after the gate rows in each of the three regions
+            // (2 * rows <= rt, and every offset stays a multiple of 16 bytes).
+            const uint32_t rows = tile_rows(r1, row0, rtile);
             const uint32_t cb = rows * half_k, sb = rows * geo.G * 2;
             const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
             const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
-            mbar_arrive_expect_tx(&full_bar[stage], cb + 2 * sb);
+            const bool fused = fused_k<EPI>(P);
+            mbar_arrive_expect_tx(&full_bar[stage], (fused ? 2u : 1u) * (cb + 2 * sb));
             bulk_g2s(st, P.codes + row0 * half_k, cb, &full_bar[stage]);
             bulk_g2s(st + sb_off, P.scales + row0 * geo.G, sb, &full_bar[stage]);
             bulk_g2s(st + sb_off + sb_tile, P.biases + row0 * geo.G, sb, &full_bar[stage]);
+            if (fused) {
+              bulk_g2s(st + cb, P.up_codes + row0 * half_k, cb, &full_bar[stage]);
+              bulk_g2s(st + sb_off + sb, P.up_scales + row0 * geo.G, sb, &full_bar[stage]);
+              bulk_g2s(st + sb_off + sb_tile + sb, P.up_biases + row0 * geo.G, sb, &full_bar[stage]);
+            }
           }
           ++issued;
           if (++stage == L.stages) { stage = 0; phase ^= 1u; }
@@ -393,26 +453,29 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     bool dead = false;
     for (int pi = 0; pi < L.count; ++pi) {
       int64_t r0, r1;
-      if (!segment_of(L, pi, lo, hi, &r0, &r1)) break;
+      if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
       const GemvProblem& P = L.prob[pi];
       const Geometry geo = geometry_of(P.K, L.consumer_threads);
-      if (geo.wpt <= 1) continue;
-      for (int64_t row0 = r0; row0 < r1; row0 += geo.rt) {
+      if (!epilogue_warp_k<EPI>(P, geo)) continue;
+      const int rtile = rtile_k<EPI>(P, geo);
+      const bool fused = fused_k<EPI>(P);
+      for (int64_t row0 = r0; row0 < r1; row0 += rtile) {
         if (!dead && !mbar_wait(&rfull_bar[slot], sph)) dead = true;
-        const int n_out = static_cast<int>(tile_rows(r1, row0, geo.rt)) * MR;
+        // Slot entry ((row * MR + m) * wpt + warp) holds one warp's partial
+        // sum of the tile's row; a fused tile's up rows follow its n gate rows.
+        const int n = static_cast<int>(tile_rows(r1, row0, rtile));
         const float* rs = red + slot * kRedSlotFloats;
-        if (lane < n_out) {
+        for (int i = lane; i < n * MR; i += 32) {
+          const int lr = i / MR, m = i - lr * MR;
           float v = 0.f;
-          for (int w = 0; w < geo.wpt; ++w) v += rs[lane * geo.wpt + w];
-          const int lr = lane / MR, m = lane - lr * MR;
-          P.y[static_cast<int64_t>(m) * P.y_ld + row0 + lr] = to_bf16_bits(v);
-        }
-        if (n_out > 32) {  // MR * rt rows beyond one per lane
-          for (int i = lane + 32; i < n_out; i += 32) {
-            float v = 0.f;
-            for (int w = 0; w < geo.wpt; ++w) v += rs[i * geo.wpt + w];
-            const int lr = i / MR, m = i - lr * MR;
-            P.y[static_cast<int64_t>(m) * P.y_ld + row0 + lr] = to_bf16_bits(v);
+          for (int w = 0; w < geo.wpt; ++w) v += rs[i * geo.wpt + w];
+          const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row0 + lr;
+          if (fused) {
+            float u = 0.f;
+            for (int w = 0; w < geo.wpt; ++w) u += rs[(i + n * MR) * geo.wpt + w];
+            P.y[idx] = float_to_bf16_bits(silu_f32(v) * u);
+          } else {
+            P.y[idx] = store_k<EPI>(v, P, idx);
           }
         }
         __syncwarp();
@@ -431,7 +494,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   bool dead = false;
   for (int pi = 0; pi < L.count; ++pi) {
     int64_t r_begin, r_end;
-    if (!segment_of(L, pi, lo, hi, &r_begin, &r_end)) break;
+    if (!segment_of<EPI>(L, pi, lo, hi, &r_begin, &r_end)) break;
     if (r_begin >= r_end) continue;
     const GemvProblem& P = L.prob[pi];
     const Geometry geo = geometry_of(P.K, L.consumer_threads);
@@ -467,17 +530,20 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     if (lane == 0) mbar_arrive(&empty_bar[stage]);
     if (++stage == L.stages) { stage = 0; phase ^= 1u; }
 
-    const bool use_red = geo.wpt > 1;
+    const bool use_red = epilogue_warp_k<EPI>(P, geo);
+    const int rtile = rtile_k<EPI>(P, geo);
     constexpr float kOffset = mac_offset<Q4_GEMV_MAC>();
 
-    for (int64_t row0 = r_begin; row0 < r_end; row0 += geo.rt) {
+    for (int64_t row0 = r_begin; row0 < r_end; row0 += rtile) {
       if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
       const uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
       // Rows of this tile are dealt to the teams round-robin (row r goes to
       // team r % teams), so a short last tile stays balanced; when a team
       // spans whole warps the row count below is warp-uniform and idle warps
-      // skip the arithmetic entirely.
-      const int tile_n = static_cast<int>((r_end - row0 < geo.rt) ? (r_end - row0) : geo.rt);
+      // skip the arithmetic entirely.  A fused tile of n output rows holds
+      // 2n weight rows (gate rows, then up rows), all computed alike.
+      const int tile_out = static_cast<int>((r_end - row0 < rtile) ? (r_end - row0) : rtile);
+      const int tile_n = fused_k<EPI>(P) ? 2 * tile_out : tile_out;
       const int nv = (team_idx >= geo.teams || team_idx >= tile_n) ? 0
                      : (tile_n == geo.rt)                          ? kRpt
                                                                    : (tile_n - team_idx + geo.teams - 1) / geo.teams;
@@ -574,7 +640,8 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
           if (holder) {
             const int lr = team_idx + rr * geo.teams;  // row within the tile
             if (!use_red) {
-              P.y[static_cast<int64_t>(m) * P.y_ld + row0 + lr] = to_bf16_bits(tot);
+              const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row0 + lr;
+              P.y[idx] = store_k<EPI>(tot, P, idx);
             } else {
               rs[(lr * MR + m) * geo.wpt + warp_in_team] = tot;
             }
@@ -594,8 +661,10 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
             if (rr < nv) {
               const int64_t row = row0 + team_idx + rr * geo.teams;
 #pragma unroll
-              for (int m = 0; m < MR; ++m)
-                P.y[static_cast<int64_t>(m) * P.y_ld + row] = to_bf16_bits(vals[rr * MR + m]);
+              for (int m = 0; m < MR; ++m) {
+                const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row;
+                P.y[idx] = store_k<EPI>(vals[rr * MR + m], P, idx);
+              }
             }
         }
       }
@@ -605,15 +674,45 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 
 // Generic path: any K, any 2-byte-aligned scales.  One warp per weight row,
 // lanes stride over the row's groups; x is read through the L1 per group.
+// A fused (SwiGLU) problem computes the gate and the up row of each output.
 struct GenericParams {
   const uint16_t* x;
   const uint8_t* codes;
   const uint16_t* scales;
   const uint16_t* biases;
   uint16_t* y;
+  const uint16_t* r;  // residual, or NULL
+  const uint8_t* up_codes;  // SwiGLU up weights, or NULL
+  const uint16_t* up_scales;
+  const uint16_t* up_biases;
   int64_t N, y_ld;
-  int K, G;
+  int K, G, epi;
 };
+
+// This lane's share of row `row` of one weight: sum over its groups of
+// x * w_hat, per activation row.
+template <int MR>
+__device__ __forceinline__ void generic_row_dot(const GenericParams& p, const uint8_t* codes, const uint16_t* scales,
+                                                const uint16_t* biases, int64_t row, int lane, float (&acc)[MR]) {
+#pragma unroll
+  for (int m = 0; m < MR; ++m) acc[m] = 0.f;
+  for (int g = lane; g < p.G; g += 32) {
+    const uint4 c4 = ld_nc_v4(codes + row * (p.K / 2) + static_cast<int64_t>(g) * 16);
+    const uint32_t words[4] = {c4.x, c4.y, c4.z, c4.w};
+    const float s = bf16_bits_to_float(scales[row * p.G + g]);
+    const float b = bf16_bits_to_float(biases[row * p.G + g]);
+    XSlice<4, kMacMixedBf16> xs[MR];
+#pragma unroll
+    for (int m = 0; m < MR; ++m) xs[m].load(p.x + static_cast<int64_t>(m) * p.K + g * 32);
+    float a0[MR], a1[MR];
+#pragma unroll
+    for (int m = 0; m < MR; ++m) a0[m] = a1[m] = 0.f;
+    dot_plus128<MR, 4, kMacMixedBf16>(words, xs, a0, a1);
+    const float c = fmaf(-128.f, s, b);
+#pragma unroll
+    for (int m = 0; m < MR; ++m) acc[m] += fmaf(s, a0[m] + a1[m], c * xs[m].sum);
+  }
+}
 
 template <int MR>
 __global__ void __launch_bounds__(256) gemv_generic_kernel(const __grid_constant__ GenericParams p) {
@@ -623,28 +722,22 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(const __grid_constant
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp; row < p.N; row += warps_total) {
     float acc[MR];
+    generic_row_dot<MR>(p, p.codes, p.scales, p.biases, row, lane, acc);
+    if (p.up_codes != nullptr) {
+      float up[MR];
+      generic_row_dot<MR>(p, p.up_codes, p.up_scales, p.up_biases, row, lane, up);
 #pragma unroll
-    for (int m = 0; m < MR; ++m) acc[m] = 0.f;
-    for (int g = lane; g < p.G; g += 32) {
-      const uint4 c4 = ld_nc_v4(p.codes + row * (p.K / 2) + static_cast<int64_t>(g) * 16);
-      const uint32_t words[4] = {c4.x, c4.y, c4.z, c4.w};
-      const float s = bf16_bits_to_float(p.scales[row * p.G + g]);
-      const float b = bf16_bits_to_float(p.biases[row * p.G + g]);
-      XSlice<4, kMacMixedBf16> xs[MR];
-#pragma unroll
-      for (int m = 0; m < MR; ++m) xs[m].load(p.x + static_cast<int64_t>(m) * p.K + g * 32);
-      float a0[MR], a1[MR];
-#pragma unroll
-      for (int m = 0; m < MR; ++m) a0[m] = a1[m] = 0.f;
-      dot_plus128<MR, 4, kMacMixedBf16>(words, xs, a0, a1);
-      const float c = fmaf(-128.f, s, b);
-#pragma unroll
-      for (int m = 0; m < MR; ++m) acc[m] += fmaf(s, a0[m] + a1[m], c * xs[m].sum);
+      for (int m = 0; m < MR; ++m) {
+        const float g = seg_allreduce<32>(acc[m]), u = seg_allreduce<32>(up[m]);
+        if (lane == 0) p.y[static_cast<int64_t>(m) * p.y_ld + row] = float_to_bf16_bits(silu_f32(g) * u);
+      }
+      continue;
     }
 #pragma unroll
     for (int m = 0; m < MR; ++m) {
       const float v = seg_allreduce<32>(acc[m]);
-      if (lane == 0) p.y[static_cast<int64_t>(m) * p.y_ld + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+      const int64_t idx = static_cast<int64_t>(m) * p.y_ld + row;
+      if (lane == 0) p.y[idx] = epilogue_bf16(v, p.epi, p.r, idx);
     }
   }
 }
@@ -693,8 +786,13 @@ int consumers_for(int mr) { return mr == 1 ? kConsumers1 : kConsumers2; }
 bool tma_ok(const MatmulArgs& a, int mr) {
   const int64_t G = a.K / 32;
   if (G % 8 != 0) return false;  // scale rows must be whole 16-byte runs for bulk copies
-  if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) return false;
+  uintptr_t sb = reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases);
+  if (a.fused()) sb |= reinterpret_cast<uintptr_t>(a.up_scales) | reinterpret_cast<uintptr_t>(a.up_biases);
+  if (sb & 15u) return false;
   const Geometry geo = geometry_of(static_cast<int>(a.K), consumers_for(mr));
+  // A fused tile pairs gate and up rows in the epilogue warp, which needs
+  // teams of whole warps.
+  if (a.fused() && geo.team < 32) return false;
   return geo.teams >= 1 && geo.team <= consumers_for(mr);
 }
 
@@ -706,10 +804,15 @@ cudaError_t run_generic(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, 
   p.scales = a.scales;
   p.biases = a.biases;
   p.y = a.y + m0 * a.N;
+  p.r = a.r ? a.r + m0 * a.N : nullptr;
+  p.up_codes = a.up_codes;
+  p.up_scales = a.up_scales;
+  p.up_biases = a.up_biases;
   p.N = a.N;
   p.y_ld = a.N;
   p.K = static_cast<int>(a.K);
   p.G = static_cast<int>(a.K / 32);
+  p.epi = a.epi;
   const int64_t blocks = (a.N + 7) / 8;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, int64_t(dev.sm_count) * 8)));
   return launch_pdl(gemv_generic_kernel<MR>, dim3(grid), dim3(256), 0, stream, p);
@@ -732,9 +835,11 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
                           2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
     stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
     stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(MR) * P.K * 2 + 127u) & ~127u);
+    if (uses_epilogue_warp(P, geo) && geo.rt * MR * geo.wpt > kRedSlotFloats)
+      return cudaErrorInvalidConfiguration;  // the reduction slots are sized for kConsumers1 / kConsumers2
     L.prob[i] = P;
     L.prob[i].byte_begin = total;
-    total += P.N * packed_row_bytes(P.K);
+    total += P.N * problem_row_bytes(P);
   }
   const size_t fixed = sizeof(float) * kRedSlots * kRedSlotFloats + 16 * kRedSlots;
   const size_t budget = std::min<size_t>(Q4_GEMV_SMEM_BUDGET, dev.smem_optin);
@@ -750,12 +855,14 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   // Enough CTAs that every one has work; one per SM.
   const int64_t rows = [&] { int64_t r = 0; for (int i = 0; i < count; ++i) r += probs[i].N; return r; }();
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, rows)));
-  auto kern = gemv_kernel<MR, kThreads, NP>;
-  static PerDeviceOnce attr_once;
-  if (attr_once.needed(dev.device)) {
+  bool epi = false;
+  for (int i = 0; i < count; ++i) epi = epi || probs[i].epi != kEpiNone || is_fused(probs[i]);
+  auto kern = epi ? gemv_kernel<MR, kThreads, NP, true> : gemv_kernel<MR, kThreads, NP, false>;
+  static PerDeviceOnce attr_once[2];
+  if (attr_once[epi].needed(dev.device)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
     if (e != cudaSuccess) return e;
-    attr_once.mark(dev.device);
+    attr_once[epi].mark(dev.device);
   }
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, L);
 }
@@ -795,10 +902,14 @@ cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t st
       P.scales = a.scales;
       P.biases = a.biases;
       P.y = a.y + m0 * a.N;
+      P.r = a.r ? a.r + m0 * a.N : nullptr;
+      P.up_codes = a.up_codes;
+      P.up_scales = a.up_scales;
+      P.up_biases = a.up_biases;
       P.N = a.N;
       P.y_ld = a.N;
       P.K = static_cast<int32_t>(a.K);
-      P.pad_ = 0;
+      P.epi = a.epi;
       P.byte_begin = 0;
       (mr == 1 ? one : two).push_back(P);
     }

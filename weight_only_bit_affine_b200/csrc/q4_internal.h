@@ -27,6 +27,15 @@ struct PerDeviceOnce {
   void mark(int device) { done.fetch_or(uint64_t(1) << device, std::memory_order_release); }
 };
 
+// Output epilogue, applied to an fp32 accumulator before its single rounding
+// to bf16.  The feed-forward block the projections belong to (SwiGLU MLP
+// after the attention, each with its residual add) supplies the steps worth
+// fusing into the matmul that produces their input:
+//   kEpiResidual: y = r + acc        (o and down projections add the residual)
+//   kEpiSiluMul:  y = silu(r) * acc  (the up projection's output times the
+//                                     activated gate, r holding bf16 gate values)
+enum Epilogue : int { kEpiNone = 0, kEpiResidual = 1, kEpiSiluMul = 2 };
+
 // Launchers return cudaSuccess or the launch error.  Arguments are already
 // validated by the ABI layer.
 cudaError_t launch_quantize(const uint16_t* W, int64_t N, int64_t K, uint8_t* codes,
@@ -43,6 +52,16 @@ struct MatmulArgs {
   const uint16_t* biases;
   uint16_t* y;  // [M, N]
   int64_t M, N, K;
+  // Output epilogue (Epilogue above) with its bf16 operand r [M, N] (NULL
+  // for kEpiNone; may equal y).
+  int epi = 0;
+  const uint16_t* r = nullptr;
+  // SwiGLU in one pass (GEMV family only): when up_codes is set, y =
+  // silu(x . w_hat^T) * (x . w_hat_up^T), the up weights with the same shape.
+  const uint8_t* up_codes = nullptr;
+  const uint16_t* up_scales = nullptr;
+  const uint16_t* up_biases = nullptr;
+  bool fused() const { return up_codes != nullptr; }
 };
 // CUDA-core GEMV family, any M (activation rows in chunks of at most two;
 // every chunk re-reads the weights).

@@ -96,11 +96,13 @@ struct StreamProblem {
   const uint16_t* scales;
   const uint16_t* biases;
   uint16_t* y;         // [M, N]
+  const uint16_t* r;   // epilogue operand [M, N] (kEpiResidual / kEpiSiluMul), else NULL
   int64_t N;
   int64_t byte_begin;  // work offset of the first tile (packed bytes of all tiles before)
   int32_t K;
   int32_t segs;        // K segments per weight row; R = 128 / segs rows per tile
   int32_t tile_bytes;  // packed bytes of a full tile (the unit of work balancing)
+  int32_t epi;         // output epilogue (q4_device.cuh)
 };
 
 template <int NP>
@@ -577,7 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
         if (seg == 0 && row < P.N) {
 #pragma unroll
           for (int m = 0; m < kMaxRows; ++m)
-            if (m < L.M) P.y[static_cast<int64_t>(m) * P.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(part[m]));
+            if (m < L.M) {
+              const int64_t idx = static_cast<int64_t>(m) * P.N + row;
+              P.y[idx] = epilogue_bf16(part[m], P.epi, P.r, idx);
+            }
         }
       }
       ++lp;
@@ -642,6 +647,8 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
     P.scales = a.scales;
     P.biases = a.biases;
     P.y = a.y;
+    P.r = a.r;
+    P.epi = a.epi;
     P.N = a.N;
     P.K = static_cast<int32_t>(a.K);
     P.segs = pl.segs;
@@ -705,6 +712,7 @@ bool stream_supported(const MatmulArgs& a, const DeviceInfo& dev) {
   return false;
 #endif
   if (a.M < kMinRows || a.M > kMaxRows) return false;
+  if (a.fused()) return false;  // one-pass SwiGLU is a GEMV-family problem
   if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) return false;
   if (a.K > (int64_t(1) << 20)) return false;
   const Plan pl = plan_of(a);

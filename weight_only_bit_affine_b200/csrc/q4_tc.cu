@@ -57,8 +57,10 @@ struct TcParams {
   const uint16_t* scales;  // [N, K/32]
   const uint16_t* biases;
   uint16_t* y;             // [M, N]
+  const uint16_t* r;       // epilogue operand [M, N] (kEpiResidual / kEpiSiluMul), else NULL
   int64_t M, N;
   int K;
+  int epi;                 // output epilogue (q4_device.cuh)
   int bn;          // activation rows per tile (multiple of 16, <= 256)
   int splits;      // CTAs per cluster along K
   int stages;
@@ -140,7 +142,15 @@ __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t remote_addr) {
 // (barrier waits, TMA issue, MMA issue and commit) when shared memory allows
 // at least three of them.
 
-template <int ATOMS>
+// Output store; the EPI = false instantiation (no epilogue in the launch)
+// keeps the epilogue's code out of the kernel.
+template <bool EPI>
+__device__ __forceinline__ uint16_t store_tc(float v, const TcParams& p, int64_t idx) {
+  if constexpr (EPI) return epilogue_bf16(v, p.epi, p.r, idx);
+  return float_to_bf16_bits(v);
+}
+
+template <int ATOMS, bool EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
               const __grid_constant__ TcParams p) {
@@ -322,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int64_t m = m0 + col_half * cols + c0 + i;
-          if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+          if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = store_tc<EPI>(v[i], p, m * p.N + n0 + trow);
         }
       } else {
         float4* dst = reinterpret_cast<float4*>(red + trow * red_ld + col_half * cols + c0);
@@ -364,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int64_t m = m0 + 4 * q + i;
-          if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
+          if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = store_tc<EPI>(out[i], p, m * p.N + n0 + trow);
         }
       }
     }
@@ -410,6 +420,7 @@ uint32_t make_idesc(int bn) {
 cudaError_t tc_device_flags(unsigned int* flags, bool clear) { return tu_device_flags(flags, clear); }
 
 bool tc_supported(const MatmulArgs& a) {
+  if (a.fused()) return false;  // one-pass SwiGLU is a GEMV-family problem
   if (a.K % kSuperK != 0) return false;
   if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) return false;
   if (a.N > (int64_t(1) << 31) - kTileN || a.M > (int64_t(1) << 31) - 256) return false;
@@ -467,6 +478,8 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
   p.scales = a.scales;
   p.biases = a.biases;
   p.y = a.y;
+  p.r = a.r;
+  p.epi = a.epi;
   p.M = a.M;
   p.N = a.N;
   p.K = static_cast<int>(a.K);
@@ -488,7 +501,7 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
 
   static PerDeviceOnce attr_once;
   if (attr_once.needed(dev.device)) {
-    for (auto kern : {tc_kernel<1>, tc_kernel<2>}) {
+    for (auto kern : {tc_kernel<1, false>, tc_kernel<2, false>, tc_kernel<1, true>, tc_kernel<2, true>}) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(dev.smem_optin));
       if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
@@ -511,8 +524,11 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   count_launch();
-  return atoms == 2 ? cudaLaunchKernelEx(&cfg, tc_kernel<2>, tmap_x, tmap_codes, p)
-                    : cudaLaunchKernelEx(&cfg, tc_kernel<1>, tmap_x, tmap_codes, p);
+  if (p.epi != kEpiNone)
+    return atoms == 2 ? cudaLaunchKernelEx(&cfg, tc_kernel<2, true>, tmap_x, tmap_codes, p)
+                      : cudaLaunchKernelEx(&cfg, tc_kernel<1, true>, tmap_x, tmap_codes, p);
+  return atoms == 2 ? cudaLaunchKernelEx(&cfg, tc_kernel<2, false>, tmap_x, tmap_codes, p)
+                    : cudaLaunchKernelEx(&cfg, tc_kernel<1, false>, tmap_x, tmap_codes, p);
 }
 
 }  // namespace q4
