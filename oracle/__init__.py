@@ -1,4 +1,5 @@
-"""CPU oracle for affine 4-bit, group-32 weight-only quantization and matmul.
+"""CPU oracle for affine 4-bit, group-32 weight-only quantization and matmul
+(and its 8-bit variant, the same rule with 255 levels; the q8_* functions).
 
 TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
 CPU-baseline leg are the only callers.  The product library never imports it,
@@ -64,6 +65,14 @@ def _load():
         lib.oq4_matmul_ref.argtypes = [p, i64, i64, p, p, p, i64, p, i64, p, p]
         lib.oq4_matmul_ref_factored.restype = ctypes.c_int
         lib.oq4_matmul_ref_factored.argtypes = [p, i64, i64, p, p, p, i64, p]
+        lib.oq8_quantize.restype = ctypes.c_int
+        lib.oq8_quantize.argtypes = [p, i64, i64, p, p, p]
+        lib.oq8_dequantize.restype = ctypes.c_int
+        lib.oq8_dequantize.argtypes = [p, p, p, i64, i64, p]
+        lib.oq8_dequantize_f64.restype = ctypes.c_int
+        lib.oq8_dequantize_f64.argtypes = [p, p, p, i64, i64, p]
+        lib.oq8_matmul_ref.restype = ctypes.c_int
+        lib.oq8_matmul_ref.argtypes = [p, i64, i64, p, p, p, i64, p, i64, p, p]
         lib.oq4_set_threads.restype = None
         lib.oq4_set_threads.argtypes = [ctypes.c_int]
         lib.oq4_max_threads.restype = ctypes.c_int
@@ -186,6 +195,74 @@ def matmul_ref_factored(x_bits, codes, scales, biases) -> np.ndarray:
     _check(_load().oq4_matmul_ref_factored(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases),
                                            N, _ptr(y)), "matmul_ref_factored")
     return y
+
+
+# ------------------------------------------------------------------ 8-bit codes
+#
+# The same affine rule with 255 levels and one byte per code (the pages'
+# "standard 8-bit conversion" and INT8 bundle name the variant, not its
+# arithmetic): s = bf16(fp32(mx - mn) / 255), b = bf16(mn),
+# q = clamp(rne((w - b) / s), 0, 255); codes [N, K] uint8.
+
+
+def q8_packed_nbytes(N: int, K: int) -> int:
+    """Bytes of the 8-bit form of an [N, K] weight: 1 B per code + bf16 s and b per 32."""
+    return N * K + 4 * N * (K // GROUP)
+
+
+def q8_quantize(W_bits: np.ndarray):
+    """W [N, K] bf16 bits -> (codes [N, K] u8, scales [N, K/32] bf16 bits, biases bf16 bits)."""
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    codes = np.zeros((N, K), np.uint8)
+    scales = np.zeros((N, K // GROUP), np.uint16)
+    biases = np.zeros((N, K // GROUP), np.uint16)
+    _check(_load().oq8_quantize(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(biases)), "q8_quantize")
+    return codes, scales, biases
+
+
+def q8_dequantize(codes, scales, biases) -> np.ndarray:
+    """8-bit reconstruction s*q + b rounded to bf16 (bits), [N, K]."""
+    codes = _c(codes, np.uint8)
+    scales, biases = _c(scales, np.uint16), _c(biases, np.uint16)
+    N, K = codes.shape
+    out = np.zeros((N, K), np.uint16)
+    _check(_load().oq8_dequantize(_ptr(codes), _ptr(scales), _ptr(biases), N, K, _ptr(out)), "q8_dequantize")
+    return out
+
+
+def q8_dequantize_f64(codes, scales, biases) -> np.ndarray:
+    """8-bit reconstruction s*q + b in binary64 (not rounded), [N, K]."""
+    codes = _c(codes, np.uint8)
+    scales, biases = _c(scales, np.uint16), _c(biases, np.uint16)
+    N, K = codes.shape
+    out = np.zeros((N, K), np.float64)
+    _check(_load().oq8_dequantize_f64(_ptr(codes), _ptr(scales), _ptr(biases), N, K, _ptr(out)),
+           "q8_dequantize_f64")
+    return out
+
+
+def q8_matmul_ref(x_bits, codes, scales, biases, rows=None):
+    """y = x . W_hat^T over the exact 8-bit w_hat, binary64; returns (y, absdot) as matmul_ref."""
+    x = _c(x_bits, np.uint16)
+    if x.ndim == 1:
+        x = x[None, :]
+    codes = _c(codes, np.uint8)
+    scales, biases = _c(scales, np.uint16), _c(biases, np.uint16)
+    M, K = x.shape
+    N = codes.shape[0]
+    if codes.shape[1] != K:
+        raise ValueError("x and codes disagree on K")
+    if rows is None:
+        nrows, rp = N, None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nrows, rp = rows_arr.size, _ptr(rows_arr)
+    y = np.zeros((M, nrows), np.float64)
+    ad = np.zeros((M, nrows), np.float64)
+    _check(_load().oq8_matmul_ref(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N,
+                                  rp, nrows, _ptr(y), _ptr(ad)), "q8_matmul_ref")
+    return y, ad
 
 
 # --------------------------------------------------------------- output epilogues

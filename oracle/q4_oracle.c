@@ -250,6 +250,122 @@ int oq4_matmul_ref_factored(const uint16_t* x, int64_t M, int64_t K, const uint8
   return OQ4_OK;
 }
 
+/* ---- 8-bit variant ---------------------------------------------------------
+ *
+ * The same affine rule with 8-bit codes: the pages compare a "standard 8-bit
+ * conversion" of the model (TWX4 comparison page, opening section) and ship
+ * an INT8 bundle (ONNX README, "All four variants"), without stating its
+ * arithmetic.  The plainest reading keeps everything of the 4-bit rule but the
+ * number of levels:
+ *   s32 = fp32(mx - mn) / 255, s = bf16(s32), b = bf16(mn),
+ *   q = 0 if s == 0, else clamp(rne((w - b) / s), 0, 255)  (binary64),
+ *   w_hat = s*q + b (exact in binary64: 8 x 8 significant bits, plus b);
+ * codes are one byte per weight, [N, K]; scales and biases [N, K/32] bf16.
+ */
+
+static int quantize_group_q8(const uint16_t* w, uint8_t* codes32, uint16_t* s_out, uint16_t* b_out) {
+  float mn = INFINITY, mx = -INFINITY;
+  for (int i = 0; i < OQ4_GROUP; ++i) {
+    float v = (float)oq4_bf16_to_f64(w[i]);
+    if (!isfinite(v)) return OQ4_ERR_NONFINITE;
+    if (v < mn) mn = v;
+    if (v > mx) mx = v;
+  }
+  float range = mx - mn;              /* binary32 subtraction */
+  float s32 = range / 255.0f;         /* binary32 division    */
+  uint16_t sh = oq4_bf16_from_f64((double)s32);
+  uint16_t bh = oq4_bf16_from_f64((double)mn);
+  double s = oq4_bf16_to_f64(sh);
+  double b = oq4_bf16_to_f64(bh);
+  if (!isfinite(s)) return OQ4_ERR_NONFINITE;
+  for (int i = 0; i < OQ4_GROUP; ++i) {
+    int q = 0;
+    if (s != 0.0) {
+      double r = nearbyint((oq4_bf16_to_f64(w[i]) - b) / s);
+      if (r < 0.0) r = 0.0;
+      if (r > 255.0) r = 255.0;
+      q = (int)r;
+    }
+    codes32[i] = (uint8_t)q;
+  }
+  *s_out = sh;
+  *b_out = bh;
+  return OQ4_OK;
+}
+
+/* W: [N, K] bf16 bits -> codes [N, K] bytes, scales and biases [N, K/32]. */
+int oq8_quantize(const uint16_t* W, int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
+                 uint16_t* biases) {
+  if (N < 0 || K <= 0 || K % OQ4_GROUP) return OQ4_ERR_SHAPE;
+  const int64_t G = K / OQ4_GROUP;
+  int status = OQ4_OK;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < G; ++g) {
+      int st = quantize_group_q8(W + n * K + g * OQ4_GROUP, codes + n * K + g * OQ4_GROUP,
+                                 scales + n * G + g, biases + n * G + g);
+      if (st != OQ4_OK) {
+#pragma omp atomic write
+        status = st;
+      }
+    }
+  }
+  return status;
+}
+
+static double dequant_value_q8(const uint8_t* codes, const uint16_t* scales, const uint16_t* biases,
+                               int64_t K, int64_t n, int64_t k) {
+  const int64_t G = K / OQ4_GROUP;
+  double s = oq4_bf16_to_f64(scales[n * G + k / OQ4_GROUP]);
+  double b = oq4_bf16_to_f64(biases[n * G + k / OQ4_GROUP]);
+  return s * (double)codes[n * K + k] + b;
+}
+
+int oq8_dequantize(const uint8_t* codes, const uint16_t* scales, const uint16_t* biases, int64_t N,
+                   int64_t K, uint16_t* W_out) {
+  if (N < 0 || K <= 0 || K % OQ4_GROUP) return OQ4_ERR_SHAPE;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k)
+      W_out[n * K + k] = oq4_bf16_from_f64(dequant_value_q8(codes, scales, biases, K, n, k));
+  return OQ4_OK;
+}
+
+int oq8_dequantize_f64(const uint8_t* codes, const uint16_t* scales, const uint16_t* biases, int64_t N,
+                       int64_t K, double* W_out) {
+  if (N < 0 || K <= 0 || K % OQ4_GROUP) return OQ4_ERR_SHAPE;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k)
+      W_out[n * K + k] = dequant_value_q8(codes, scales, biases, K, n, k);
+  return OQ4_OK;
+}
+
+/* y = x . W_hat^T over the exact 8-bit w_hat; arguments as oq4_matmul_ref. */
+int oq8_matmul_ref(const uint16_t* x, int64_t M, int64_t K, const uint8_t* codes, const uint16_t* scales,
+                   const uint16_t* biases, int64_t N, const int64_t* rows, int64_t nrows, double* y,
+                   double* absdot) {
+  if (M < 0 || N < 0 || K <= 0 || K % OQ4_GROUP) return OQ4_ERR_SHAPE;
+  if (!rows) nrows = N;
+  for (int64_t r = 0; r < nrows; ++r)
+    if (rows && (rows[r] < 0 || rows[r] >= N)) return OQ4_ERR_SHAPE;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t n = rows ? rows[r] : r;
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0, aacc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        double p = oq4_bf16_to_f64(x[m * K + k]) * dequant_value_q8(codes, scales, biases, K, n, k);
+        acc += p;
+        aacc += fabs(p);
+      }
+      y[m * nrows + r] = acc;
+      if (absdot) absdot[m * nrows + r] = aacc;
+    }
+  }
+  return OQ4_OK;
+}
+
 /* Threads used by the OpenMP loops above (timing only; results do not depend
  * on it: every output element is computed by one thread in a fixed order). */
 void oq4_set_threads(int n) {
