@@ -317,6 +317,28 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
                 "(silu(gate) * up in the GEMV epilogue); compare temporal_layer_M1, the 7 plain projections",
     }
 
+    # the 8-bit variant of the same layer (9 bits per weight), one q8_matmul per
+    # projection, four layers rotated (925 MB > L2)
+    seed8 = workloads.seed_of("batched_layer")
+    lay8 = []
+    for rep in range(4):
+        for t, p in enumerate(workloads.TEMPORAL_LAYER):
+            W = workloads.weight(p.N, p.K, seed8, 100 * rep + t, device=dev)
+            lay8.append((p,) + tuple(q4.q8_quantize(W)))
+            del W
+    ys8 = [torch.empty((1, p.N), dtype=torch.bfloat16, device=dev) for p, _, _, _ in lay8]
+    bytes8 = sum(c.numel() + 2 * s.numel() + 2 * b.numel() for _, c, s, b in lay8[:7])
+
+    def q8_layers():
+        for (p, c, s, b), y in zip(lay8, ys8):
+            q4.q8_matmul(x_down if p.K == 11264 else x, c, s, b, out=y)
+
+    ms8 = _graph_ms(dev, q8_layers, 50) / 4
+    rows["q8_layer_M1"] = {"us_per_layer": round(ms8 * 1e3, 2), "GBps": round(bytes8 / (ms8 * 1e-3) / 1e9, 1),
+                           "bytes": bytes8, "launches_per_layer": 7,
+                           "path": "q8_gemv_kernel: CUDA cores, warp per row (8-bit codes, 9 bits per weight)"}
+    del lay8
+
     # depformer: stacked [16 N, K] weights per projection, drawn and quantized on the GPU
     seed = workloads.seed_of("depformer_steps")
     steps = workloads.DEPFORMER_STEPS

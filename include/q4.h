@@ -224,6 +224,38 @@ Q4_API q4_status q4_matmul_swiglu(const q4_bf16* x, int64_t M, int64_t K, const 
 Q4_API q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int group,
                                  q4_stream_t stream);
 
+/*
+ * The 8-bit variant: the same affine rule with 255 levels and one byte per
+ * code.  The pages compare a "standard 8-bit conversion" of the model with
+ * the 4-bit builds (TWX4 comparison page, opening section) and ship an INT8
+ * bundle (ONNX README, "All four variants"), without its arithmetic; read
+ * plainly it is the 4-bit rule with 255 in place of 15:
+ *   scale = bf16(fp32(mx - mn) / 255), bias = bf16(mn),
+ *   q = 0 if scale == 0, else clamp(round_half_even((w - bias)/scale), 0, 255)
+ * (binary64 quotient).  A bf16 scale is within 2^-8 of fp32(mx - mn)/255, so
+ * the maximum lands on code 254 or 255 and the clamp can bind: elements above
+ * the top code then reconstruct within one scale step instead of half.
+ * Layout: codes [N, K] uint8 (byte k of row n is q[n,k]), 16-byte aligned;
+ * scales, biases [N, K/32] bf16.  9 bits per weight.  Same conventions and
+ * status codes as the 4-bit calls.
+ */
+Q4_API q4_status q8_quantize(const q4_bf16* W, int64_t N, int64_t K, int group, uint8_t* codes,
+                             q4_bf16* scales, q4_bf16* biases, q4_stream_t stream);
+
+/* W_out [N, K] = bf16(scale * q + bias), the value taken in binary64. */
+Q4_API q4_status q8_dequantize(const uint8_t* codes, const q4_bf16* scales, const q4_bf16* biases,
+                               int64_t N, int64_t K, int group, q4_bf16* W_out, q4_stream_t stream);
+
+/*
+ * y [M, N] = x . w_hat^T with 8-bit codes: fp32 accumulation of exact
+ * products (each code an exact fp32, x in fp32), bf16 output.  CUDA-core
+ * GEMV for every M (activation rows in pairs; each pair reads the weights
+ * once).  K <= 196608 (Q4_ERR_UNSUPPORTED above).
+ */
+Q4_API q4_status q8_matmul(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes,
+                           const q4_bf16* scales, const q4_bf16* biases, int64_t N, int group,
+                           q4_bf16* y, q4_stream_t stream);
+
 /* Message for the calling thread's last non-OK status ("" if none). */
 Q4_API const char* q4_last_error(void);
 

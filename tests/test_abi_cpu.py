@@ -30,14 +30,15 @@ def declared_symbols():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(q4_\w+)\s*\(", text, flags=re.M)
+        names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(q[48]_\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
 
 
 def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ["q4_quantize", "q4_dequantize", "q4_matmul", "q4_matmul_step", "q4_matmul_residual",
-              "q4_matmul_swiglu", "q4_matmul_batch", "q4_last_error"]:
+              "q4_matmul_swiglu", "q4_matmul_batch", "q4_last_error", "q8_quantize", "q8_dequantize",
+              "q8_matmul"]:
         assert n in names
 
 
@@ -46,7 +47,7 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
     assert set(declared_symbols()) <= set(q4.SIGNATURES)
     out = subprocess.run(["nm", "-D", "--defined-only", q4.library_path()], capture_output=True, text=True).stdout
-    exported = set(re.findall(r"\bT (q4_\w+)", out))
+    exported = set(re.findall(r"\bT (q[48]_\w+)", out))
     assert set(declared_symbols()) <= exported
 
 
@@ -150,6 +151,21 @@ def test_descriptor_layout_matches_c(tmp_path):
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
     D = q4.MatmulDesc
     assert got == [ctypes.sizeof(D), D.epilogue.offset, D.r.offset, D.up_codes.offset, D.up_biases.offset]
+
+
+def test_q8_validation(lib):
+    mm = lambda x=P, M=1, K=64, codes=P, group=32: lib.q8_matmul(x, M, K, codes, P, P, 8, group, P, None)
+    assert mm(K=48) == SHAPE
+    assert mm(group=64) == UNSUP
+    assert mm(K=196608 + 32) == UNSUP
+    assert b"K" in lib.q4_last_error()
+    assert mm(codes=P + 8) == ALIGN
+    assert mm(x=None) == NULL
+    assert mm(M=0) == OK
+    assert lib.q8_quantize(P, 4, 64, 32, P + 4, P, P, None) == ALIGN
+    assert lib.q8_quantize(P, -1, 64, 32, P, P, P, None) == SHAPE
+    assert lib.q8_dequantize(P, P, P, 4, 64, 32, P + 8, None) == ALIGN
+    assert lib.q8_dequantize(None, P, P, 4, 64, 32, P, None) == NULL
 
 
 def test_valid_call_without_gpu_reports_cuda_error(lib):

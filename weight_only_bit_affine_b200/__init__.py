@@ -15,6 +15,8 @@ come from PyTorch) and have the same names as the C entry points:
     y = q4_matmul_residual(x, codes, scales, biases, r)   # r + x . w_hat^T
     h = q4_matmul_swiglu(x, (gc, gs, gb), (uc, us, ub))   # silu(gate) * up
     q4_matmul_batch([(x, codes, scales, biases, y), ...]) # one launch per kernel path
+    codes8, scales, biases = q8_quantize(W)             # 8-bit variant: codes [N, K]
+    y = q8_matmul(x, codes8, scales, biases)
 
 Layout (model card "personaplex-edge-q4", "Release details": affine Q4,
 group size 32, BF16): codes [N, K/2] uint8 (low nibble = even k), scales
@@ -42,6 +44,9 @@ __all__ = [
     "q4_matmul_batch",
     "Residual",
     "SwiGLU",
+    "q8_quantize",
+    "q8_dequantize",
+    "q8_matmul",
     "q4_debug_device_flags",
     "q4_debug_launch_count",
 ]
@@ -70,6 +75,9 @@ SIGNATURES = {
     "q4_matmul_residual": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P, _P]),
     "q4_matmul_swiglu": (_INT, [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I64, _INT, _P, _P]),
     "q4_matmul_batch": (_INT, [_P, _INT, _I64, _INT, _P]),
+    "q8_quantize": (_INT, [_P, _I64, _I64, _INT, _P, _P, _P, _P]),
+    "q8_dequantize": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),
+    "q8_matmul": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P]),
     "q4_last_error": (ctypes.c_char_p, []),
     "q4_debug_device_flags": (_INT, [_INT]),
     "q4_debug_launch_count": (ctypes.c_ulonglong, []),
@@ -350,6 +358,59 @@ def q4_matmul_batch(problems, group: int = GROUP):
     with torch.cuda.device(dev):
         _check(lib().q4_matmul_batch(ctypes.cast(descs, ctypes.c_void_p), len(problems), M, group, _stream(dev)))
     return [p[4] for p in problems]
+
+
+# ------------------------------------------------------------------ 8-bit codes
+
+
+def q8_quantize(W: torch.Tensor, group: int = GROUP) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """W [N, K] bf16 -> (codes [N, K] uint8, scales [N, K/32] bf16, biases [N, K/32] bf16), 255 levels."""
+    _want(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    dev = W.device
+    codes = torch.empty((N, K), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, max(K // GROUP, 0)), dtype=torch.bfloat16, device=dev)
+    biases = torch.empty_like(scales)
+    with torch.cuda.device(dev):
+        _check(lib().q8_quantize(_ptr(W), N, K, group, _ptr(codes), _ptr(scales), _ptr(biases), _stream(dev)))
+    return codes, scales, biases
+
+
+def _q8_shapes(codes, scales, biases, K, what="codes"):
+    _want(codes, what, torch.uint8, 2)
+    _want(scales, "scales", torch.bfloat16, 2)
+    _want(biases, "biases", torch.bfloat16, 2)
+    if codes.shape[1] != K or scales.shape != (codes.shape[0], K // GROUP) or biases.shape != scales.shape:
+        raise ValueError(f"8-bit weights: codes [N, K], scales and biases [N, K/32] with K = {K}")
+
+
+def q8_dequantize(codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor, group: int = GROUP,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """8-bit (codes, scales, biases) -> W_hat [N, K] bf16 = bf16(scale * q + bias)."""
+    _want(codes, "codes", torch.uint8, 2)
+    N, K = codes.shape
+    _q8_shapes(codes, scales, biases, K)
+    out = _out(out, N, K, codes.device)
+    with torch.cuda.device(codes.device):
+        _check(lib().q8_dequantize(_ptr(codes), _ptr(scales), _ptr(biases), N, K, group, _ptr(out),
+                                   _stream(codes.device)))
+    return out
+
+
+def q8_matmul(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+              group: int = GROUP, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = x . w_hat^T with 8-bit codes:  x [M, K] bf16 -> y [M, N] bf16."""
+    _want(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    _q8_shapes(codes, scales, biases, K)
+    if not (x.device == codes.device == scales.device == biases.device):
+        raise ValueError("all tensors must be on the same device")
+    N = codes.shape[0]
+    out = _out(out, M, N, x.device)
+    with torch.cuda.device(x.device):
+        _check(lib().q8_matmul(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N, group, _ptr(out),
+                               _stream(x.device)))
+    return out
 
 
 def q4_debug_device_flags(clear: bool = False) -> int:

@@ -315,6 +315,55 @@ q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int
   return run_problems(list, *dev, reinterpret_cast<cudaStream_t>(stream), "q4_matmul_batch launch");
 }
 
+// ---- the 8-bit variant (q8.cu) --------------------------------------------
+
+q4_status q8_quantize(const q4_bf16* W, int64_t N, int64_t K, int group, uint8_t* codes, q4_bf16* scales,
+                      q4_bf16* biases, q4_stream_t stream) {
+  q4_status st = check_k_group(K, group);
+  if (st != Q4_OK) return st;
+  if (N < 0) return fail(Q4_ERR_SHAPE, "negative N = %lld", (long long)N);
+  if (N == 0) return Q4_OK;
+  if (!W || !codes || !scales || !biases) return fail(Q4_ERR_NULL, "q8_quantize: NULL pointer argument");
+  if (!aligned(W, 16) || !aligned(codes, 16))
+    return fail(Q4_ERR_ALIGN, "q8_quantize: W and codes must be 16-byte aligned");
+  if (!aligned(scales, 2) || !aligned(biases, 2))
+    return fail(Q4_ERR_ALIGN, "q8_quantize: scales and biases must be 2-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  return from_cuda(launch_q8_quantize(W, N, K, codes, scales, biases, reinterpret_cast<cudaStream_t>(stream), *dev),
+                   "q8_quantize launch");
+}
+
+q4_status q8_dequantize(const uint8_t* codes, const q4_bf16* scales, const q4_bf16* biases, int64_t N, int64_t K,
+                        int group, q4_bf16* W_out, q4_stream_t stream) {
+  q4_status st = check_k_group(K, group);
+  if (st != Q4_OK) return st;
+  if (N < 0) return fail(Q4_ERR_SHAPE, "negative N = %lld", (long long)N);
+  if (N == 0) return Q4_OK;
+  if (!W_out || !codes || !scales || !biases) return fail(Q4_ERR_NULL, "q8_dequantize: NULL pointer argument");
+  if (!aligned(W_out, 16) || !aligned(codes, 16))
+    return fail(Q4_ERR_ALIGN, "q8_dequantize: W_out and codes must be 16-byte aligned");
+  if (!aligned(scales, 2) || !aligned(biases, 2))
+    return fail(Q4_ERR_ALIGN, "q8_dequantize: scales and biases must be 2-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  return from_cuda(
+      launch_q8_dequantize(codes, scales, biases, N, K, W_out, reinterpret_cast<cudaStream_t>(stream), *dev),
+      "q8_dequantize launch");
+}
+
+q4_status q8_matmul(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes, const q4_bf16* scales,
+                    const q4_bf16* biases, int64_t N, int group, q4_bf16* y, q4_stream_t stream) {
+  bool empty = false;
+  q4_status st = check_matmul("q8_matmul", x, M, K, codes, scales, biases, N, group, y, &empty);
+  if (st != Q4_OK || empty) return st;
+  if (K > kQ8MaxK) return fail(Q4_ERR_UNSUPPORTED, "q8_matmul: K = %lld above %lld", (long long)K, (long long)kQ8MaxK);
+  const DeviceInfo* dev = nullptr;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  MatmulArgs a{x, codes, scales, biases, y, M, N, K};
+  return from_cuda(launch_q8_matmul(a, reinterpret_cast<cudaStream_t>(stream), *dev), "q8_matmul launch");
+}
+
 const char* q4_last_error(void) { return t_last_error; }
 
 unsigned long long q4_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

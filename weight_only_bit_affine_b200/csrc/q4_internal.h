@@ -63,6 +63,14 @@ struct MatmulArgs {
   const uint16_t* up_biases = nullptr;
   bool fused() const { return up_codes != nullptr; }
 };
+// The 8-bit variant (q8.cu): codes [N, K] one byte each; K <= kQ8MaxK.
+constexpr int64_t kQ8MaxK = 196608;  // per-group sums of two activation rows fill 48 KB of shared memory
+cudaError_t launch_q8_quantize(const uint16_t* W, int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
+                               uint16_t* biases, cudaStream_t stream, const DeviceInfo& dev);
+cudaError_t launch_q8_dequantize(const uint8_t* codes, const uint16_t* scales, const uint16_t* biases, int64_t N,
+                                 int64_t K, uint16_t* W_out, cudaStream_t stream, const DeviceInfo& dev);
+cudaError_t launch_q8_matmul(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev);
+
 // CUDA-core GEMV family, any M (activation rows in chunks of at most two;
 // every chunk re-reads the weights).
 cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev);

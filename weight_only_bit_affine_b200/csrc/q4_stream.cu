@@ -277,7 +277,9 @@ __device__ __forceinline__ void tile_range(const StreamProblem& P, int64_t lo, i
   j1 = first_from(hi);
 }
 
-template <int NP>
+// EPI: some problem of the launch has an output epilogue; the plain
+// instantiation keeps the epilogue's code out of the kernel.
+template <int NP, bool EPI>
 __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_constant__ StreamLaunch<NP> L) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -581,7 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
           for (int m = 0; m < kMaxRows; ++m)
             if (m < L.M) {
               const int64_t idx = static_cast<int64_t>(m) * P.N + row;
-              P.y[idx] = epilogue_bf16(part[m], P.epi, P.r, idx);
+              if constexpr (EPI) P.y[idx] = epilogue_bf16(part[m], P.epi, P.r, idx);
+              else P.y[idx] = float_to_bf16_bits(part[m]);
             }
         }
       }
@@ -681,13 +684,15 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
   L.total_bytes = total;
   const size_t smem = kFixedSmem + b_bytes + static_cast<size_t>(stages) * stage_bytes;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, tiles)));
-  auto kern = stream_kernel<NP>;
-  static PerDeviceOnce attr_once;
-  if (attr_once.needed(dev.device)) {
+  bool epi = false;
+  for (int i = 0; i < count; ++i) epi = epi || list[i].epi != kEpiNone;
+  auto kern = epi ? stream_kernel<NP, true> : stream_kernel<NP, false>;
+  static PerDeviceOnce attr_once[2];
+  if (attr_once[epi].needed(dev.device)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(dev.smem_optin));
     if (e != cudaSuccess) return e;
-    attr_once.mark(dev.device);
+    attr_once[epi].mark(dev.device);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
