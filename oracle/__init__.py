@@ -310,7 +310,7 @@ def matmul_swiglu_ref(x_bits, gate, up, rows=None):
     |silu(g') u' - silu(g) u| <= L (|dg|) (|u| + Tu) + |silu(g)| Tu with
     L = SILU_LIPSCHITZ, where |dg| <= Tg + 2^-8 (|g| + Tg) also covers a gate
     stored as bf16 between two passes; then one bf16 rounding of h, relative
-    2^-8 of its magnitude (with margin over the 2^-9 of round-to-nearest).
+    2^-8 of its magnitude (bf16's unit roundoff: 8 significant bits).
     """
     g, adg = matmul_ref(x_bits, *gate, rows=rows)
     u, adu = matmul_ref(x_bits, *up, rows=rows)
