@@ -140,6 +140,29 @@ def test_batch_descriptor_validation(lib):
     assert one(epilogue=q4.EPI_SWIGLU, up_codes=P + 4, up_scales=P, up_biases=P) == ALIGN
 
 
+def test_batch_validates_every_entry_before_the_device():
+    """A bad epilogue in the last entry is reported as such (not as the device
+    error a valid batch reaches on a machine without a GPU): validation of the
+    whole list precedes any device work, so nothing is enqueued."""
+    from weight_only_bit_affine_b200 import build
+
+    build.build()
+    lib = q4.lib()
+    good = q4.MatmulDesc(P, P, P, P, P, 8, 64)
+    res = q4.MatmulDesc(P, P, P, P, P + 64, 8, 64)
+    res.epilogue, res.r = q4.EPI_RESIDUAL, P + 64  # in place: allowed
+    bad = q4.MatmulDesc(P, P, P, P, P + 128, 8, 64)
+    bad.epilogue = 9
+    arr = (q4.MatmulDesc * 3)(good, res, bad)
+    assert lib.q4_matmul_batch(ctypes.cast(arr, ctypes.c_void_p), 3, 1, 32, None) == UNSUP
+    assert b"q4_matmul_batch[2]" in lib.q4_last_error()
+    import torch
+
+    if not torch.cuda.is_available():
+        arr = (q4.MatmulDesc * 2)(good, res)
+        assert lib.q4_matmul_batch(ctypes.cast(arr, ctypes.c_void_p), 2, 1, 32, None) == CUDA
+
+
 def test_descriptor_layout_matches_c(tmp_path):
     src = tmp_path / "l.c"
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "q4.h"\n'
