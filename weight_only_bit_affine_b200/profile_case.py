@@ -14,6 +14,11 @@ whole case once, after one warm-up rep):
                  one q4_matmul_batch.
   layer_m4       one temporal layer (7 projections) at M = 4 as one
                  q4_matmul_batch: the tensor-core streaming kernel.
+  fused_layer    one temporal layer at M = 1 with its epilogues fused (o and
+                 down + residual, gate/up as one SwiGLU problem), one
+                 q4_matmul_batch: the GEMV's epilogue instantiation.
+  q8_layer       one temporal layer with 8-bit codes at M = 1, one q8_matmul
+                 per projection: the 8-bit GEMV.
 
 Every case checks the library's bounded-wait flag at the end.
 """
@@ -96,8 +101,49 @@ def _layer_m4(dev):
     return lambda: q4.q4_matmul_batch(probs)
 
 
+def _fused_layer(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    x = workloads.activation(1, 4096, seed, 101, device=dev)
+    xd = workloads.activation(1, 11264, seed, 201, device=dev)
+    w = {p.name: q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+         for t, p in enumerate(workloads.TEMPORAL_LAYER)}
+    out = lambda n: torch.empty((1, n), dtype=torch.bfloat16, device=dev)
+    r_o = torch.zeros((1, 4096), dtype=torch.bfloat16, device=dev)  # two residual streams: problems of
+    r_d = torch.zeros((1, 4096), dtype=torch.bfloat16, device=dev)  # one launch may not share an output
+    probs = [(x, *w[n], out(4096)) for n in ("q", "k", "v")]
+    probs += [(x, *w["o"], r_o, q4.Residual(r_o)), (x, *w["gate"], out(11264), q4.SwiGLU(*w["up"])),
+              (xd, *w["down"], r_d, q4.Residual(r_d))]
+    return lambda: q4.q4_matmul_batch(probs)
+
+
+def _q8_layer(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    x = workloads.activation(1, 4096, seed, 101, device=dev)
+    xd = workloads.activation(1, 11264, seed, 201, device=dev)
+    items = []
+    for t, p in enumerate(workloads.TEMPORAL_LAYER):
+        c, s, b = q4.q8_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+        items.append((xd if p.K == 11264 else x, c, s, b, torch.empty((1, p.N), dtype=torch.bfloat16, device=dev)))
+
+    def run():
+        for xx, c, s, b, y in items:
+            q4.q8_matmul(xx, c, s, b, out=y)
+
+    return run
+
+
 CASES = {"stream_small": _stream_small, "tc_layer": _tc_layer, "depformer_step": _depformer_step,
-         "layer_m4": _layer_m4}
+         "layer_m4": _layer_m4, "fused_layer": _fused_layer, "q8_layer": _q8_layer}
 
 
 def main(argv=None):
