@@ -306,17 +306,17 @@ def matmul_swiglu_ref(x_bits, gate, up, rows=None):
     the gate and up weights ((codes, scales, biases) triples).
 
     Returns (h, bound).  The bound carries the product bounds
-    T = 4e-3 * sum|x w_hat| + 1e-6 of g and u through h to first order:
-    |silu(g') u' - silu(g) u| <= L (|dg|) (|u| + Tu) + |silu(g)| Tu with
-    L = SILU_LIPSCHITZ, where |dg| <= Tg + 2^-8 (|g| + Tg) also covers a gate
-    stored as bf16 between two passes; then one bf16 rounding of h, relative
-    2^-8 of its magnitude (bf16's unit roundoff: 8 significant bits).
+    T = 4e-3 * sum|x w_hat| + 1e-6 of g and u through h to first order, for a
+    computation that keeps both products unrounded until h:
+    |silu(g') u' - silu(g) u| <= L Tg (|u| + Tu) + |silu(g)| Tu with
+    L = SILU_LIPSCHITZ; then one bf16 rounding of h, relative 2^-8 of its
+    magnitude (bf16's unit roundoff: 8 significant bits).
     """
     g, adg = matmul_ref(x_bits, *gate, rows=rows)
     u, adu = matmul_ref(x_bits, *up, rows=rows)
     tg, tu = 4e-3 * adg + 1e-6, 4e-3 * adu + 1e-6
     sg = silu(g)
-    dg = SILU_LIPSCHITZ * (tg + 2.0 ** -8 * (np.abs(g) + tg))
+    dg = SILU_LIPSCHITZ * tg
     mag_u = np.abs(u) + tu
     bound = dg * mag_u + np.abs(sg) * tu + 2.0 ** -8 * (np.abs(sg) + dg) * mag_u + 1e-6
     return sg * u, bound
