@@ -657,7 +657,7 @@ def run_ours(args):
     if not args.no_rows:
         extra = workload_rows(dev, packed, x, x_down, _bf16_peak())
 
-    flags = q4.q4_debug_device_flags()
+    flags = q4.q4_device_status()
     peak, peak_kind = _peaks()
     kh = _kernel_source_hash()
     traffic = _traffic_per_launch(kh)

@@ -26,9 +26,16 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and never synchronize the host or copy between host
  *    and device.
- *  - Arguments are validated on the host before anything is launched; a
- *    non-OK status means nothing was enqueued.  q4_last_error() returns a
+ *  - Arguments are validated, and every host-side step of the launches
+ *    (tensor-map encoding, launch configurations) is done, before anything is
+ *    enqueued: a status other than Q4_ERR_CUDA means nothing was enqueued.
+ *    Q4_ERR_CUDA from a launch that the CUDA runtime rejected may leave the
+ *    earlier launches of the same call enqueued.  q4_last_error() returns a
  *    message for the last non-OK status of the calling thread.
+ *  - Every wait inside the kernels is bounded (one second); a kernel that
+ *    gives one up writes NaN where it cannot vouch for a result and raises a
+ *    device flag that q4_device_status() reports.  Results of work enqueued
+ *    since the flag was last clear are invalid while it is set.
  *  - Alignment: W, W_out, codes and x must be 16-byte aligned; scales,
  *    biases and y 2-byte aligned.  Row strides are implied by K (dense).
  *  - Sizes: 0 <= M, N; 32 <= K, K % 32 == 0.  M == 0 or N == 0 is a no-op.
@@ -105,13 +112,17 @@ Q4_API q4_status q4_dequantize(const uint8_t* codes, const q4_bf16* scales,
  * are not expanded back to BF16).
  * In:  x [M, K] bf16 (row-major), codes [N, K/2], scales, biases [N, K/32].
  * Out: y [M, N] bf16 (row-major).
- * Kernel by M (the same for every problem, alone or batched, so a batched
- * result is bit-identical to the single call): M = 1, 2 the CUDA-core GEMV;
- * M = 3, 4 (K % 256 == 0, 16-byte aligned scale and bias rows) tensor-core
- * weight streaming, dequantized weights in tensor memory; M >= 16 (K % 256
- * == 0, same alignment) tensor-core tiles; otherwise the GEMV on pairs of
- * activation rows.  Results of the tensor-core kernels use w_hat rounded to
- * bf16 (exactly q4_dequantize's values); the GEMV uses the exact s*q + b.
+ * Kernel by problem (the same for a problem alone or batched, so a batched
+ * result is bit-identical to the single call): M = 1, 2 the CUDA-core GEMV
+ * (exact products x * (128 + q) in fp32, the offset removed per group);
+ * M = 3..8 tensor-core weight streaming where its shared and tensor memory
+ * hold the problem (K % 256 == 0, 16-byte aligned scale and bias rows,
+ * segments * M <= 128); otherwise, for M >= 3 with K % 256 == 0 and the same
+ * alignment, tensor-core tiles; otherwise the GEMV on pairs of activation
+ * rows.  Every kernel reads each weight byte once per call, except the GEMV
+ * on pairs (once per pair).  The tensor-core kernels feed each weight to the
+ * MMA as two bf16 parts hi + lo with |s*q + b - hi - lo| <= ~2^-16 |s*q + b|
+ * (two MMAs per K step), so no path rounds w_hat to bf16.
  * Launch-order contract: the kernels may be launched with programmatic
  * dependent launch; they read nothing written by an earlier kernel in the
  * stream before that kernel has completed.
@@ -147,12 +158,8 @@ Q4_API q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K,
  *   Q4_EPI_SWIGLU    y = bf16(silu(acc) * acc_up), silu(z) = z / (1 + e^-z),
  *                    acc the gate projection's and acc_up the up
  *                    projection's fp32 accumulators (weights of the same
- *                    shape).  Where q4_matmul would run the CUDA-core GEMV
- *                    both come from one pass that reads x and the two
- *                    weights once per pair of activation rows; where it
- *                    would run a tensor-core kernel, the gate result is
- *                    stored in y as bf16 and the up pass reads it back, so
- *                    silu sees the bf16-rounded gate.
+ *                    shape), both from one pass in one launch on every
+ *                    kernel: silu sees the fp32 gate.
  */
 typedef enum { Q4_EPI_NONE = 0, Q4_EPI_RESIDUAL = 1, Q4_EPI_SWIGLU = 2 } q4_epilogue;
 
@@ -191,10 +198,9 @@ Q4_API q4_status q4_matmul_residual(const q4_bf16* x, int64_t M, int64_t K, cons
  * the gate and up projections of the SwiGLU MLP and its activation in one
  * call (Q4_EPI_SWIGLU above).  Both weights are [N, K] in the packed format
  * with the same alignment rules as q4_matmul; h [M, N] must not overlap any
- * input.  Kernels as q4_matmul chooses them for M: on the GEMV one pass
- * (M = 1, 2: one launch reading each weight once); on a tensor-core kernel
- * two passes (gate into h, then up with the silu-multiply epilogue reading
- * h), one launch each.
+ * input.  Kernels as q4_matmul chooses them; every kernel computes the gate
+ * and up products in one pass (one launch) and keeps both in fp32 until the
+ * single rounding of h.
  */
 Q4_API q4_status q4_matmul_swiglu(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* gate_codes,
                                   const q4_bf16* gate_scales, const q4_bf16* gate_biases,
@@ -207,7 +213,7 @@ Q4_API q4_status q4_matmul_swiglu(const q4_bf16* x, int64_t M, int64_t K, const 
  * activation rows M, each computing exactly what q4_matmul computes, enqueued
  * as few kernel launches as possible: one for up to 256 problems that take
  * the bulk-copy GEMV path (or the weight-streaming path), one per problem on
- * the tensor-core tile path.  The Swift/MLX blog ("Performance optimizations":
+ * the tensor-core tile path and on the GEMV's generic fallback.  The Swift/MLX blog ("Performance optimizations":
  * compiling the temporal transformer fuses its ~450 per-step kernel
  * dispatches) and the ONNX README ("All four variants": CUDA Graph capture)
  * both cut per-call launch overhead; this is that fusion for a whole weight
@@ -215,8 +221,7 @@ Q4_API q4_status q4_matmul_swiglu(const q4_bf16* x, int64_t M, int64_t K, const 
  * `descs` is a HOST array of `count` entries, read before the call returns.
  * The problems run concurrently: no output may overlap any input of any
  * problem in the list (a residual operand may be its own problem's output).
- * Each entry's epilogue applies as in q4_matmul_residual / q4_matmul_swiglu;
- * a SwiGLU entry on the two-pass path adds one launch for the up passes.
+ * Each entry's epilogue applies as in q4_matmul_residual / q4_matmul_swiglu.
  * Validation covers every entry before anything is enqueued; count == 0 is
  * a no-op; count < 0 is Q4_ERR_SHAPE; an unknown epilogue or a nonzero
  * `reserved` is Q4_ERR_UNSUPPORTED.
@@ -260,14 +265,16 @@ Q4_API q4_status q8_matmul(const q4_bf16* x, int64_t M, int64_t K, const uint8_t
 Q4_API const char* q4_last_error(void);
 
 /*
- * Diagnostic, not part of the compute path: bit 0 is set on the current
- * device if any libq4 kernel gave up a bounded internal wait (a pipeline
- * stage that never arrived within one second; the kernel then finishes
- * without waiting and its output is invalid).  Synchronizes with the device
- * (it copies the flag to the host).  clear != 0 resets the flags.  Returns
- * the flags, or -1 if the copy failed.
+ * Status of the kernels on the current device: bit 0 is set if any libq4
+ * kernel gave up a bounded internal wait (a pipeline stage that never
+ * arrived within one second, e.g. when the context was preempted for that
+ * long).  The kernel then finished without waiting, wrote NaN where it could
+ * not vouch for a result, and every result enqueued since the flag was last
+ * clear must be treated as invalid.  Synchronizes with the device (it copies
+ * the flag to the host); call it after the work to be checked.  clear != 0
+ * resets the flag.  Returns the flags, or -1 if the copy failed.
  */
-Q4_API int q4_debug_device_flags(int clear);
+Q4_API int q4_device_status(int clear);
 
 /* Diagnostic: number of kernel launches libq4 has enqueued in this process
  * (counted on the host when each launch is issued; graph replays of captured

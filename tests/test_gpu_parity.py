@@ -26,9 +26,9 @@ def _gpu():
     from weight_only_bit_affine_b200 import build
 
     build.build()
-    q4.q4_debug_device_flags(clear=True)
+    q4.q4_device_status(clear=True)
     yield
-    assert q4.q4_debug_device_flags() == 0, "a bounded wait gave up inside a kernel"
+    assert q4.q4_device_status() == 0, "a bounded wait gave up inside a kernel"
 
 
 def _quant(W):

@@ -1,6 +1,9 @@
 """Full-size temporal weight stream at M = 1 (32 layers x 7 projections + text
-head, 4,192,337,920 packed bytes), in the launch configuration the benchmark
-times: one q4_matmul per projection on one stream, x reused per layer.
+head, 4,192,337,920 packed bytes), x reused per layer: as 225 separate
+q4_matmul calls, and in the launch configuration the benchmark times -- one
+q4_matmul_batch over all 225 projections (one launch of the GEMV, whose
+byte-balanced CTA ranges cross problem boundaries), the outputs views of one
+buffer.
 
 The weights are drawn and quantized on the GPU (a host draw of 6.7e9 values is
 too slow); the codes of layers 0 and 31 and of the head are compared bit for
@@ -61,4 +64,30 @@ def test_stream_matmul_sampled(stream):
         rows = sample_rows(p.N, 12, seed=i)
         worst = max(worst, check_matmul(xi, c, s, b, y, rows=rows, what=p.name))
     assert worst < 4e-3
-    assert q4.q4_debug_device_flags() == 0
+    assert q4.q4_device_status() == 0
+
+
+def test_stream_batch_as_benchmarked(stream):
+    """One q4_matmul_batch over the 225 projections with the benchmark's output
+    layout: bit-identical to the single calls, and within the bound on sampled
+    rows of every projection."""
+    packed, x, x_down = stream
+    y_all = torch.empty(sum(p.N for p, _, _, _ in packed), dtype=torch.bfloat16, device="cuda")
+    ys, off = [], 0
+    for p, _, _, _ in packed:
+        ys.append(y_all[off:off + p.N].view(1, p.N))
+        off += p.N
+    n0 = q4.q4_debug_launch_count()
+    q4.q4_matmul_batch([(x_down if p.K == 11264 else x, c, s, b, y) for (p, c, s, b), y in zip(packed, ys)])
+    assert q4.q4_debug_launch_count() - n0 == 1, "the step is one launch"
+    singles = [q4.q4_matmul(x_down if p.K == 11264 else x, c, s, b) for p, c, s, b in packed]
+    torch.cuda.synchronize()
+    for (p, _, _, _), y, y1 in zip(packed, ys, singles):
+        assert torch.equal(y.view(torch.int16), y1.view(torch.int16)), p.name
+    worst = 0.0
+    for i, ((p, c, s, b), y) in enumerate(zip(packed, ys)):
+        xi = x_down if p.K == 11264 else x
+        rows = sample_rows(p.N, 8, seed=1000 + i)
+        worst = max(worst, check_matmul(xi, c, s, b, y, rows=rows, what=p.name))
+    assert worst < 4e-3
+    assert q4.q4_device_status() == 0

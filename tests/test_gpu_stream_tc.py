@@ -31,9 +31,9 @@ ROWS_PER_TILE = {256: 16, 768: 16, 1024: 16, 2816: 16, 4096: 16, 8192: 8, 11264:
 def _gpu():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    q4.q4_debug_device_flags(clear=True)
+    q4.q4_device_status(clear=True)
     yield
-    assert q4.q4_debug_device_flags() == 0, "a bounded wait gave up inside a kernel"
+    assert q4.q4_device_status() == 0, "a bounded wait gave up inside a kernel"
 
 
 def _packed(N, K, seed, tensor):

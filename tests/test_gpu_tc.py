@@ -23,9 +23,9 @@ DEV = "cuda"
 def _gpu():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    q4.q4_debug_device_flags(clear=True)
+    q4.q4_device_status(clear=True)
     yield
-    assert q4.q4_debug_device_flags() == 0, "a bounded wait gave up inside a kernel"
+    assert q4.q4_device_status() == 0, "a bounded wait gave up inside a kernel"
 
 
 def _packed(N, K, seed, tensor):

@@ -47,7 +47,8 @@ __all__ = [
     "q8_quantize",
     "q8_dequantize",
     "q8_matmul",
-    "q4_debug_device_flags",
+    "q4_device_status",
+    "q4_check_device",
     "q4_debug_launch_count",
 ]
 
@@ -79,7 +80,7 @@ SIGNATURES = {
     "q8_dequantize": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),
     "q8_matmul": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P]),
     "q4_last_error": (ctypes.c_char_p, []),
-    "q4_debug_device_flags": (_INT, [_INT]),
+    "q4_device_status": (_INT, [_INT]),
     "q4_debug_launch_count": (ctypes.c_ulonglong, []),
 }
 
@@ -222,12 +223,7 @@ def q4_matmul(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases
     M, K = _matmul_shapes(x, codes, scales, biases, None)
     N = codes.shape[0]
     dev = x.device
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    else:
-        _want(out, "out", torch.bfloat16, 2)
-        if out.shape != (M, N):
-            raise ValueError(f"out must be [{M}, {N}]")
+    out = _out(out, M, N, dev)
     with torch.cuda.device(dev):
         _check(lib().q4_matmul(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N, group, _ptr(out),
                                _stream(dev)))
@@ -244,12 +240,7 @@ def q4_matmul_step(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, b
         raise ValueError(f"stacked rows {rows} not divisible by num_steps {num_steps}")
     N = rows // num_steps
     dev = x.device
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    else:
-        _want(out, "out", torch.bfloat16, 2)
-        if out.shape != (M, N):
-            raise ValueError(f"out must be [{M}, {N}]")
+    out = _out(out, M, N, dev)
     with torch.cuda.device(dev):
         _check(lib().q4_matmul_step(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N, num_steps, step,
                                     group, _ptr(out), _stream(dev)))
@@ -413,12 +404,22 @@ def q8_matmul(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases
     return out
 
 
-def q4_debug_device_flags(clear: bool = False) -> int:
-    """Bounded-wait flags of the current device (synchronizes); 0 means none fired."""
-    r = lib().q4_debug_device_flags(1 if clear else 0)
+def q4_device_status(clear: bool = False) -> int:
+    """Kernel status flags of the current device (synchronizes); 0 means no
+    bounded wait gave up.  While nonzero, results enqueued since the flags were
+    last cleared are invalid (the kernels wrote NaN where they gave up)."""
+    r = lib().q4_device_status(1 if clear else 0)
     if r < 0:
         raise Q4Error(6, "could not read device flags")
     return r
+
+
+def q4_check_device(clear: bool = True) -> None:
+    """Raise Q4Error if a kernel on the current device gave up a bounded wait
+    since the flags were last cleared (synchronizes; clears them by default)."""
+    r = q4_device_status(clear)
+    if r != 0:
+        raise Q4Error(6, f"a libq4 kernel gave up a bounded wait (flags {r:#x}); recent results are invalid")
 
 
 def q4_debug_launch_count() -> int:

@@ -1,7 +1,7 @@
 // q4_api.cu -- the extern "C" boundary of libq4 (declared in include/q4.h):
 // argument validation on the host, device checks, dispatch to the kernels.
-// Nothing throws across the boundary; a non-OK status means nothing was
-// enqueued on the stream.
+// Nothing throws across the boundary; a non-OK status from validation means
+// nothing was enqueued on the stream.
 #include "q4.h"
 #include "q4_internal.h"
 
@@ -107,56 +107,37 @@ q4_status check_epilogue(const char* who, int32_t epi, int32_t reserved, const u
 
 // Enqueues a validated, non-empty list.  Each problem takes the kernel it
 // would take alone (so a batched result is bit-identical to the single
-// call); problems on the bulk-copy GEMV and on the weight-streaming kernel
-// share a launch per path.  A SwiGLU problem bound for a tensor-core kernel
-// becomes two problems: the gate into y, then the up projection with the
-// silu-multiply epilogue reading y, enqueued after every first pass.
+// call): the weight-streaming kernel where it takes the problem (3..8
+// activation rows), else the tensor-core tiles (3 or more rows), else the
+// CUDA-core GEMV.  Problems on the bulk-copy GEMV and on the weight-streaming
+// kernel share a launch per path; SwiGLU problems run in one pass on every
+// path.  Every host-side step that can fail for a valid call (tensor-map
+// encoding, configuration checks) runs before the first launch.
 q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& dev, cudaStream_t cs,
                        const char* what) {
-  std::vector<MatmulArgs> gemv, streamed, tc, streamed_up, tc_up;
+  std::vector<MatmulArgs> gemv, streamed;
+  thread_local std::vector<TcLaunch> tc;
+  tc.clear();
   for (const MatmulArgs& a : list) {
-    if (a.fused()) {
-      MatmulArgs g = a, u = a;
-      g.up_codes = u.up_codes = nullptr;
-      g.up_scales = u.up_scales = nullptr;
-      g.up_biases = u.up_biases = nullptr;
-      u.codes = a.up_codes;
-      u.scales = a.up_scales;
-      u.biases = a.up_biases;
-      u.epi = kEpiSiluMul;
-      u.r = a.y;
-      if (stream_supported(g, dev) && stream_supported(u, dev)) {
-        streamed.push_back(g);
-        streamed_up.push_back(u);
-      } else if (a.M >= kTensorCoreMinRows && tc_supported(g) && tc_supported(u)) {
-        tc.push_back(g);
-        tc_up.push_back(u);
-      } else {
-        gemv.push_back(a);
-      }
-    } else if (stream_supported(a, dev)) {
+    if (stream_supported(a, dev)) {
       streamed.push_back(a);
     } else if (a.M >= kTensorCoreMinRows && tc_supported(a)) {
-      tc.push_back(a);
+      tc.emplace_back();
+      const cudaError_t e = plan_tc(a, dev, &tc.back());
+      if (e != cudaSuccess) return from_cuda(e, what);
     } else {
       gemv.push_back(a);
     }
   }
   q4_status st = Q4_OK;
-  for (const MatmulArgs& a : tc)
-    if ((st = from_cuda(launch_tc(a, cs, dev), what)) != Q4_OK) return st;
+  for (const TcLaunch& t : tc)
+    if ((st = from_cuda(launch_planned_tc(t, cs), what)) != Q4_OK) return st;
   if (!streamed.empty() &&
       (st = from_cuda(launch_stream_batch(streamed.data(), static_cast<int>(streamed.size()), cs, dev), what)) != Q4_OK)
     return st;
   if (!gemv.empty() &&
       (st = from_cuda(launch_gemv_batch(gemv.data(), static_cast<int>(gemv.size()), cs, dev), what)) != Q4_OK)
     return st;
-  if (!streamed_up.empty() &&
-      (st = from_cuda(launch_stream_batch(streamed_up.data(), static_cast<int>(streamed_up.size()), cs, dev), what)) !=
-          Q4_OK)
-    return st;
-  for (const MatmulArgs& a : tc_up)
-    if ((st = from_cuda(launch_tc(a, cs, dev), what)) != Q4_OK) return st;
   return Q4_OK;
 }
 
@@ -207,6 +188,18 @@ const DeviceInfo* current_device_info() {
       return nullptr;
     }
     d.smem_optin = static_cast<size_t>(smem_optin);
+    // The kernels' one-time settings on this device (only on the GPU they
+    // are built for; check_device rejects any other before a launch).
+    // cudaFuncSetAttribute applies to the current device, which is `dev`.
+    if (d.cc_major == 10 && d.cc_minor == 0) {
+      if ((e = gemv_prepare_device(d)) == cudaSuccess && (e = tc_prepare_device(d)) == cudaSuccess &&
+          (e = stream_prepare_device(d)) == cudaSuccess)
+        e = q8_prepare_device(d);
+      if (e != cudaSuccess) {
+        fail(Q4_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(e));
+        return nullptr;
+      }
+    }
     g_devices[dev] = d;
     g_device_ready[dev].store(true, std::memory_order_release);
   }
@@ -368,7 +361,7 @@ const char* q4_last_error(void) { return t_last_error; }
 
 unsigned long long q4_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-int q4_debug_device_flags(int clear) {
+int q4_device_status(int clear) {
   unsigned int f = 0, t = 0, s = 0;
   if (gemv_device_flags(&f, clear != 0) != cudaSuccess || tc_device_flags(&t, clear != 0) != cudaSuccess ||
       stream_device_flags(&s, clear != 0) != cudaSuccess)

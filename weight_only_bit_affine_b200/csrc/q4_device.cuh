@@ -13,7 +13,7 @@ namespace q4 {
 
 // Set (never cleared by kernels) when a bounded wait gives up.  Each
 // translation unit has its own copy; the host reads and clears them through
-// q4_debug_device_flags().
+// q4_device_status().
 enum : unsigned int { kFlagWaitTimeout = 1u };
 static __device__ unsigned int g_device_flags = 0;
 
@@ -140,7 +140,6 @@ __device__ __forceinline__ float silu_f32(float z) { return z / (1.f + expf(-z))
 
 __device__ __forceinline__ uint16_t epilogue_bf16(float acc, int epi, const uint16_t* r, int64_t idx) {
   if (epi == kEpiResidual) return float_to_bf16_bits(acc + bf16_bits_to_float(r[idx]));
-  if (epi == kEpiSiluMul) return float_to_bf16_bits(silu_f32(bf16_bits_to_float(r[idx])) * acc);
   return float_to_bf16_bits(acc);
 }
 

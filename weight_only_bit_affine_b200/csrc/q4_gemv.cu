@@ -242,6 +242,7 @@ struct GemvLaunch {
   GemvProblem prob[NP];
 };
 
+constexpr float kNaN = __builtin_nanf("");  // written by a thread whose bounded wait gave up
 constexpr int kRedSlots = 8;    // tiles of cross-warp partial sums in flight to the epilogue warp
 constexpr int kRedSlotFloats = 64 * 2;  // >= rt * MR * warps-per-team (<= 4 * 22 at MR = 1, 4 * 2 * 12 at MR = 2)
 
@@ -467,7 +468,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         const float* rs = red + slot * kRedSlotFloats;
         for (int i = lane; i < n * MR; i += 32) {
           const int lr = i / MR, m = i - lr * MR;
-          float v = 0.f;
+          float v = dead ? kNaN : 0.f;
           for (int w = 0; w < geo.wpt; ++w) v += rs[i * geo.wpt + w];
           const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row0 + lr;
           if (fused) {
@@ -633,7 +634,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         float* rs = red + slot * kRedSlotFloats;
         if (use_red && !dead && !mbar_wait(&rempty_bar[slot], sph ^ 1u)) dead = true;
         if (compute) {
-          const float tot = transpose_reduce<VP>(vals, lane);
+          const float tot = dead ? kNaN : transpose_reduce<VP>(vals, lane);
           const int idx = lane >> (5 - ilog2(VP));
           const int rr = idx / MR, m = idx % MR;
           const bool holder = (lane & ((32 / VP) - 1)) == 0 && idx < V && rr < nv;
@@ -654,7 +655,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < V; ++i) vals[i] = seg_allreduce_dyn(vals[i], geo.team);
+        for (int i = 0; i < V; ++i) vals[i] = dead ? kNaN : seg_allreduce_dyn(vals[i], geo.team);
         if (j == 0) {
 #pragma unroll
           for (int rr = 0; rr < kRpt; ++rr)
@@ -858,12 +859,6 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   bool epi = false;
   for (int i = 0; i < count; ++i) epi = epi || probs[i].epi != kEpiNone || is_fused(probs[i]);
   auto kern = epi ? gemv_kernel<MR, kThreads, NP, true> : gemv_kernel<MR, kThreads, NP, false>;
-  static PerDeviceOnce attr_once[2];
-  if (attr_once[epi].needed(dev.device)) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
-    if (e != cudaSuccess) return e;
-    attr_once[epi].mark(dev.device);
-  }
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, L);
 }
 
@@ -882,6 +877,22 @@ cudaError_t run_problems(std::vector<GemvProblem>& probs, const DeviceInfo& dev,
 }  // namespace
 
 cudaError_t gemv_device_flags(unsigned int* flags, bool clear) { return tu_device_flags(flags, clear); }
+
+cudaError_t gemv_prepare_device(const DeviceInfo& dev) {
+  for (const void* kern : {reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, true>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, true>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true>)}) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dev.smem_optin));
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev) {
   // Activation rows in chunks of at most two; every chunk of every problem

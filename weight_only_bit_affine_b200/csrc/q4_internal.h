@@ -1,6 +1,7 @@
 // q4_internal.h -- host-side launcher declarations shared inside libq4.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <atomic>
 #include <cstdint>
@@ -32,9 +33,9 @@ struct PerDeviceOnce {
 // after the attention, each with its residual add) supplies the steps worth
 // fusing into the matmul that produces their input:
 //   kEpiResidual: y = r + acc        (o and down projections add the residual)
-//   kEpiSiluMul:  y = silu(r) * acc  (the up projection's output times the
-//                                     activated gate, r holding bf16 gate values)
-enum Epilogue : int { kEpiNone = 0, kEpiResidual = 1, kEpiSiluMul = 2 };
+// SwiGLU, y = silu(acc_gate) * acc_up, is a problem with two weights
+// (MatmulArgs::fused()), computed in one pass by every kernel family.
+enum Epilogue : int { kEpiNone = 0, kEpiResidual = 1 };
 
 // Launchers return cudaSuccess or the launch error.  Arguments are already
 // validated by the ABI layer.
@@ -56,8 +57,8 @@ struct MatmulArgs {
   // for kEpiNone; may equal y).
   int epi = 0;
   const uint16_t* r = nullptr;
-  // SwiGLU in one pass (GEMV family only): when up_codes is set, y =
-  // silu(x . w_hat^T) * (x . w_hat_up^T), the up weights with the same shape.
+  // SwiGLU in one pass: when up_codes is set, y = silu(x . w_hat^T) *
+  // (x . w_hat_up^T), the up weights with the same shape.
   const uint8_t* up_codes = nullptr;
   const uint16_t* up_scales = nullptr;
   const uint16_t* up_biases = nullptr;
@@ -78,15 +79,55 @@ cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceIn
 // launch (per chunk size).
 cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
 
-// Tensor-core path (tcgen05) for many activation rows.
-constexpr int64_t kTensorCoreMinRows = 16;
+// Tensor-core tiles (tcgen05, dequantized weights in tensor memory) for
+// three or more activation rows (from kTensorCoreMinRows, or where the
+// weight-streaming kernel does not take a problem).  One launch per problem;
+// plan_tc does every host-side step (tensor-map encoding, configuration
+// checks), so a call can plan all its problems before launching any.
+constexpr int64_t kTensorCoreMinRows = 3;
 bool tc_supported(const MatmulArgs& a);
-cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev);
+struct TcParams {
+  const uint16_t* scales;     // [N, K/32] (the gate's, for SwiGLU)
+  const uint16_t* biases;
+  const uint16_t* up_scales;  // SwiGLU: the up weight's; else NULL
+  const uint16_t* up_biases;
+  uint16_t* y;                // [M, N]
+  const uint16_t* r;          // residual [M, N] (kEpiResidual), else NULL
+  int64_t M, N;
+  int K;
+  int epi;                    // kEpiNone / kEpiResidual (SwiGLU: nacc == 2)
+  int bn;                     // activation rows per tile (multiple of 16, <= 256)
+  int nacc;                   // accumulators: 1, or 2 for SwiGLU (gate, up)
+  int splits;                 // CTAs per cluster along K
+  int stages;
+  int a_slots;                // A ring slots in tensor memory
+  uint32_t stage_bytes, b_atom_bytes;
+  uint32_t a_col0;            // first tensor-memory column of the A ring
+  uint32_t idesc;             // tcgen05 instruction descriptor
+};
+struct TcLaunch {
+  CUtensorMap tmap_x, tmap_codes, tmap_up;
+  TcParams p;
+  dim3 grid;
+  size_t smem;
+  int atoms;  // 64-wide K atoms per pipeline stage
+};
+cudaError_t plan_tc(const MatmulArgs& a, const DeviceInfo& dev, TcLaunch* out);
+cudaError_t launch_planned_tc(const TcLaunch& plan, cudaStream_t stream);
 
-// Tensor-core weight streaming (tcgen05, A operand in tensor memory) for
-// three or four activation rows; several problems share one launch.
+// Tensor-core weight streaming (tcgen05, A operand in tensor memory, segmented
+// K) for kStreamMinRows..kStreamMaxRows activation rows; several problems share
+// one launch.
+constexpr int kStreamMinRows = 3, kStreamMaxRows = 8;
 bool stream_supported(const MatmulArgs& a, const DeviceInfo& dev);
 cudaError_t launch_stream_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
+
+// One-time settings of a device's kernels (dynamic shared memory, cluster
+// sizes), made before the first launch on the device.
+cudaError_t gemv_prepare_device(const DeviceInfo& dev);
+cudaError_t tc_prepare_device(const DeviceInfo& dev);
+cudaError_t stream_prepare_device(const DeviceInfo& dev);
+cudaError_t q8_prepare_device(const DeviceInfo& dev);
 
 // Counts every kernel launch libq4 enqueues (host side).
 void count_launch();

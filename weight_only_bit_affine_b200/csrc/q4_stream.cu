@@ -1,16 +1,16 @@
-// q4_stream.cu -- tensor-core weight streaming for three or four activation
+// q4_stream.cu -- tensor-core weight streaming for three to eight activation
 // rows (batched decode): the affine Q4 group-32 matmul
 //
-//   y[m,n] = sum_k x[m,k] * w_hat[n,k],   w_hat = bf16(s*q + b)  (group 32 along k)
+//   y[m,n] = sum_k x[m,k] * w_hat[n,k],   w_hat = s*q + b  (group 32 along k)
 //
 // with the products and the fp32 accumulation done by the 5th-generation
 // tensor cores (tcgen05.mma, kind::f16) and the CUDA cores doing nothing but
-// the dequantization (about two instructions per weight, whatever the number
-// of activation rows).  At three or four rows the CUDA-core GEMV, which works
-// on pairs of rows, reads the weights twice and multiplies every weight by
-// every row on the CUDA cores; this kernel reads them once and the rows cost
-// tensor-core time only.  (At one or two rows the GEMV is faster: measured
-// 4.7 TB/s at one row against this kernel's 2.7.)
+// the dequantization, whatever the number of activation rows.  At these row
+// counts the CUDA-core GEMV, which works on pairs of rows, would read the
+// weights once per pair and multiply every weight by every row on the CUDA
+// cores; this kernel reads them once and the rows cost tensor-core time only.
+// Each weight enters the MMA as two bf16 parts hi + lo (q4_tcgen05.cuh,
+// split_hi_lo), within ~2^-16 of the exact s*q + b.
 //
 // Segmented-K tiles.  The MMA's 128 rows (tensor-memory lanes) are not 128
 // weight rows: a tile is R weight rows x `segs` segments of K (R * segs =
@@ -34,6 +34,11 @@
 // and B holds each segment's x in the same rotated order.  The segments of a
 // row sit in one warp, so the epilogue sums them with shuffles.
 //
+// SwiGLU (gate and up weights of the same shape) in one pass: each tile of a
+// SwiGLU problem is two consecutive "virtual" tiles, the gate's R rows and
+// then the same rows of the up weight; the epilogue keeps the gate's fp32
+// sums in registers and writes silu(gate) * up when the up tile completes.
+//
 // Per CTA (one per SM, 768 threads):
 //   warp 0       producer: three bulk copies per tile;
 //   warps 1..3   MMA issue (warp 1 also allocates tensor memory): issuer i
@@ -46,10 +51,9 @@
 //                result never depends on the batch;
 //   warps 4..19  dequantize: four groups of four warps (one warp per
 //                tensor-memory lane quarter) take 64-wide K chunks in turn;
-//                a thread turns 64 codes of its (row, segment) into 32 bf16x2
-//                words -- "128 + q" by one LOP3 per two codes, q by an exact
-//                packed subtract, bf16(s*q + b) by one packed FMA (one
-//                rounding, as the dequantizer computes it) -- and stores them
+//                a thread turns 64 codes of its (row, segment) into 32 hi and
+//                32 lo bf16 pairs -- "128 + q" by one LOP3 per two codes, q by
+//                an exact packed subtract, then split_hi_lo -- and stores them
 //                to tensor memory (tcgen05.st);
 //   warps 20..23 epilogue: per tile, read the diagonals of the issuers' fp32
 //                tiles from tensor memory, sum them and the segments
@@ -57,10 +61,11 @@
 //                its B operand.
 // The code pairs come out as (q[t], q[t+4]) of each 8-code word; the B
 // operand is built with the same order of k, so the products pair up.
-// Every wait is bounded (q4_device.cuh); programmatic dependent launch as in
-// the GEMV family.
+// Every wait is bounded (q4_device.cuh); a thread whose wait gave up writes
+// NaN.  Programmatic dependent launch as in the GEMV family.
 #include "q4_device.cuh"
 #include "q4_internal.h"
+#include "q4_tcgen05.cuh"
 
 #include <algorithm>
 #include <cstdint>
@@ -76,33 +81,38 @@ namespace {
 constexpr bool kSleepWaits = Q4_STREAM_WAIT_SLEEP != 0;
 
 constexpr int kLanes = 128;                                  // tensor-memory lanes = MMA rows
-constexpr int kChunkK = 64;                                  // K per lane per A chunk (32 columns)
+constexpr int kChunkK = 64;                                  // K per lane per A chunk
+constexpr int kChunkCols = 64;                               // A chunk in tensor memory: hi (32 columns), lo (32)
 constexpr int kGroups = 4;                                   // dequantizing warp groups
 constexpr int kMaxIssuers = 3;                               // MMA-issuing warps
 constexpr int kFirstDqWarp = 1 + kMaxIssuers;                // 4
 constexpr int kFirstEpiWarp = kFirstDqWarp + 4 * kGroups;   // 20
 constexpr int kThreads = 32 * (kFirstEpiWarp + 4);           // 768: 6 warps per SM sub-partition, <= 80 registers
-constexpr int kMaxRows = 4;                                  // activation rows per launch
-constexpr int kMinRows = 3;  // below this the CUDA-core GEMV is faster (it reads the weights once for 1-2 rows)
+constexpr int kMaxRows = kStreamMaxRows;                     // activation rows per launch
+constexpr int kMinRows = kStreamMinRows;  // below this the CUDA-core GEMV is faster (it reads the weights once for 1-2 rows)
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxASlots = 16;  // A ring in tensor memory: up to 16 chunks of 32 columns
+constexpr int kMaxASlots = 8;   // A ring in tensor memory: up to 8 chunks of 64 columns
 constexpr int kMaxStages = 12;
 constexpr int kMaxProblems = 256;
 constexpr int kFewProblems = 4;
+constexpr float kNaN = __builtin_nanf("");
 
 struct StreamProblem {
   const uint16_t* x;  // [M, K]
   const uint8_t* codes;
   const uint16_t* scales;
   const uint16_t* biases;
+  const uint8_t* up_codes;  // SwiGLU: the up weight (NULL otherwise)
+  const uint16_t* up_scales;
+  const uint16_t* up_biases;
   uint16_t* y;         // [M, N]
-  const uint16_t* r;   // epilogue operand [M, N] (kEpiResidual / kEpiSiluMul), else NULL
+  const uint16_t* r;   // residual [M, N] (kEpiResidual), else NULL
   int64_t N;
   int64_t byte_begin;  // work offset of the first tile (packed bytes of all tiles before)
   int32_t K;
   int32_t segs;        // K segments per weight row; R = 128 / segs rows per tile
-  int32_t tile_bytes;  // packed bytes of a full tile (the unit of work balancing)
-  int32_t epi;         // output epilogue (q4_device.cuh)
+  int32_t tile_bytes;  // packed bytes of a full tile (both weights for SwiGLU): the unit of work balancing
+  int32_t epi;         // output epilogue (q4_internal.h)
 };
 
 template <int NP>
@@ -113,79 +123,7 @@ struct StreamLaunch {
   StreamProblem prob[NP];
 };
 
-// ---- tcgen05 wrappers -------------------------------------------------------
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// K-major operand with the 128-byte swizzle: rows of 128 bytes, 8-row groups
-// 1024 bytes apart, base 1024-byte aligned.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);  // start address
-  d |= static_cast<uint64_t>(16u >> 4) << 16;                // leading byte offset (unused)
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;              // stride byte offset
-  d |= static_cast<uint64_t>(1) << 46;                       // descriptor version
-  d |= static_cast<uint64_t>(2) << 61;                       // 128-byte swizzle
-  return d;
-}
-
-// D (tensor memory) [+]= A (tensor memory) x B (shared memory descriptor).
-__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
-      ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-
-__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// W (8, 16 or 32) consecutive fp32 columns of this thread's lane into r;
-// complete with tmem_wait_ld().
-template <int W>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[W]) {
-  if constexpr (W == 8) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
-  } else if constexpr (W == 16) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-  } else {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-  }
-}
+__device__ __forceinline__ bool is_swiglu(const StreamProblem& P) { return P.up_codes != nullptr; }
 
 template <int W>
 __device__ __forceinline__ float pick(const uint32_t (&r)[W], int sel) {
@@ -213,31 +151,24 @@ __device__ __forceinline__ void gather_diag(uint32_t base, uint32_t issuer_strid
   }
 }
 
-// tcgen05 instruction descriptor: D fp32, A and B bf16, both K-major, M = 128.
-__device__ __forceinline__ uint32_t make_idesc(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
-         (static_cast<uint32_t>(kLanes >> 4) << 24);
-}
-
-
-// Eight codes (one word: q0..q7 of eight consecutive k) -> four bf16x2 words
-// of w_hat for the k pairs (t, t + 4), t = 0..3: "128 + q" by one LOP3 per
-// pair (0x43004300 is bf16 (128, 128), whose last significand bit weighs 1),
-// q by an exact packed subtract, bf16(s*q + b) by one packed FMA (one
-// rounding).  One PTX block with the two constants passed in registers (held
-// by the caller across the loop), so none of them is rebuilt per use.
-__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t s2, uint32_t b2, uint32_t mask, uint32_t magic,
-                                             uint32_t* o) {
-  asm("{\n\t.reg .b32 t1, t2, t3, v0, v1, v2, v3;\n\t"
+// Eight codes (one word: q0..q7 of eight consecutive k) -> the hi and lo
+// bf16 parts of w_hat for the k pairs (t, t + 4), t = 0..3: "128 + q" by one
+// LOP3 per pair (0x43004300 is bf16 (128, 128), whose last significand bit
+// weighs 1), q by an exact packed subtract, then split_hi_lo.  The LOP3
+// constants come in registers held by the caller across its loop.
+__device__ __forceinline__ void dequant_word(uint32_t w, uint16_t s, float b, uint32_t mask, uint32_t magic,
+                                             uint32_t* hi, uint32_t* lo) {
+  uint32_t v[4];
+  asm("{\n\t.reg .b32 t1, t2, t3;\n\t"
       "shr.b32 t1, %4, 4;\n\tshr.b32 t2, %4, 8;\n\tshr.b32 t3, %4, 12;\n\t"
-      "lop3.b32 v0, %4, %7, %8, 0xEA;\n\tlop3.b32 v1, t1, %7, %8, 0xEA;\n\t"
-      "lop3.b32 v2, t2, %7, %8, 0xEA;\n\tlop3.b32 v3, t3, %7, %8, 0xEA;\n\t"
-      "sub.rn.bf16x2 v0, v0, %8;\n\tsub.rn.bf16x2 v1, v1, %8;\n\t"
-      "sub.rn.bf16x2 v2, v2, %8;\n\tsub.rn.bf16x2 v3, v3, %8;\n\t"
-      "fma.rn.bf16x2 %0, v0, %5, %6;\n\tfma.rn.bf16x2 %1, v1, %5, %6;\n\t"
-      "fma.rn.bf16x2 %2, v2, %5, %6;\n\tfma.rn.bf16x2 %3, v3, %5, %6;\n\t}"
-      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
-      : "r"(w), "r"(s2), "r"(b2), "r"(mask), "r"(magic));
+      "lop3.b32 %0, %4, %5, %6, 0xEA;\n\tlop3.b32 %1, t1, %5, %6, 0xEA;\n\t"
+      "lop3.b32 %2, t2, %5, %6, 0xEA;\n\tlop3.b32 %3, t3, %5, %6, 0xEA;\n\t"
+      "sub.rn.bf16x2 %0, %0, %6;\n\tsub.rn.bf16x2 %1, %1, %6;\n\t"
+      "sub.rn.bf16x2 %2, %2, %6;\n\tsub.rn.bf16x2 %3, %3, %6;\n\t}"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+      : "r"(w), "r"(mask), "r"(magic));
+#pragma unroll
+  for (int t = 0; t < 4; ++t) split_hi_lo(v[t], s, b, kBf16MinusOne, hi[t], lo[t]);
 }
 
 // x[k..k+8) (one 16-byte run) in the (t, t + 4) pair order of dequant_word.
@@ -263,7 +194,8 @@ struct ProblemShape {
 };
 
 // The tiles of problem p that this CTA owns: those whose first byte (in the
-// work order of all problems' tiles) falls in [lo, hi).
+// work order of all problems' tiles) falls in [lo, hi).  A SwiGLU problem's
+// tile is its gate and up rows together, so the two always go to one CTA.
 __device__ __forceinline__ void tile_range(const StreamProblem& P, int64_t lo, int64_t hi, int64_t& j0, int64_t& j1) {
   const int64_t R = kLanes / P.segs;
   const int64_t tiles = (P.N + R - 1) / R;
@@ -277,8 +209,17 @@ __device__ __forceinline__ void tile_range(const StreamProblem& P, int64_t lo, i
   j1 = first_from(hi);
 }
 
-// EPI: some problem of the launch has an output epilogue; the plain
-// instantiation keeps the epilogue's code out of the kernel.
+// Virtual tiles (v) of problem P for this CTA: [v0, v1); v maps to weight
+// tile v >> sh and, for SwiGLU (sh = 1), to the gate (v even) or up (v odd).
+__device__ __forceinline__ void vtile_range(const StreamProblem& P, int64_t lo, int64_t hi, int64_t& v0, int64_t& v1,
+                                            int& sh) {
+  int64_t j0, j1;
+  tile_range(P, lo, hi, j0, j1);
+  sh = is_swiglu(P) ? 1 : 0;
+  v0 = j0 << sh;
+  v1 = j1 << sh;
+}
+
 template <int NP, bool EPI>
 __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_constant__ StreamLaunch<NP> L) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -313,12 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     mbar_init(bempty, kMaxIssuers);
     fence_mbar_init();
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -355,21 +291,24 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     uint32_t ph = 0;
     for (int p = 0; p < L.count; ++p) {
       const StreamProblem& P = L.prob[p];
-      int64_t j0, j1;
-      tile_range(P, lo, hi, j0, j1);
+      int64_t v0, v1;
+      int sh;
+      vtile_range(P, lo, hi, v0, v1, sh);
       const int R = kLanes / P.segs;
       const uint32_t row_bytes = static_cast<uint32_t>(P.K / 2), sb_row = static_cast<uint32_t>(P.K / 16);
-      for (int64_t j = j0; j < j1; ++j) {
+      for (int64_t v = v0; v < v1; ++v) {
         if (lane == 0) {
           if (!dead && !mbar_wait<kSleepWaits>(&empty[s], ph ^ 1u)) dead = true;
-          const int64_t row0 = j * R;
+          const int64_t row0 = (v >> sh) * R;
+          const bool up = sh && (v & 1);
           const uint32_t rows = static_cast<uint32_t>((P.N - row0 < R) ? P.N - row0 : R);
           uint8_t* st = ring + static_cast<size_t>(s) * L.stage_bytes;
           mbar_arrive_expect_tx(&full[s], rows * (row_bytes + 2 * sb_row));
           // the tile's codes, scales and biases: three contiguous runs
-          bulk_g2s(st, P.codes + row0 * row_bytes, rows * row_bytes, &full[s]);
-          bulk_g2s(st + R * row_bytes, P.scales + row0 * (P.K / 32), rows * sb_row, &full[s]);
-          bulk_g2s(st + R * (row_bytes + sb_row), P.biases + row0 * (P.K / 32), rows * sb_row, &full[s]);
+          bulk_g2s(st, (up ? P.up_codes : P.codes) + row0 * row_bytes, rows * row_bytes, &full[s]);
+          bulk_g2s(st + R * row_bytes, (up ? P.up_scales : P.scales) + row0 * (P.K / 32), rows * sb_row, &full[s]);
+          bulk_g2s(st + R * (row_bytes + sb_row), (up ? P.up_biases : P.biases) + row0 * (P.K / 32), rows * sb_row,
+                   &full[s]);
         }
         if (++s == L.stages) { s = 0; ph ^= 1u; }
       }
@@ -387,12 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
       const uint32_t a_base = tmem + a_col0;
       for (int p = 0; p < L.count; ++p) {
         const StreamProblem& P = L.prob[p];
-        int64_t j0, j1;
-        tile_range(P, lo, hi, j0, j1);
-        if (j0 >= j1) continue;
+        int64_t v0, v1;
+        int sh;
+        vtile_range(P, lo, hi, v0, v1, sh);
+        if (v0 >= v1) continue;
         const ProblemShape S(P, L.M);
         const bool active = me < S.issuers;
-        const uint32_t idesc = make_idesc(S.nb);
+        const uint32_t idesc = idesc_bf16_m128(S.nb);
         const uint32_t atom16 = static_cast<uint32_t>(S.nb) * 128u >> 4;  // B atom size in 16-byte units
         // B of the previous problem is free once its MMAs are done.  Waiting
         // for this problem's B also means the epilogue has drained every
@@ -400,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
         if (lp > 0) tc_commit(bempty);
         if (!dead && !mbar_wait<kSleepWaits>(bfull, static_cast<uint32_t>(lp & 1))) dead = true;
         tc_fence_after();
-        for (int64_t j = j0; j < j1; ++j, ++gt) {
+        for (int64_t v = v0; v < v1; ++v, ++gt) {
           const int db = static_cast<int>(gt & 1);
           const uint32_t dt = tmem + static_cast<uint32_t>(2 * me + db) * S.dstride;
           // every issuer waits, so none can arrive twice on one phase of dfull
@@ -413,15 +353,14 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
               while (slot >= A) { slot -= A; sph ^= 1u; }
               if (!dead && !mbar_wait<kSleepWaits>(&afull[slot], sph)) dead = true;
               tc_fence_after();
-              const uint32_t at = a_base + static_cast<uint32_t>(slot) * 32u;
+              const uint32_t at = a_base + static_cast<uint32_t>(slot) * kChunkCols;
               const uint64_t bd = bdesc0 + static_cast<uint64_t>(c) * atom16;
+              const int ksteps = c < S.full_chunks ? 4 : 2;
               // the first MMA of this issuer in the tile overwrites its accumulator
-              tc_mma_ts(dt, at, bd, idesc, c >= S.issuers ? 1u : 0u);
-              tc_mma_ts(dt, at + 8u, bd + 2u, idesc, 1u);
-              if (c < S.full_chunks) {
-                tc_mma_ts(dt, at + 16u, bd + 4u, idesc, 1u);
-                tc_mma_ts(dt, at + 24u, bd + 6u, idesc, 1u);
-              }
+              for (int kk = 0; kk < ksteps; ++kk)  // hi
+                tc_mma_ts(dt, at + 8u * kk, bd + 2u * kk, idesc, (c >= S.issuers || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < ksteps; ++kk)  // lo, same activations
+                tc_mma_ts(dt, at + 32u + 8u * kk, bd + 2u * kk, idesc, 1u);
               tc_commit(&aempty[slot]);
             }
           }
@@ -449,14 +388,15 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     uint32_t ph0 = 0;         // and its phase
     for (int p = 0; p < L.count; ++p) {
       const StreamProblem& P = L.prob[p];
-      int64_t j0, j1;
-      tile_range(P, lo, hi, j0, j1);
-      if (j0 >= j1) continue;
+      int64_t v0, v1;
+      int sh;
+      vtile_range(P, lo, hi, v0, v1, sh);
+      if (v0 >= v1) continue;
       const ProblemShape S(P, L.M);
       const int r = tl / S.segs, seg = tl % S.segs;  // this lane: row r, segment seg
       const int rot = seg % S.pieces;                  // its code runs, rotated by seg
       const int groups = P.K / 32;
-      for (int64_t j = j0; j < j1; ++j, gc += static_cast<uint32_t>(S.chunks)) {
+      for (int64_t v = v0; v < v1; ++v, gc += static_cast<uint32_t>(S.chunks)) {
         if (!dead && !mbar_wait<kSleepWaits>(&full[s], ph)) dead = true;
         const uint8_t* st = ring + static_cast<size_t>(s) * L.stage_bytes;
         const uint8_t* crow = st + r * (P.K / 2) + seg * (S.kseg / 2);  // the segment's 16-byte code runs
@@ -468,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
           uint32_t sph = ph0;
           while (slot >= A) { slot -= A; sph ^= 1u; }
           if (!dead && !mbar_wait<kSleepWaits>(&aempty[slot], sph ^ 1u)) dead = true;
-          const uint32_t taddr = a_addr + static_cast<uint32_t>(slot) * 32u;
-          uint32_t o[16];
+          tc_fence_after();
+          const uint32_t taddr = a_addr + static_cast<uint32_t>(slot) * kChunkCols;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             if (h == 0 || c < S.full_chunks) {
@@ -477,13 +417,18 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
               int run = 2 * c + h + rot;
               if (run >= S.pieces) run -= S.pieces;
               const uint4 cw = *reinterpret_cast<const uint4*>(crow + 16 * run);
-              const uint32_t s2 = __byte_perm(static_cast<uint32_t>(srow[run]), 0, 0x1010);
-              const uint32_t b2 = __byte_perm(static_cast<uint32_t>(brow[run]), 0, 0x1010);
-              dequant_word(cw.x, s2, b2, kmask, kmagic, o + 0);
-              dequant_word(cw.y, s2, b2, kmask, kmagic, o + 4);
-              dequant_word(cw.z, s2, b2, kmask, kmagic, o + 8);
-              dequant_word(cw.w, s2, b2, kmask, kmagic, o + 12);
-              tmem_st_x16(taddr + 16u * h, o);
+              const uint16_t sv = srow[run];
+              const float bv = bf16_bits_to_float(brow[run]);
+              // two words (16 codes) at a time: 8 hi and 8 lo columns
+              uint32_t oh[8], ol[8];
+              dequant_word(cw.x, sv, bv, kmask, kmagic, oh + 0, ol + 0);
+              dequant_word(cw.y, sv, bv, kmask, kmagic, oh + 4, ol + 4);
+              tmem_st_x8(taddr + 16u * h, oh);
+              tmem_st_x8(taddr + 32u + 16u * h, ol);
+              dequant_word(cw.z, sv, bv, kmask, kmagic, oh + 0, ol + 0);
+              dequant_word(cw.w, sv, bv, kmask, kmagic, oh + 4, ol + 4);
+              tmem_st_x8(taddr + 16u * h + 8u, oh);
+              tmem_st_x8(taddr + 32u + 16u * h + 8u, ol);
             }
           }
           tmem_wait_st();
@@ -509,9 +454,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     int64_t gt = 0;
     for (int p = 0; p < L.count; ++p) {
       const StreamProblem& P = L.prob[p];
-      int64_t j0, j1;
-      tile_range(P, lo, hi, j0, j1);
-      if (j0 >= j1) continue;
+      int64_t v0, v1;
+      int sh;
+      vtile_range(P, lo, hi, v0, v1, sh);
+      if (v0 >= v1) continue;
       const ProblemShape S(P, L.M);
       // B: atom c (positions 2c, 2c + 1 of every segment: 64 k) holds rows
       // n = m * segs + s' of 128 bytes, 16-byte runs swizzled as the MMA's
@@ -558,7 +504,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
       // issuers with chunks in a tile (the others' accumulators hold an older tile)
       const int I = S.issuers;
       const uint32_t mask = (1u << (S.chunks < I ? S.chunks : I)) - 1u;
-      for (int64_t j = j0; j < j1; ++j, ++gt) {
+      float gate[kMaxRows];  // SwiGLU: the gate's sums of the current tile, kept for its up tile
+#pragma unroll
+      for (int m = 0; m < kMaxRows; ++m) gate[m] = 0.f;
+      for (int64_t v = v0; v < v1; ++v, ++gt) {
         const int db = static_cast<int>(gt & 1);
         if (!dead && !mbar_wait<kSleepWaits>(&dfull[db], static_cast<uint32_t>((gt >> 1) & 1))) dead = true;
         tc_fence_after();
@@ -577,14 +526,24 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
 #pragma unroll
         for (int m = 0; m < kMaxRows; ++m)
           for (int o = 1; o < S.segs; o <<= 1) part[m] += __shfl_xor_sync(0xFFFFFFFFu, part[m], o);
-        const int64_t row = j * S.R + rq;
+        if (sh && !(v & 1)) {  // a SwiGLU gate tile: keep its sums for the up tile that follows
+#pragma unroll
+          for (int m = 0; m < kMaxRows; ++m) gate[m] = part[m];
+          continue;
+        }
+        const int64_t row = (v >> sh) * S.R + rq;
         if (seg == 0 && row < P.N) {
 #pragma unroll
           for (int m = 0; m < kMaxRows; ++m)
             if (m < L.M) {
               const int64_t idx = static_cast<int64_t>(m) * P.N + row;
-              if constexpr (EPI) P.y[idx] = epilogue_bf16(part[m], P.epi, P.r, idx);
-              else P.y[idx] = float_to_bf16_bits(part[m]);
+              const float val = dead ? kNaN : part[m];
+              if constexpr (EPI) {
+                if (sh) P.y[idx] = float_to_bf16_bits(silu_f32(gate[m]) * val);
+                else P.y[idx] = epilogue_bf16(val, P.epi, P.r, idx);
+              } else {
+                P.y[idx] = float_to_bf16_bits(val);
+              }
             }
         }
       }
@@ -596,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -635,6 +594,11 @@ Plan plan_of(const MatmulArgs& a) {
 
 constexpr size_t kFixedSmem = 1024 /* alignment */ + 8 * (2 * kMaxStages + 2 * kMaxASlots + 6) + 16;
 
+uint32_t acc_cols_of(uint32_t nb) {
+  const uint32_t issuers = nb <= 16 ? 3u : nb <= 32 ? 2u : 1u;  // as ProblemShape
+  return 2u * issuers * nb;
+}
+
 template <int NP>
 cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev, cudaStream_t stream) {
   static_assert(sizeof(StreamLaunch<NP>) <= 32000, "kernel parameters exceed the launch limit");
@@ -649,6 +613,9 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
     P.codes = a.codes;
     P.scales = a.scales;
     P.biases = a.biases;
+    P.up_codes = a.up_codes;
+    P.up_scales = a.up_scales;
+    P.up_biases = a.up_biases;
     P.y = a.y;
     P.r = a.r;
     P.epi = a.epi;
@@ -656,14 +623,13 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
     P.K = static_cast<int32_t>(a.K);
     P.segs = pl.segs;
     const int R = kLanes / pl.segs;
-    P.tile_bytes = static_cast<int32_t>(R * (a.K / 2 + a.K / 8));
+    P.tile_bytes = static_cast<int32_t>(R * (a.K / 2 + a.K / 8) * (a.fused() ? 2 : 1));
     P.byte_begin = total;
     const int64_t t = (a.N + R - 1) / R;
     total += t * P.tile_bytes;
     tiles += t;
     stage_bytes = std::max(stage_bytes, pl.stage_bytes);
-    const uint32_t issuers = pl.nb <= 16 ? 3u : pl.nb <= 32 ? 2u : 1u;  // as ProblemShape
-    acc_cols = std::max(acc_cols, 2u * issuers * pl.nb);
+    acc_cols = std::max(acc_cols, acc_cols_of(pl.nb));
     b_bytes = std::max(b_bytes, pl.b_bytes);
   }
   const size_t avail = dev.smem_optin - kFixedSmem - b_bytes;
@@ -677,23 +643,17 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
   // A ring as the rest holds (a multiple of 4 chunks: one slot per dequantizing
   // group per turn).
   L.a_col0 = (acc_cols + 31u) & ~31u;
-  L.a_slots = static_cast<int32_t>(std::min<uint32_t>(kMaxASlots, (kTmemCols - L.a_col0) / 32u) & ~3u);
+  L.a_slots = static_cast<int32_t>(std::min<uint32_t>(kMaxASlots, (kTmemCols - L.a_col0) / kChunkCols) & ~3u);
   if (L.a_slots < 4) return cudaErrorInvalidConfiguration;
   L.stage_bytes = stage_bytes;
   L.b_bytes = b_bytes;
   L.total_bytes = total;
-  const size_t smem = kFixedSmem + b_bytes + static_cast<size_t>(stages) * stage_bytes;
+  // All of the SM's shared memory: one CTA per SM (each allocates all 512
+  // tensor-memory columns).
+  const size_t smem = dev.smem_optin;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, tiles)));
   bool epi = false;
-  for (int i = 0; i < count; ++i) epi = epi || list[i].epi != kEpiNone;
-  auto kern = epi ? stream_kernel<NP, true> : stream_kernel<NP, false>;
-  static PerDeviceOnce attr_once[2];
-  if (attr_once[epi].needed(dev.device)) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(dev.smem_optin));
-    if (e != cudaSuccess) return e;
-    attr_once[epi].mark(dev.device);
-  }
+  for (int i = 0; i < count; ++i) epi = epi || list[i].epi != kEpiNone || list[i].fused();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
@@ -705,32 +665,64 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   count_launch();
-  return cudaLaunchKernelEx(&cfg, kern, L);
+  return epi ? cudaLaunchKernelEx(&cfg, stream_kernel<NP, true>, L) : cudaLaunchKernelEx(&cfg, stream_kernel<NP, false>, L);
 }
 
 }  // namespace
 
 cudaError_t stream_device_flags(unsigned int* flags, bool clear) { return tu_device_flags(flags, clear); }
 
+cudaError_t stream_prepare_device(const DeviceInfo& dev) {
+  for (const void* kern : {reinterpret_cast<const void*>(stream_kernel<kFewProblems, false>),
+                           reinterpret_cast<const void*>(stream_kernel<kFewProblems, true>),
+                           reinterpret_cast<const void*>(stream_kernel<kMaxProblems, false>),
+                           reinterpret_cast<const void*>(stream_kernel<kMaxProblems, true>)}) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dev.smem_optin));
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 bool stream_supported(const MatmulArgs& a, const DeviceInfo& dev) {
-#if defined(Q4_STREAM_TC) && Q4_STREAM_TC == 0
-  return false;
-#endif
   if (a.M < kMinRows || a.M > kMaxRows) return false;
-  if (a.fused()) return false;  // one-pass SwiGLU is a GEMV-family problem
-  if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) return false;
+  uintptr_t sb = reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases);
+  if (a.fused()) sb |= reinterpret_cast<uintptr_t>(a.up_scales) | reinterpret_cast<uintptr_t>(a.up_biases);
+  if (sb & 15u) return false;
   if (a.K > (int64_t(1) << 20)) return false;
   const Plan pl = plan_of(a);
-  if (pl.segs == 0) return false;
+  if (pl.segs == 0 || pl.nb > 128) return false;
+  if ((kTmemCols - ((acc_cols_of(pl.nb) + 31u) & ~31u)) / kChunkCols < 4) return false;
   return kFixedSmem + pl.b_bytes + 2 * static_cast<size_t>(pl.stage_bytes) <= dev.smem_optin;
 }
 
+// Problems share a launch while their combined layout fits: every problem
+// fits alone (stream_supported), but the largest stage of one and the
+// largest B operand of another may not fit together.
+bool fits_together(uint32_t stage_bytes, uint32_t b_bytes, uint32_t acc_cols, const DeviceInfo& dev) {
+  if (kFixedSmem + b_bytes + 2 * static_cast<size_t>(stage_bytes) > dev.smem_optin) return false;
+  return (kTmemCols - ((acc_cols + 31u) & ~31u)) / kChunkCols >= 4;
+}
+
 cudaError_t launch_stream_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev) {
-  for (int i = 0; i < count; i += kMaxProblems) {
-    const int n = std::min(kMaxProblems, count - i);
+  int i = 0;
+  while (i < count) {
+    uint32_t sb = 0, bb = 0, ac = 0;
+    int n = 0;
+    while (i + n < count && n < kMaxProblems) {
+      const Plan pl = plan_of(list[i + n]);
+      const uint32_t sb2 = std::max(sb, pl.stage_bytes), bb2 = std::max(bb, pl.b_bytes),
+                     ac2 = std::max(ac, acc_cols_of(pl.nb));
+      if (n > 0 && !fits_together(sb2, bb2, ac2, dev)) break;
+      sb = sb2;
+      bb = bb2;
+      ac = ac2;
+      ++n;
+    }
     cudaError_t e = (n <= kFewProblems) ? run_stream<kFewProblems>(list + i, n, dev, stream)
                                         : run_stream<kMaxProblems>(list + i, n, dev, stream);
     if (e != cudaSuccess) return e;
+    i += n;
   }
   return cudaSuccess;
 }

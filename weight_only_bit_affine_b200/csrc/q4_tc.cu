@@ -1,36 +1,48 @@
-// q4_tc.cu -- tensor-core path of the affine Q4 group-32 matmul for many
-// activation rows (prefill, concurrent conversations: M >= 16).
+// q4_tc.cu -- tensor-core tiles of the affine Q4 group-32 matmul for many
+// activation rows (prefill, concurrent conversations):
 //
 //   y[m,n] = sum_k x[m,k] * w_hat[n,k],   w_hat = s*q + b  (group 32 along k)
 //
-// The packed weights are dequantized tile by tile into shared memory (never
+// The packed weights are dequantized tile by tile into tensor memory (never
 // to HBM) and multiplied on the 5th-generation tensor cores (tcgen05.mma,
 // kind::f16, bf16 x bf16 -> fp32 accumulation in tensor memory).  The Swift
 // blog's prefill batching (voice prompt and prefill as one batched forward)
 // and the four concurrent conversations of "A smaller voice model" are the
 // workloads with several rows.
 //
-// Tile: 128 weight rows (the MMA's M side: D[n, m] = w_hat . x^T, so the
-// output tile is y^T) x BN activation rows (the MMA's N side, 16..256) x a
-// K range; K advances in chunks of 64 (one 128-byte swizzle span of bf16).
-// Per CTA (320 threads):
-//   warp 0      TMA producer: x tile (tensor map, 128-byte swizzle) and the
-//               4 KB code tile (tensor map, 32-byte rows) per chunk;
-//   warp 1      allocates tensor memory; one thread issues 4 MMAs per chunk
-//               and commits them to the stage's "free" barrier;
-//   warps 2..9  dequantize: thread t owns group (t / 128) of weight row
-//               (t % 128) in every chunk: bf16 "128 + q" by PRMT + LOP3, exact
-//               q by a packed subtract, w_hat = fma.rn.bf16x2(q, s, b) (one
-//               rounding), stored in the canonical K-major SWIZZLE_128B layout
-//               the MMA descriptor reads; then the epilogue (tensor memory ->
-//               registers -> bf16 y).
+// Tile: 128 weight rows (the MMA's M side and the 128 tensor-memory lanes:
+// D[n, m] = w_hat . x^T, so the output tile is y^T) x BN activation rows
+// (the MMA's N side, 16..256) x the CTA's K range, walked in atoms of 64
+// inputs (one 128-byte swizzle span of bf16 x).  Each weight enters the MMA
+// as two bf16 parts, hi + lo (q4_tcgen05.cuh, split_hi_lo), so the operand
+// is within ~2^-16 of the exact s*q + b; every atom is two groups of four
+// K16 MMAs (hi, then lo) into the same accumulator.
+//
+// Per CTA (576 threads):
+//   warp 0       TMA producer: per stage, the x tiles (tensor map, 128-byte
+//                swizzle) and the code tile (tensor map, 128 rows x 32 bytes
+//                per atom);
+//   warp 1       allocates tensor memory; one thread issues the MMAs (A from
+//                tensor memory, B = the x tile in shared memory) and commits
+//                them to the barriers that free the A slot and the stage;
+//   warps 2..17  dequantize, in two groups of eight warps taking the atoms in
+//                turn: the thread of lane r and half h turns the 32 codes of
+//                group h of weight row r in an atom into 16 hi and 16 lo
+//                bf16 pairs and stores them to its tensor-memory lane
+//                (tcgen05.st) in the atom's A slot, a ring of slots after
+//                the accumulators; then the epilogue (tensor memory ->
+//                registers -> bf16 y).
+// SwiGLU (gate and up weights of the same shape): the up weight's atoms
+// follow the gate's over the same K range into a second accumulator, and the
+// epilogue writes silu(gate) * up from the two fp32 results.
 // Split-K: when there are too few tiles to fill the GPU, the K range is split
 // across the CTAs of a thread-block cluster, and the fp32 partial tiles are
 // summed through distributed shared memory (no global workspace).
-// Every wait is bounded (q4_device.cuh); programmatic dependent launch as in
-// the GEMV family.
+// Every wait is bounded (q4_device.cuh); a thread whose wait gave up writes
+// NaN.  Programmatic dependent launch as in the GEMV family.
 #include "q4_device.cuh"
 #include "q4_internal.h"
+#include "q4_tcgen05.cuh"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -38,86 +50,30 @@
 #include <algorithm>
 #include <mutex>
 
-#ifndef Q4_TC_WAIT_SLEEP
-#define Q4_TC_WAIT_SLEEP 0
-#endif
-
 namespace q4 {
 namespace {
 
-constexpr int kTileN = 128;        // weight rows per tile (MMA M)
-constexpr int kChunkK = 64;        // K per pipeline stage (one 128-byte bf16 swizzle span)
-constexpr int kSuperK = 256;       // K per scale/bias load (8 groups = 16 bytes per row)
-constexpr int kDequantWarps = 8;
-constexpr int kThreads = 64 + 32 * kDequantWarps;
-constexpr int kATileBytes = kTileN * kChunkK * 2;   // 16 KB
-constexpr int kCodeTileBytes = kTileN * kChunkK / 2;  // 4 KB
+constexpr int kTileN = 128;                  // weight rows per tile (MMA M, tensor-memory lanes)
+constexpr int kAtomK = 64;                   // K per atom (one 128-byte swizzle span of bf16)
+constexpr int kSuperK = 256;                 // K per scale/bias load (8 groups = 16 bytes per row)
+constexpr int kAtomsPerSuper = kSuperK / kAtomK;
+constexpr int kDqGroups = 2;                 // dequantizing warp groups, taking atoms in turn
+constexpr int kDqWarpsPerGroup = 8;          // two per tensor-memory lane quarter (one per group of an atom)
+constexpr int kDqWarps = kDqGroups * kDqWarpsPerGroup;
+constexpr int kThreads = 64 + 32 * kDqWarps;  // 576
+constexpr uint32_t kTmemCols = 512;
+constexpr int kASlotCols = 64;               // one atom of A: hi (32 columns of bf16 pairs), then lo (32)
+constexpr int kMaxASlots = 8;
+constexpr int kMaxStages = 8;
+constexpr int kCodeAtomBytes = kTileN * kAtomK / 2;  // 4 KB
+constexpr float kNaN = __builtin_nanf("");
 
-struct TcParams {
-  const uint16_t* scales;  // [N, K/32]
-  const uint16_t* biases;
-  uint16_t* y;             // [M, N]
-  const uint16_t* r;       // epilogue operand [M, N] (kEpiResidual / kEpiSiluMul), else NULL
-  int64_t M, N;
-  int K;
-  int epi;                 // output epilogue (q4_device.cuh)
-  int bn;          // activation rows per tile (multiple of 16, <= 256)
-  int splits;      // CTAs per cluster along K
-  int stages;
-  uint32_t stage_bytes, b_tile_bytes;
-  uint32_t tmem_cols;
-  uint32_t idesc;  // tcgen05 instruction descriptor
-};
-
-// ---- tcgen05 / TMA wrappers ------------------------------------------------
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// K-major operand tile with the 128-byte swizzle: rows of 128 bytes, 8-row
-// groups 1024 bytes apart (stride byte offset), tile base 1024-byte aligned.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);  // start address
-  d |= static_cast<uint64_t>(16u >> 4) << 16;                // leading byte offset (unused here)
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;              // stride byte offset
-  d |= static_cast<uint64_t>(1) << 46;                       // descriptor version
-  d |= static_cast<uint64_t>(2) << 61;                       // 128-byte swizzle
-  return d;
-}
-
-__device__ __forceinline__ void tc_mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
-      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_ld_x8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void cluster_sync_all() {
@@ -135,35 +91,47 @@ __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t remote_addr) {
   return v;
 }
 
-// ---- the kernel ------------------------------------------------------------
-//
-// A pipeline stage covers ATOMS x 64 inputs k (one or two 128-byte swizzle
-// spans): fewer, larger stages cut the fixed per-stage cost of every role
-// (barrier waits, TMA issue, MMA issue and commit) when shared memory allows
-// at least three of them.
-
-// Output store; the EPI = false instantiation (no epilogue in the launch)
-// keeps the epilogue's code out of the kernel.
+// One output element from the tile's fp32 result(s).
 template <bool EPI>
-__device__ __forceinline__ uint16_t store_tc(float v, const TcParams& p, int64_t idx) {
-  if constexpr (EPI) return epilogue_bf16(v, p.epi, p.r, idx);
-  return float_to_bf16_bits(v);
+__device__ __forceinline__ uint16_t out_tc(float g, float u, const TcParams& p, int64_t idx) {
+  if constexpr (EPI) {
+    if (p.nacc == 2) return float_to_bf16_bits(silu_f32(g) * u);
+    return epilogue_bf16(g, p.epi, p.r, idx);
+  }
+  return float_to_bf16_bits(g);
+}
+
+// Two code words (16 codes in natural k order) -> 8 hi and 8 lo bf16 pairs.
+__device__ __forceinline__ void dequant_words(uint32_t w0, uint32_t w1, uint16_t s, float b, uint32_t (&hi)[8],
+                                              uint32_t (&lo)[8]) {
+  const uint32_t words[2] = {w0, w1};
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const uint32_t wd = words[w], w4 = wd >> 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // bytes [wd.i, wd.i, w4.i, w4.i] -> q[2i] at bits 0..3, q[2i+1] at 16..19
+      const uint32_t pr = __byte_perm(wd, w4, i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
+      const uint32_t v = (pr & 0x000F000Fu) | 0x43004300u;  // (128 + q, 128 + q') exactly
+      const uint32_t q = bf16x2_sub(v, 0x43004300u);          // (q, q') exactly
+      split_hi_lo(q, s, b, kBf16MinusOne, hi[4 * w + i], lo[4 * w + i]);
+    }
+  }
 }
 
 template <int ATOMS, bool EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
-              const __grid_constant__ TcParams p) {
-  constexpr int kStageK = kChunkK * ATOMS;
-  constexpr int kStagesPerSuper = kSuperK / kStageK;
+              const __grid_constant__ CUtensorMap tmap_up, const __grid_constant__ TcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte alignment for the swizzled operand tiles.
+  // 1024-byte alignment for the swizzled x tiles.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint64_t* tma_full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);
-  uint64_t* a_full = tma_full + p.stages;
-  uint64_t* stage_free = a_full + p.stages;
-  uint64_t* accum_full = stage_free + p.stages;
+  uint64_t* stage_free = tma_full + kMaxStages;
+  uint64_t* a_full = stage_free + kMaxStages;
+  uint64_t* a_empty = a_full + kMaxASlots;
+  uint64_t* accum_full = a_empty + kMaxASlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
 
   const int split = static_cast<int>(blockIdx.x);  // == cluster rank along x
@@ -171,24 +139,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t m0 = static_cast<int64_t>(blockIdx.z) * p.bn;
   const int supers = p.K / kSuperK;
   const int sc_begin = split * supers / p.splits, sc_end = (split + 1) * supers / p.splits;
-  const int stage_begin = sc_begin * kStagesPerSuper;
-  const int nstages = (sc_end - sc_begin) * kStagesPerSuper;
+  const int pass_supers = sc_end - sc_begin;
+  const int pass_atoms = pass_supers * kAtomsPerSuper;  // atoms of one weight over this CTA's K range
+  const int natoms = pass_atoms * p.nacc;               // SwiGLU: the up weight's atoms follow the gate's
+  const int k_begin = sc_begin * kSuperK;
 
   if (tid == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&tma_full[s], 1);
-      mbar_init(&a_full[s], kDequantWarps);
       mbar_init(&stage_free[s], 1);
+    }
+    for (int a = 0; a < p.a_slots; ++a) {
+      mbar_init(&a_full[a], kDqWarpsPerGroup);
+      mbar_init(&a_empty[a], 1);
     }
     mbar_init(accum_full, 1);
     fence_mbar_init();
   }
-  if (warp == 1) {  // tensor memory for the fp32 accumulator tile: 128 lanes x bn columns
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(p.tmem_cols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -196,13 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   pdl_wait_predecessors();
 
-  // Stage layout: ATOMS A tiles (128 rows x 128 B each, 16 KB apart), then
-  // ATOMS x tiles (bn rows x 128 B each), then the code tile (128 rows x
-  // 32*ATOMS bytes).
-  const uint32_t b_atom = static_cast<uint32_t>(p.bn) * 128u;
-  auto a_tile = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
-  auto b_tile = [&](int s) { return a_tile(s) + ATOMS * kATileBytes; };
+  // Stage layout: ATOMS x tiles (bn rows x 128 B each), then the code tile
+  // (128 rows x 32 * ATOMS bytes).
+  const uint32_t b_atom = p.b_atom_bytes;
+  auto b_tile = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
   auto c_tile = [&](int s) { return b_tile(s) + ATOMS * b_atom; };
+  const int nsteps = natoms / ATOMS;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -210,134 +177,146 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool dead = false;
       int s = 0;
       uint32_t ph = 0;
-      for (int c = 0; c < nstages; ++c) {
-        if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&stage_free[s], ph ^ 1u)) dead = true;
-        const int k0 = (stage_begin + c) * kStageK;
-        mbar_arrive_expect_tx(&tma_full[s], ATOMS * b_atom + kTileN * kStageK / 2);
+      for (int j = 0; j < nsteps; ++j) {
+        if (!dead && !mbar_wait<false>(&stage_free[s], ph ^ 1u)) dead = true;
+        const int a = j * ATOMS;
+        const bool up = a >= pass_atoms;
+        const int k0 = k_begin + (a - (up ? pass_atoms : 0)) * kAtomK;
+        mbar_arrive_expect_tx(&tma_full[s], ATOMS * (b_atom + kCodeAtomBytes));
 #pragma unroll
         for (int at = 0; at < ATOMS; ++at)
-          tma_load_2d(b_tile(s) + at * b_atom, &tmap_x, k0 + at * kChunkK, static_cast<int>(m0), &tma_full[s]);
-        tma_load_2d(c_tile(s), &tmap_codes, k0 / 2, static_cast<int>(n0), &tma_full[s]);
+          tma_load_2d(b_tile(s) + at * b_atom, &tmap_x, k0 + at * kAtomK, static_cast<int>(m0), &tma_full[s]);
+        tma_load_2d(c_tile(s), up ? &tmap_up : &tmap_codes, k0 / 2, static_cast<int>(n0), &tma_full[s]);
         if (++s == p.stages) { s = 0; ph ^= 1u; }
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     // Waits only for the dequantizing warps: they arrive after having waited
-    // for this stage's TMA themselves, so the x tile is in place too.
+    // for the stage's TMA themselves, so the x tile is in place too.
     if (lane == 0) {
       bool dead = false;
-      int s = 0;
-      uint32_t ph = 0;
-      for (int c = 0; c < nstages; ++c) {
-        if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&a_full[s], ph)) dead = true;
+      const uint32_t a_base = tmem_base + p.a_col0;
+      int slot = 0, s = 0, sub = 0;
+      uint32_t aph = 0, ph = 0;
+      for (int a = 0; a < natoms; ++a) {
+        if (!dead && !mbar_wait<false>(&a_full[slot], aph)) dead = true;
         tc_fence_after();
-        const uint64_t ad = sw128_desc(smem_u32(a_tile(s)));
-        const uint64_t bd = sw128_desc(smem_u32(b_tile(s)));
+        const bool up = a >= pass_atoms;
+        const uint32_t acc = tmem_base + (up ? static_cast<uint32_t>(p.bn) : 0u);
+        const bool first = (a == 0) || (a == pass_atoms);
+        const uint64_t bd = sw128_desc(smem_u32(b_tile(s) + sub * b_atom));
+        const uint32_t at = a_base + static_cast<uint32_t>(slot) * kASlotCols;
 #pragma unroll
-        for (int at = 0; at < ATOMS; ++at)
+        for (int kk = 0; kk < kAtomK / 16; ++kk)  // hi: 8 columns (16 bf16 along K) per MMA
+          tc_mma_ts(acc, at + 8 * kk, bd + 2 * kk, p.idesc, (first && kk == 0) ? 0u : 1u);
 #pragma unroll
-          for (int kk = 0; kk < kChunkK / 16; ++kk)  // 16 bf16 = 32 bytes per MMA step
-            tc_mma_f16(tmem_base, ad + at * (kATileBytes >> 4) + 2 * kk, bd + at * (b_atom >> 4) + 2 * kk, p.idesc,
-                       (c > 0 || at > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&stage_free[s]);
-        if (++s == p.stages) { s = 0; ph ^= 1u; }
+        for (int kk = 0; kk < kAtomK / 16; ++kk)  // lo, same activations
+          tc_mma_ts(acc, at + 32 + 8 * kk, bd + 2 * kk, p.idesc, 1u);
+        tc_commit(&a_empty[slot]);
+        if (++slot == p.a_slots) { slot = 0; aph ^= 1u; }
+        if (++sub == ATOMS) {
+          sub = 0;
+          tc_commit(&stage_free[s]);
+          if (++s == p.stages) { s = 0; ph ^= 1u; }
+        }
       }
       tc_commit(accum_full);
     }
   } else {
     // ---------------- dequantize, then epilogue ----------------
-    const int t = tid - 64;
-    const int row = t & (kTileN - 1);  // weight row within the tile
-    const int half = t >> 7;           // which group of each 64-wide atom
+    const int quarter = warp & 3;  // the tensor-memory lanes this warp may access
+    const int half = ((warp - 2) >> 2) & 1;
+    const int grp = (warp - 2) >> 3;
+    const int row = 32 * quarter + lane;  // weight row within the tile
     const int64_t grow = n0 + row;
     const bool row_ok = grow < p.N;
     const int G = p.K / 32;
-    // Scales and biases of this row, 8 groups (one super-chunk) per 16-byte load,
-    // fetched one super-chunk ahead.
-    uint4 s_cur = make_uint4(0, 0, 0, 0), b_cur = s_cur, s_nxt = s_cur, b_nxt = s_cur;
-    auto load_sb = [&](int sc, uint4& sv, uint4& bv) {
-      if (row_ok && sc < sc_end) {
-        const int64_t off = grow * G + static_cast<int64_t>(sc) * (kSuperK / 32);
-        sv = *reinterpret_cast<const uint4*>(p.scales + off);
-        bv = *reinterpret_cast<const uint4*>(p.biases + off);
-      } else {
-        sv = make_uint4(0, 0, 0, 0);
-        bv = sv;
-      }
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
+    // Scales and biases of this row, 8 groups (one super-chunk) per 16-byte
+    // load, fetched one super-chunk ahead; u counts super-chunks over both
+    // passes of a SwiGLU tile.
+    auto load_sb = [&](int u, uint4& sv, uint4& bv) {
+      sv = bv = make_uint4(0, 0, 0, 0);
+      if (!row_ok || u >= pass_supers * p.nacc) return;
+      const bool up = u >= pass_supers;
+      const int64_t off = grow * G + static_cast<int64_t>(sc_begin + u - (up ? pass_supers : 0)) * (kSuperK / 32);
+      sv = *reinterpret_cast<const uint4*>((up ? p.up_scales : p.scales) + off);
+      bv = *reinterpret_cast<const uint4*>((up ? p.up_biases : p.biases) + off);
     };
-    load_sb(sc_begin, s_cur, b_cur);
-    load_sb(sc_begin + 1, s_nxt, b_nxt);
+    uint4 s_cur, b_cur, s_nxt, b_nxt;
+    load_sb(0, s_cur, b_cur);
+    load_sb(1, s_nxt, b_nxt);
     bool dead = false;
-    int s = 0, sub = 0, sc_next = sc_begin + 2;
-    uint32_t ph = 0;
-    for (int c = 0; c < nstages; ++c) {
-      if (c > 0 && sub == 0) {
+    int cur_u = 0;
+    for (int a = grp; a < natoms; a += kDqGroups) {
+      const int u = a / kAtomsPerSuper;
+      if (u != cur_u) {  // atoms advance by kDqGroups < kAtomsPerSuper: at most one super-chunk at a time
         s_cur = s_nxt;
         b_cur = b_nxt;
-        load_sb(sc_next++, s_nxt, b_nxt);
+        load_sb(u + 1, s_nxt, b_nxt);
+        cur_u = u;
       }
-      if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&stage_free[s], ph ^ 1u)) dead = true;  // A buffer no longer read
-      if (!dead && !mbar_wait<Q4_TC_WAIT_SLEEP>(&tma_full[s], ph)) dead = true;         // codes arrived
-      const uint8_t* crow = c_tile(s) + row * (32 * ATOMS);
-#pragma unroll
-      for (int at = 0; at < ATOMS; ++at) {
-        // group (2*(sub*ATOMS + at) + half) of the current super-chunk
-        const int gi = 2 * (sub * ATOMS + at) + half;
-        const uint32_t sw = (gi < 2) ? s_cur.x : (gi < 4) ? s_cur.y : (gi < 6) ? s_cur.z : s_cur.w;
-        const uint32_t bw = (gi < 2) ? b_cur.x : (gi < 4) ? b_cur.y : (gi < 6) ? b_cur.z : b_cur.w;
-        const uint32_t sel = (gi & 1) ? 0x3232u : 0x1010u;  // broadcast one bf16 to both halves
-        const uint32_t s2 = __byte_perm(sw, 0, sel);
-        const uint32_t b2 = __byte_perm(bw, 0, sel);
-        const uint4 cw = *reinterpret_cast<const uint4*>(crow + at * 32 + half * 16);
-        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-        uint8_t* arow = a_tile(s) + at * kATileBytes + row * 128;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const uint32_t wd = words[w], w4 = wd >> 4;
-          uint32_t o[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            // bytes: [wd.byte_i, -, w4.byte_i, -] -> nibbles q[2i] at bits 0..3, q[2i+1] at 16..19
-            const uint32_t pr = __byte_perm(wd, w4, (i) | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-            const uint32_t v = (pr & 0x000F000Fu) | 0x43004300u;  // (128 + q, 128 + q') exactly
-            const uint32_t q = bf16x2_sub(v, 0x43004300u);          // (q, q') exactly
-            o[i] = bf16x2_fma(q, s2, b2);                           // bf16(s*q + b), one rounding
-          }
-          const int chunk16 = 4 * half + w;  // 16-byte chunk (8 k) within the 128-byte row
-          *reinterpret_cast<uint4*>(arow + ((chunk16 ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      }
-      fence_proxy_async_smem();  // make the generic stores visible to the tensor core
+      const int st = (a / ATOMS) % p.stages;
+      const uint32_t ph = static_cast<uint32_t>((a / ATOMS) / p.stages) & 1u;
+      if (!dead && !mbar_wait(&tma_full[st], ph)) dead = true;  // codes arrived
+      const uint4 cw =
+          *reinterpret_cast<const uint4*>(c_tile(st) + row * (32 * ATOMS) + (a % ATOMS) * 32 + half * 16);
+      const int gi = 2 * (a % kAtomsPerSuper) + half;  // group within the super-chunk
+      const uint32_t sw = (gi < 2) ? s_cur.x : (gi < 4) ? s_cur.y : (gi < 6) ? s_cur.z : s_cur.w;
+      const uint32_t bw = (gi < 2) ? b_cur.x : (gi < 4) ? b_cur.y : (gi < 6) ? b_cur.z : b_cur.w;
+      const uint16_t sh = static_cast<uint16_t>((gi & 1) ? (sw >> 16) : (sw & 0xFFFFu));
+      const float bf = __uint_as_float((gi & 1) ? (bw & 0xFFFF0000u) : (bw << 16));
+      const int slot = a % p.a_slots;
+      const uint32_t sph = static_cast<uint32_t>(a / p.a_slots) & 1u;
+      if (!dead && !mbar_wait(&a_empty[slot], sph ^ 1u)) dead = true;  // the MMAs of the slot's last atom are done
+      tc_fence_after();
+      const uint32_t taddr = lane_addr + p.a_col0 + static_cast<uint32_t>(slot) * kASlotCols + 16u * half;
+      uint32_t hi[8], lo[8];  // 16 codes at a time: 8 hi and 8 lo columns
+      dequant_words(cw.x, cw.y, sh, bf, hi, lo);
+      tmem_st_x8(taddr, hi);
+      tmem_st_x8(taddr + 32u, lo);
+      dequant_words(cw.z, cw.w, sh, bf, hi, lo);
+      tmem_st_x8(taddr + 8u, hi);
+      tmem_st_x8(taddr + 40u, lo);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[s]);
-      if (++s == p.stages) { s = 0; ph ^= 1u; }
-      if (++sub == kStagesPerSuper) sub = 0;
+      if (lane == 0) mbar_arrive(&a_full[slot]);
     }
 
     // ---- epilogue: tensor memory -> y (or partial sums for the cluster) ----
     if (!dead && !mbar_wait(accum_full, 0)) dead = true;
     tc_fence_after();
-    const int lane_base = 32 * (warp & 3);
-    const int trow = lane_base + lane;  // tile row held by this thread
-    const int col_half = (warp - 2) >> 2;
-    const int cols = p.bn / 2;
-    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lane_base) << 16) + col_half * cols;
+    const int part = (warp - 2) >> 2;  // 0..3: which column octets this warp reads
     float* red = reinterpret_cast<float*>(smem);  // reuses the stage area (all MMAs are done)
-    const int red_ld = p.bn + 4;                  // 16-byte rows; row r and r + 1 four banks apart
-    for (int c0 = 0; c0 < cols; c0 += 8) {
-      float v[8];
-      tc_ld_x8(taddr + c0, v);
+    const int red_ld = p.nacc * p.bn + 4;          // 16-byte rows; row r and r + 1 four banks apart
+    for (int c0 = 8 * part; c0 < p.bn; c0 += 32) {
+      uint32_t gr[8], ur[8];
+      tmem_ld_cols<8>(lane_addr + c0, gr);
+      if (p.nacc == 2) tmem_ld_cols<8>(lane_addr + p.bn + c0, ur);
+      tmem_wait_ld();
+      float g[8], u[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        g[i] = dead ? kNaN : __uint_as_float(gr[i]);
+        u[i] = (p.nacc == 2) ? (dead ? kNaN : __uint_as_float(ur[i])) : 0.f;
+      }
       if (p.splits == 1) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int64_t m = m0 + col_half * cols + c0 + i;
-          if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = store_tc<EPI>(v[i], p, m * p.N + n0 + trow);
+          const int64_t m = m0 + c0 + i;
+          if (row_ok && m < p.M) p.y[m * p.N + grow] = out_tc<EPI>(g[i], u[i], p, m * p.N + grow);
         }
       } else {
-        float4* dst = reinterpret_cast<float4*>(red + trow * red_ld + col_half * cols + c0);
-        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+        float4* dst = reinterpret_cast<float4*>(red + row * red_ld + c0);
+        dst[0] = make_float4(g[0], g[1], g[2], g[3]);
+        dst[1] = make_float4(g[4], g[5], g[6], g[7]);
+        if (p.nacc == 2) {
+          float4* du = reinterpret_cast<float4*>(red + row * red_ld + p.bn + c0);
+          du[0] = make_float4(u[0], u[1], u[2], u[3]);
+          du[1] = make_float4(u[4], u[5], u[6], u[7]);
+        }
       }
     }
   }
@@ -349,32 +328,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp >= 2) {
       const int t = tid - 64;
       const int trow = t & (kTileN - 1);
+      const int64_t grow = n0 + trow;
+      const int red_ld = p.nacc * p.bn + 4;
       // Column slice of this CTA, in float4 units (bn and the slice are multiples of 4).
       const int q_beg = split * (p.bn / 4) / p.splits, q_end = (split + 1) * (p.bn / 4) / p.splits;
-      const uint32_t row_addr = smem_u32(smem) + static_cast<uint32_t>(trow * (p.bn + 4)) * 4u;
+      const uint32_t row_addr = smem_u32(smem) + static_cast<uint32_t>(trow * red_ld) * 4u;
       uint32_t peer[8];
 #pragma unroll
       for (int r = 0; r < 8; ++r) peer[r] = dsmem_map(row_addr, static_cast<uint32_t>(r < p.splits ? r : 0));
-      for (int q = q_beg + (t >> 7); q < q_end; q += 2) {
-        // all peers' loads first, then the sums
-        float4 v[8];
+      for (int q = q_beg + (t >> 7); q < q_end; q += kDqWarps * 32 / kTileN) {
+        float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
-          if (r < p.splits) v[r] = ld_dsmem_v4(peer[r] + static_cast<uint32_t>(q) * 16u);
-        float4 acc = v[0];
+        for (int w = 0; w < 2; ++w) {  // the gate's (or only) partial tiles, then the up weight's
+          if (w >= p.nacc) break;
+          float4 v[8];
 #pragma unroll
-        for (int r = 1; r < 8; ++r)
-          if (r < p.splits) {
-            acc.x += v[r].x;
-            acc.y += v[r].y;
-            acc.z += v[r].z;
-            acc.w += v[r].w;
-          }
-        const float out[4] = {acc.x, acc.y, acc.z, acc.w};
+          for (int r = 0; r < 8; ++r)  // all peers' loads first, then the sums
+            if (r < p.splits)
+              v[r] = ld_dsmem_v4(peer[r] + static_cast<uint32_t>(w * p.bn) * 4u + static_cast<uint32_t>(q) * 16u);
+          float4 t = v[0];
+#pragma unroll
+          for (int r = 1; r < 8; ++r)
+            if (r < p.splits) {
+              t.x += v[r].x;
+              t.y += v[r].y;
+              t.z += v[r].z;
+              t.w += v[r].w;
+            }
+          acc[w] = t;
+        }
+        const float4 ag = acc[0], au = acc[1];
+        const float og[4] = {ag.x, ag.y, ag.z, ag.w}, ou[4] = {au.x, au.y, au.z, au.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int64_t m = m0 + 4 * q + i;
-          if (n0 + trow < p.N && m < p.M) p.y[m * p.N + n0 + trow] = store_tc<EPI>(out[i], p, m * p.N + n0 + trow);
+          if (grow < p.N && m < p.M) p.y[m * p.N + grow] = out_tc<EPI>(og[i], ou[i], p, m * p.N + grow);
         }
       }
     }
@@ -385,8 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(p.tmem_cols)
-                 : "memory");
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -405,32 +392,44 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-uint32_t make_idesc(int bn) {
-  uint32_t d = 0;
-  d |= 1u << 4;                                  // D: fp32
-  d |= 1u << 7;                                  // A: bf16
-  d |= 1u << 10;                                 // B: bf16
-  d |= static_cast<uint32_t>(bn >> 3) << 17;     // N
-  d |= static_cast<uint32_t>(kTileN >> 4) << 24;  // M
-  return d;                                      // both operands K-major, no negation
+constexpr size_t kBarrierBytes = 8 * (2 * kMaxStages + 2 * kMaxASlots + 1) + 16;
+
+template <int ATOMS, bool EPI>
+void* kernel_of() {
+  return reinterpret_cast<void*>(tc_kernel<ATOMS, EPI>);
 }
 
 }  // namespace
 
 cudaError_t tc_device_flags(unsigned int* flags, bool clear) { return tu_device_flags(flags, clear); }
 
+cudaError_t tc_prepare_device(const DeviceInfo& dev) {
+  for (void* kern : {kernel_of<1, false>(), kernel_of<2, false>(), kernel_of<1, true>(), kernel_of<2, true>()}) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dev.smem_optin));
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 bool tc_supported(const MatmulArgs& a) {
-  if (a.fused()) return false;  // one-pass SwiGLU is a GEMV-family problem
   if (a.K % kSuperK != 0) return false;
-  if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) return false;
+  uintptr_t sb = reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases);
+  if (a.fused()) sb |= reinterpret_cast<uintptr_t>(a.up_scales) | reinterpret_cast<uintptr_t>(a.up_biases);
+  if (sb & 15u) return false;
   if (a.N > (int64_t(1) << 31) - kTileN || a.M > (int64_t(1) << 31) - 256) return false;
   return encode_fn() != nullptr;
 }
 
-cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev) {
+
+cudaError_t plan_tc(const MatmulArgs& a, const DeviceInfo& dev, TcLaunch* out) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
-  const int bn = static_cast<int>(std::min<int64_t>(256, (a.M + 15) / 16 * 16));
+  const bool swiglu = a.fused();
+  const int nacc = swiglu ? 2 : 1;
+  const int bn_max = swiglu ? 128 : 256;  // the accumulators and a 4-slot A ring share 512 columns
+  const int bn = static_cast<int>(std::min<int64_t>(bn_max, (a.M + 15) / 16 * 16));
   const int64_t n_tiles = (a.N + kTileN - 1) / kTileN;
   const int64_t m_tiles = (a.M + bn - 1) / bn;
   const int supers = static_cast<int>(a.K / kSuperK);
@@ -443,40 +442,43 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
     if (want > splits && want <= supers && tiles * want <= dev.sm_count * 1.05) splits = want;
   }
 
-  // Two 64-wide atoms per stage when at least three such stages fit.
-  const uint32_t b_atom = static_cast<uint32_t>(bn) * kChunkK * 2;
+  // Two atoms per stage when at least three such stages fit.
+  const uint32_t b_atom = static_cast<uint32_t>(bn) * kAtomK * 2;
   auto stage_size = [&](int atoms) {
-    return (static_cast<uint32_t>(atoms) * (kATileBytes + b_atom + kCodeTileBytes) + 1023u) & ~1023u;
+    return (static_cast<uint32_t>(atoms) * (b_atom + kCodeAtomBytes) + 1023u) & ~1023u;
   };
-  const size_t barrier_bytes = 8 * (3 * 12 + 1) + 16;
-  const size_t avail = dev.smem_optin - 1024 - barrier_bytes;
+  const size_t avail = dev.smem_optin - 1024 - kBarrierBytes;
   const int atoms = (avail / stage_size(2) >= 3) ? 2 : 1;
 
-  CUtensorMap tmap_x, tmap_codes;
+  TcLaunch& L = *out;
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunkK), static_cast<cuuint32_t>(bn)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kAtomK), static_cast<cuuint32_t>(bn)};
     cuuint32_t estr[2] = {1, 1};
-    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box, estr,
+    if (encode(&L.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  {
+  for (int w = 0; w < nacc; ++w) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 2), static_cast<cuuint64_t>(a.N)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 2)};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunkK / 2 * atoms), static_cast<cuuint32_t>(kTileN)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kAtomK / 2 * atoms), static_cast<cuuint32_t>(kTileN)};
     cuuint32_t estr[2] = {1, 1};
-    if (encode(&tmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.codes), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    const uint8_t* codes = w == 0 ? a.codes : a.up_codes;
+    if (encode(w == 0 ? &L.tmap_codes : &L.tmap_up, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes),
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  if (!swiglu) L.tmap_up = L.tmap_codes;
 
-  TcParams p;
+  TcParams& p = L.p;
   p.scales = a.scales;
   p.biases = a.biases;
+  p.up_scales = swiglu ? a.up_scales : nullptr;
+  p.up_biases = swiglu ? a.up_biases : nullptr;
   p.y = a.y;
   p.r = a.r;
   p.epi = a.epi;
@@ -484,51 +486,52 @@ cudaError_t launch_tc(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo
   p.N = a.N;
   p.K = static_cast<int>(a.K);
   p.bn = bn;
+  p.nacc = nacc;
   p.splits = splits;
-  p.b_tile_bytes = b_atom;
+  p.b_atom_bytes = b_atom;
   p.stage_bytes = stage_size(atoms);
-  const size_t red_bytes = static_cast<size_t>(kTileN) * (bn + 4) * 4;
-  p.stages = static_cast<int>(std::min<size_t>(12, avail / p.stage_bytes));
-  while (p.stages > 2 && static_cast<size_t>(p.stages) * p.stage_bytes < red_bytes) ++p.stages;
+  const size_t red_bytes = static_cast<size_t>(kTileN) * (nacc * bn + 4) * 4;
+  p.stages = static_cast<int>(std::min<size_t>(kMaxStages, avail / p.stage_bytes));
+  while (p.stages < kMaxStages && static_cast<size_t>(p.stages) * p.stage_bytes < red_bytes) ++p.stages;
   if (p.stages < 2 || static_cast<size_t>(p.stages) * p.stage_bytes < red_bytes ||
       static_cast<size_t>(p.stages) * p.stage_bytes > avail)
     return cudaErrorInvalidConfiguration;
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(bn)) cols <<= 1;
-  p.tmem_cols = cols;
-  p.idesc = make_idesc(bn);
-  const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + barrier_bytes + 1024;
+  p.a_col0 = static_cast<uint32_t>((nacc * bn + kASlotCols - 1) / kASlotCols * kASlotCols);
+  p.a_slots = static_cast<int>(std::min<uint32_t>(kMaxASlots, (kTmemCols - p.a_col0) / kASlotCols));
+  if (p.a_slots < 2) return cudaErrorInvalidConfiguration;
+  p.idesc = idesc_bf16_m128(bn);
+  // All of the SM's shared memory, whatever the stages use: one CTA per SM,
+  // so no two CTAs ever wait for each other's tensor memory (each allocates
+  // all 512 columns; two clusters interleaved on the same SMs could deadlock).
+  L.smem = dev.smem_optin;
+  if (static_cast<size_t>(p.stages) * p.stage_bytes + kBarrierBytes + 1024 > L.smem) return cudaErrorInvalidConfiguration;
+  L.grid = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(n_tiles), static_cast<unsigned>(m_tiles));
+  L.atoms = atoms;
+  return cudaSuccess;
+}
 
-  static PerDeviceOnce attr_once;
-  if (attr_once.needed(dev.device)) {
-    for (auto kern : {tc_kernel<1, false>, tc_kernel<2, false>, tc_kernel<1, true>, tc_kernel<2, true>}) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(dev.smem_optin));
-      if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-      if (e != cudaSuccess) return e;
-    }
-    attr_once.mark(dev.device);
-  }
+cudaError_t launch_planned_tc(const TcLaunch& L, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(n_tiles), static_cast<unsigned>(m_tiles));
+  cfg.gridDim = L.grid;
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = static_cast<unsigned>(splits);
+  attr[1].val.clusterDim.x = L.grid.x;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   count_launch();
-  if (p.epi != kEpiNone)
-    return atoms == 2 ? cudaLaunchKernelEx(&cfg, tc_kernel<2, true>, tmap_x, tmap_codes, p)
-                      : cudaLaunchKernelEx(&cfg, tc_kernel<1, true>, tmap_x, tmap_codes, p);
-  return atoms == 2 ? cudaLaunchKernelEx(&cfg, tc_kernel<2, false>, tmap_x, tmap_codes, p)
-                    : cudaLaunchKernelEx(&cfg, tc_kernel<1, false>, tmap_x, tmap_codes, p);
+  const bool epi = L.p.epi != kEpiNone || L.p.nacc == 2;
+  if (epi)
+    return L.atoms == 2 ? cudaLaunchKernelEx(&cfg, tc_kernel<2, true>, L.tmap_x, L.tmap_codes, L.tmap_up, L.p)
+                        : cudaLaunchKernelEx(&cfg, tc_kernel<1, true>, L.tmap_x, L.tmap_codes, L.tmap_up, L.p);
+  return L.atoms == 2 ? cudaLaunchKernelEx(&cfg, tc_kernel<2, false>, L.tmap_x, L.tmap_codes, L.tmap_up, L.p)
+                      : cudaLaunchKernelEx(&cfg, tc_kernel<1, false>, L.tmap_x, L.tmap_codes, L.tmap_up, L.p);
 }
 
 }  // namespace q4

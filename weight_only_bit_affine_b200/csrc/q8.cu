@@ -214,6 +214,9 @@ cudaError_t run_q8_gemv(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, 
 
 }  // namespace
 
+// The 8-bit kernels need no per-device settings (at most 48 KB of shared memory).
+cudaError_t q8_prepare_device(const DeviceInfo&) { return cudaSuccess; }
+
 cudaError_t launch_q8_quantize(const uint16_t* W, int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
                                uint16_t* biases, cudaStream_t stream, const DeviceInfo& dev) {
   const int64_t groups = N * (K / 32);

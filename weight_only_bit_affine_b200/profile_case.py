@@ -162,7 +162,7 @@ def main(argv=None):
     for _ in range(1 + reps):
         run()
     torch.cuda.synchronize(dev)
-    if q4.q4_debug_device_flags() != 0:
+    if q4.q4_device_status() != 0:
         raise SystemExit("a bounded wait gave up inside a kernel")
     print(f"{argv[0]}: {reps} reps ok")
 
