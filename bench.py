@@ -244,6 +244,12 @@ def _graph_ms(dev, fn, reps):
     return ms
 
 
+# Rows of the batched-layer workload (M in {4, 64, 256}), with the row counts
+# in between where the kernel choice changes (weight streaming up to 8 rows,
+# tensor-core tiles from 9, one 16-row tile up to 16).
+BATCHED_ROWS = (4, 8, 12, 16, 64, 256)
+
+
 def workload_rows(dev, packed, x, x_down, bf16_peak):
     """The other workloads, as informational rows (not the metric).
 
@@ -317,6 +323,39 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
                 "(silu(gate) * up in the GEMV epilogue); compare temporal_layer_M1, the 7 plain projections",
     }
 
+    # A decode-shaped step over the same 4.19 GB: the projections in the order a
+    # model runs them, each launch reading what the one before wrote.  Per
+    # layer: q, k, v as one batch on the layer input h; o adding into h (v's
+    # output standing in for the attention output, which is not on this path);
+    # gate and up as one SwiGLU problem on h; down adding into h, the next
+    # layer's input; then the text head.  32 * 4 + 1 launches in one CUDA graph
+    # (programmatic dependent launch between them).
+    h = x.clone()
+    qkv = [torch.empty((1, 4096), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    act = torch.empty((1, 11264), dtype=torch.bfloat16, device=dev)
+    logits = torch.empty((1, packed[-1][0].N), dtype=torch.bfloat16, device=dev)
+    layers_w = [{p.name.split(".")[1]: (c, s, b) for p, c, s, b in packed[7 * l:7 * l + 7]} for l in range(32)]
+
+    def chain():
+        for P in layers_w:
+            q4.q4_matmul_batch([(h, *P["q"], qkv[0]), (h, *P["k"], qkv[1]), (h, *P["v"], qkv[2])])
+            q4.q4_matmul_residual(qkv[2], *P["o"], h, out=h)
+            q4.q4_matmul_swiglu(h, P["gate"], P["up"], out=act)
+            q4.q4_matmul_residual(act, *P["down"], h, out=h)
+        q4.q4_matmul(h, *packed[-1][1:], out=logits)
+
+    n0 = q4.q4_debug_launch_count()
+    chain()
+    chain_launches = q4.q4_debug_launch_count() - n0
+    ms_chain = _graph_ms(dev, chain, 20)
+    rows["decode_chain_M1"] = {
+        "ms_per_step": round(ms_chain, 4), "GBps": round(STREAM_BYTES / (ms_chain * 1e-3) / 1e9, 1),
+        "launches_per_step": int(chain_launches), "bytes": STREAM_BYTES,
+        "note": "dependent launches per layer: q/k/v batch -> o + residual -> SwiGLU(gate, up) -> down + residual; "
+                "32 layers + head in one CUDA graph; compare stream_ms_batch_graph (one launch over independent "
+                "problems with x reused)",
+    }
+
     # the 8-bit variant of the same layer (9 bits per weight), one q8_matmul per
     # projection, four layers rotated (925 MB > L2)
     seed8 = workloads.seed_of("batched_layer")
@@ -385,14 +424,14 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
     rows["depformer_steps_M4"] = {
         "batched_us_per_step": round(ms_m4 * 1e3 / steps, 2), "batched_ms_per_frame": round(ms_m4, 4),
         "packed_GBps": round(fbytes / (ms_m4 * 1e-3) / 1e9, 1),
-        "path": "stream_kernel: tcgen05, dequantized weights in tensor memory",
+        "path": "stream_kernel: tcgen05 weight streaming, dequantized hi/lo operand in tensor memory",
         "note": "four conversations' rows per step slice, one q4_matmul_batch launch per codebook step",
     }
     del dep
 
     # batched layer for concurrent conversations / prefill
     flops_layer = 2 * sum(p.N * p.K for p, _, _, _ in layer[0])
-    for M in workloads.BATCHED_M:
+    for M in BATCHED_ROWS:
         xb = workloads.activation(M, 4096, seed, 100 + M, device=dev)
         xbd = workloads.activation(M, 11264, seed, 200 + M, device=dev)
         ysm = [y_for(M, l) for l in layer]
@@ -406,9 +445,9 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
         rows[f"batched_layer_M{M}"] = {
             "us_per_layer": round(t * 1e3, 2), "TFLOPs": round(tf, 1),
             "frac_of_bf16_peak": round(tf / bf16_peak, 4), "packed_GBps": round(lbytes / (t * 1e-3) / 1e9, 1),
-            "path": ("tc_kernel: tcgen05, dequantized tile in shared memory" if M >= 16 else
-                     "stream_kernel: tcgen05, dequantized weights in tensor memory" if M >= 3 else
-                     "gemv_kernel: CUDA cores"),
+            "path": ("tc_kernel: tcgen05 tiles, dequantized hi/lo operand in tensor memory" if M > 8 else
+                     "stream_kernel: tcgen05 weight streaming, dequantized hi/lo operand in tensor memory"
+                     if M >= 3 else "gemv_kernel: CUDA cores"),
         }
     return rows
 
@@ -478,6 +517,179 @@ class OracleSample:
         finally:
             oracle.set_threads(self.threads)
         return nbytes / spent / 1e9, n, spent
+
+
+# --------------------------------------------------------------------- profiling cases
+#
+# Small, named workloads for ncu captures: `python bench.py --profile-case
+# <case> [--reps R]` builds the case (seeded synthetic inputs of the workload
+# shapes), runs it once to warm up and then R times, checks the kernels'
+# status flag and exits.  Nothing is timed or printed as a bench line.
+#
+#   stream_small   3 temporal layers + the text head (553 MB packed) as one
+#                  q4_matmul_batch per rep: the benchmark's kernel on a case
+#                  small enough for a full ncu capture.
+#   tc_layer       one temporal layer (7 projections, 128 MB) through q4_matmul
+#                  at M = 64 and then M = 256: the tensor-core tile kernel.
+#   tc_gate        the gate projection (11264 x 4096) alone at M = 64, then 256.
+#   depformer_step one depformer codebook step (43 step-sliced projections) as
+#                  one q4_matmul_batch.
+#   layer_m4       one temporal layer (7 projections) at M = 4 as one
+#                  q4_matmul_batch: the tensor-core weight-streaming kernel.
+#   layer_m8       the same at M = 8.
+#   fused_layer    one temporal layer at M = 1 with its epilogues fused (o and
+#                  down + residual, gate/up as one SwiGLU problem), one
+#                  q4_matmul_batch: the GEMV's epilogue instantiation.
+#   q8_layer       one temporal layer with 8-bit codes at M = 1, one q8_matmul
+#                  per projection: the 8-bit GEMV.
+
+
+def _stream_small(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    projs = workloads.stream_projs()
+    sel = [(t, p) for t, p in enumerate(projs) if p.name.startswith(("L0.", "L1.", "L2."))] + [(len(projs) - 1, projs[-1])]
+    seed = workloads.seed_of("temporal_stream")
+    x = workloads.activation(1, 4096, seed, 10000, device=dev)
+    xd = workloads.activation(1, 11264, seed, 10001, device=dev)
+    probs = []
+    for t, p in sel:
+        c, s, b = q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+        probs.append((xd if p.K == 11264 else x, c, s, b, torch.empty((1, p.N), dtype=torch.bfloat16, device=dev)))
+    return lambda: q4.q4_matmul_batch(probs)
+
+
+def _tc_layer(dev):
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    packed = [(p,) + tuple(q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev)))
+              for t, p in enumerate(workloads.TEMPORAL_LAYER)]
+    xs = {M: (workloads.activation(M, 4096, seed, 100 + M, device=dev),
+              workloads.activation(M, 11264, seed, 200 + M, device=dev)) for M in (64, 256)}
+
+    def run():
+        for M in (64, 256):
+            for p, c, s, b in packed:
+                q4.q4_matmul(xs[M][1] if p.K == 11264 else xs[M][0], c, s, b)
+
+    return run
+
+
+def _depformer_step(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("depformer_steps")
+    steps = workloads.DEPFORMER_STEPS
+    xs = {K: workloads.activation(1, K, seed, 500 + K, device=dev) for K in (1024, 2816)}
+    probs = []
+    for t, p in enumerate(workloads.depformer_projs()):
+        c, s, b = q4.q4_quantize(workloads.weight(steps * p.N, p.K, seed, t, device=dev))
+        probs.append((xs[p.K], c[:p.N], s[:p.N], b[:p.N], torch.empty((1, p.N), dtype=torch.bfloat16, device=dev)))
+    return lambda: q4.q4_matmul_batch(probs)
+
+
+def _layer_rows(dev, M):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    x = workloads.activation(M, 4096, seed, 100 + M, device=dev)
+    xd = workloads.activation(M, 11264, seed, 200 + M, device=dev)
+    probs = []
+    for t, p in enumerate(workloads.TEMPORAL_LAYER):
+        c, s, b = q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+        probs.append((xd if p.K == 11264 else x, c, s, b, torch.empty((M, p.N), dtype=torch.bfloat16, device=dev)))
+    return lambda: q4.q4_matmul_batch(probs)
+
+
+def _fused_layer(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    x = workloads.activation(1, 4096, seed, 101, device=dev)
+    xd = workloads.activation(1, 11264, seed, 201, device=dev)
+    w = {p.name: q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+         for t, p in enumerate(workloads.TEMPORAL_LAYER)}
+    out = lambda n: torch.empty((1, n), dtype=torch.bfloat16, device=dev)
+    r_o = torch.zeros((1, 4096), dtype=torch.bfloat16, device=dev)  # two residual streams: problems of
+    r_d = torch.zeros((1, 4096), dtype=torch.bfloat16, device=dev)  # one launch may not share an output
+    probs = [(x, *w[n], out(4096)) for n in ("q", "k", "v")]
+    probs += [(x, *w["o"], r_o, q4.Residual(r_o)), (x, *w["gate"], out(11264), q4.SwiGLU(*w["up"])),
+              (xd, *w["down"], r_d, q4.Residual(r_d))]
+    return lambda: q4.q4_matmul_batch(probs)
+
+
+def _q8_layer(dev):
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    x = workloads.activation(1, 4096, seed, 101, device=dev)
+    xd = workloads.activation(1, 11264, seed, 201, device=dev)
+    items = []
+    for t, p in enumerate(workloads.TEMPORAL_LAYER):
+        c, s, b = q4.q8_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+        items.append((xd if p.K == 11264 else x, c, s, b, torch.empty((1, p.N), dtype=torch.bfloat16, device=dev)))
+
+    def run():
+        for xx, c, s, b, y in items:
+            q4.q8_matmul(xx, c, s, b, out=y)
+
+    return run
+
+
+def _tc_gate(dev):
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    seed = workloads.seed_of("batched_layer")
+    p = workloads.TEMPORAL_LAYER[4]
+    c, s, b = q4.q4_quantize(workloads.weight(p.N, p.K, seed, 4, device=dev))
+    xs = [workloads.activation(M, p.K, seed, 100 + M, device=dev) for M in (64, 256)]
+
+    def run():
+        for x in xs:
+            q4.q4_matmul(x, c, s, b)
+
+    return run
+
+
+PROFILE_CASES = {"stream_small": _stream_small, "tc_layer": _tc_layer, "tc_gate": _tc_gate,
+                 "depformer_step": _depformer_step, "layer_m4": lambda dev: _layer_rows(dev, 4),
+                 "layer_m8": lambda dev: _layer_rows(dev, 8), "fused_layer": _fused_layer, "q8_layer": _q8_layer}
+
+
+def run_profile_case(name: str, reps: int):
+    import torch
+
+    import weight_only_bit_affine_b200 as q4
+    from weight_only_bit_affine_b200 import build as q4build
+
+    q4build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    run = PROFILE_CASES[name](dev)
+    torch.cuda.synchronize(dev)
+    for _ in range(1 + reps):
+        run()
+    torch.cuda.synchronize(dev)
+    q4.q4_check_device()
+    print(f"{name}: {reps} reps ok", flush=True)
 
 
 # --------------------------------------------------------------------- arms
@@ -626,30 +838,46 @@ def run_ours(args):
     shapes = {k: {"launches": v[2], "us_per_launch": round(v[1] / v[2] * 1e3, 2),
                   "GBps": round(v[0] / (v[1] * 1e-3) / 1e9, 1)} for k, v in by_shape.items()}
 
-    # end to end through the public API: pinned x H2D, the step, y D2H
+    # end to end through the public API: pinned x H2D, the step, y D2H.  The
+    # step is the C entry point q4_matmul_batch called directly every step
+    # (its descriptor array marshalled once, as for any fixed weight stream):
+    # host validation and the launch are inside the timed region.  The same
+    # with the call replayed from a CUDA graph is reported beside it.
     x_host = x.cpu().pin_memory()
     xd_host = x_down.cpu().pin_memory()
     y_host = torch.empty(y_all.numel(), dtype=torch.bfloat16).pin_memory()
     h2d = (x_host.numel() + xd_host.numel()) * 2
     d2h = y_all.numel() * 2
     e2e_steps = max(3, min(args.steps, 200))
+    prepared = q4.q4_prepare_batch(
+        [(x_down if p.K == 11264 else x, c, s, b, y) for (p, c, s, b), y in zip(packed, ys)])
 
-    def e2e_step():
+    def e2e_call():
+        x.copy_(x_host, non_blocking=True)
+        x_down.copy_(xd_host, non_blocking=True)
+        prepared.run()
+        y_host.copy_(y_all, non_blocking=True)
+
+    def e2e_graph():
         x.copy_(x_host, non_blocking=True)
         x_down.copy_(xd_host, non_blocking=True)
         graph.replay()
         y_host.copy_(y_all, non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    t_wall0 = time.perf_counter()
-    ev0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms_e2e = max(ev0.elapsed_time(ev1), (time.perf_counter() - t_wall0) * 1e3) / e2e_steps
+    def time_e2e(step):
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize(dev)
+        t_wall0 = time.perf_counter()
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        return max(ev0.elapsed_time(ev1), (time.perf_counter() - t_wall0) * 1e3) / e2e_steps
+
+    ms_e2e = time_e2e(e2e_call)
+    ms_e2e_graph = time_e2e(e2e_graph)
 
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], device=dev)
 
@@ -695,7 +923,9 @@ def run_ours(args):
         },
         "e2e": {"value": round(job_gbps(world, nbytes, ms_e2e), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "how": "pinned x H2D + graph replay of the public q4_matmul_batch call + y D2H, per step"},
+                "how": "per step: pinned x H2D, one direct call of the C entry point q4_matmul_batch "
+                       "(descriptors marshalled once), y D2H",
+                "graph_replay_GBps": round(job_gbps(world, nbytes, ms_e2e_graph), 2)},
         "gpu_launches": int(launches_per_step) * args.steps,
         "clocks": clocks,
         "rows": {
@@ -733,7 +963,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip the informational rows of the other workloads")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run a named profiling case (for ncu) instead of the benchmark")
+    ap.add_argument("--reps", type=int, default=3, help="repetitions of --profile-case after one warm-up")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case, args.reps)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

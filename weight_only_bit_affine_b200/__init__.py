@@ -15,6 +15,7 @@ come from PyTorch) and have the same names as the C entry points:
     y = q4_matmul_residual(x, codes, scales, biases, r)   # r + x . w_hat^T
     h = q4_matmul_swiglu(x, (gc, gs, gb), (uc, us, ub))   # silu(gate) * up
     q4_matmul_batch([(x, codes, scales, biases, y), ...]) # one launch per kernel path
+    b = q4_prepare_batch([...]); b.run()                  # the same, descriptors built once
     codes8, scales, biases = q8_quantize(W)             # 8-bit variant: codes [N, K]
     y = q8_matmul(x, codes8, scales, biases)
 
@@ -42,6 +43,8 @@ __all__ = [
     "q4_matmul_residual",
     "q4_matmul_swiglu",
     "q4_matmul_batch",
+    "q4_prepare_batch",
+    "PreparedBatch",
     "Residual",
     "SwiGLU",
     "q8_quantize",
@@ -191,12 +194,9 @@ def q4_dequantize(codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tenso
     _want(biases, "biases", torch.bfloat16, 2)
     N, K = codes.shape[0], codes.shape[1] * 2
     dev = codes.device
-    if out is None:
-        out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
-    else:
-        _want(out, "out", torch.bfloat16, 2)
-    if scales.shape != (N, K // GROUP) or biases.shape != (N, K // GROUP) or out.shape != (N, K):
-        raise ValueError("codes / scales / biases / out shapes disagree")
+    if scales.shape != (N, K // GROUP) or biases.shape != (N, K // GROUP):
+        raise ValueError("codes / scales / biases shapes disagree")
+    out = _out(out, N, K, dev)
     with torch.cuda.device(dev):
         _check(lib().q4_dequantize(_ptr(codes), _ptr(scales), _ptr(biases), N, K, group, _ptr(out), _stream(dev)))
     return out
@@ -312,9 +312,38 @@ def q4_matmul_batch(problems, group: int = GROUP):
     element Residual(r) or SwiGLU(up_codes, up_scales, up_biases) adds that
     epilogue.  Returns the list of outputs.
     """
+    batch = q4_prepare_batch(problems, group)
+    if batch is None:
+        return []
+    batch.run()
+    return batch.outputs
+
+
+class PreparedBatch:
+    """A q4_matmul_batch call whose descriptor array is built once.
+
+    run() calls the C entry point with it on the current stream of the
+    problems' device (host-side validation and the launches happen on every
+    call); the tensors must stay alive and keep their storage in between, as
+    for a CUDA graph.
+    """
+
+    def __init__(self, descs, count, M, group, device, outputs):
+        self._descs, self._count, self._M, self._group = descs, count, M, group
+        self.device, self.outputs = device, outputs
+
+    def run(self) -> None:
+        with torch.cuda.device(self.device):
+            _check(lib().q4_matmul_batch(ctypes.cast(self._descs, ctypes.c_void_p), self._count, self._M, self._group,
+                                         _stream(self.device)))
+
+
+def q4_prepare_batch(problems, group: int = GROUP) -> Optional[PreparedBatch]:
+    """Validate and marshal a q4_matmul_batch problem list once (same tuples
+    as q4_matmul_batch); None for an empty list."""
     problems = list(problems)
     if not problems:
-        return []
+        return None
     descs = (MatmulDesc * len(problems))()
     M = None
     dev = None
@@ -346,9 +375,7 @@ def q4_matmul_batch(problems, group: int = GROUP):
         elif epi is not None:
             raise TypeError(f"problem {i}: epilogue must be Residual or SwiGLU")
         descs[i] = d
-    with torch.cuda.device(dev):
-        _check(lib().q4_matmul_batch(ctypes.cast(descs, ctypes.c_void_p), len(problems), M, group, _stream(dev)))
-    return [p[4] for p in problems]
+    return PreparedBatch(descs, len(problems), M, group, dev, [p[4] for p in problems])
 
 
 # ------------------------------------------------------------------ 8-bit codes

@@ -346,6 +346,9 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   uint64_t* empty_bar = full_bar + L.stages;
   uint64_t* rfull_bar = empty_bar + L.stages;   // [kRedSlots]
   uint64_t* rempty_bar = rfull_bar + kRedSlots;  // [kRedSlots]
+  // Set by any thread whose bounded wait gave up: the epilogue warp then
+  // writes NaN for the partial sums it cannot vouch for.
+  volatile uint32_t* gave_up = reinterpret_cast<volatile uint32_t*>(rempty_bar + kRedSlots);
 
   if (tid == 0) {
     for (int s = 0; s < L.stages; ++s) {
@@ -356,6 +359,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       mbar_init(&rfull_bar[s], consumer_warps);
       mbar_init(&rempty_bar[s], 1);
     }
+    *gave_up = 0u;
     fence_mbar_init();
   }
   __syncthreads();
@@ -404,7 +408,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         const int half_k = P.K >> 1;
         const int rtile = rtile_k<EPI>(P, geo);
         for (int64_t row0 = r0 - rtile; row0 < r1; row0 += rtile) {  // first pass: x
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; break; }
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; *gave_up = 1u; break; }
           uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
           if (row0 < r0) {
             const uint32_t xbytes = static_cast<uint32_t>(MR) * P.K * 2;
@@ -461,14 +465,14 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       const int rtile = rtile_k<EPI>(P, geo);
       const bool fused = fused_k<EPI>(P);
       for (int64_t row0 = r0; row0 < r1; row0 += rtile) {
-        if (!dead && !mbar_wait(&rfull_bar[slot], sph)) dead = true;
+        if (!dead && !mbar_wait(&rfull_bar[slot], sph)) { dead = true; *gave_up = 1u; }
         // Slot entry ((row * MR + m) * wpt + warp) holds one warp's partial
         // sum of the tile's row; a fused tile's up rows follow its n gate rows.
         const int n = static_cast<int>(tile_rows(r1, row0, rtile));
         const float* rs = red + slot * kRedSlotFloats;
         for (int i = lane; i < n * MR; i += 32) {
           const int lr = i / MR, m = i - lr * MR;
-          float v = dead ? kNaN : 0.f;
+          float v = (dead || *gave_up) ? kNaN : 0.f;
           for (int w = 0; w < geo.wpt; ++w) v += rs[i * geo.wpt + w];
           const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row0 + lr;
           if (fused) {
@@ -515,7 +519,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 
     // Activations: this lane's 32 inputs of each row, from the ring stage
     // that precedes the segment's tiles.
-    if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
+    if (!dead && !mbar_wait(&full_bar[stage], phase)) { dead = true; *gave_up = 1u; }
     XSlice<4, Q4_GEMV_MAC> xsl[MR];
     {
       const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(smem + static_cast<size_t>(stage) * L.stage_bytes);
@@ -536,7 +540,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     constexpr float kOffset = mac_offset<Q4_GEMV_MAC>();
 
     for (int64_t row0 = r_begin; row0 < r_end; row0 += rtile) {
-      if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
+      if (!dead && !mbar_wait(&full_bar[stage], phase)) { dead = true; *gave_up = 1u; }
       const uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
       // Rows of this tile are dealt to the teams round-robin (row r goes to
       // team r % teams), so a short last tile stays balanced; when a team
@@ -632,9 +636,9 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 
       if (geo.team >= 32) {
         float* rs = red + slot * kRedSlotFloats;
-        if (use_red && !dead && !mbar_wait(&rempty_bar[slot], sph ^ 1u)) dead = true;
+        if (use_red && !dead && !mbar_wait(&rempty_bar[slot], sph ^ 1u)) { dead = true; *gave_up = 1u; }
         if (compute) {
-          const float tot = dead ? kNaN : transpose_reduce<VP>(vals, lane);
+          const float tot = transpose_reduce<VP>(vals, lane);
           const int idx = lane >> (5 - ilog2(VP));
           const int rr = idx / MR, m = idx % MR;
           const bool holder = (lane & ((32 / VP) - 1)) == 0 && idx < V && rr < nv;
@@ -642,7 +646,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
             const int lr = team_idx + rr * geo.teams;  // row within the tile
             if (!use_red) {
               const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row0 + lr;
-              P.y[idx] = store_k<EPI>(tot, P, idx);
+              P.y[idx] = store_k<EPI>(dead ? kNaN : tot, P, idx);
             } else {
               rs[(lr * MR + m) * geo.wpt + warp_in_team] = tot;
             }
@@ -655,7 +659,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < V; ++i) vals[i] = dead ? kNaN : seg_allreduce_dyn(vals[i], geo.team);
+        for (int i = 0; i < V; ++i) vals[i] = seg_allreduce_dyn(vals[i], geo.team);
         if (j == 0) {
 #pragma unroll
           for (int rr = 0; rr < kRpt; ++rr)
@@ -664,7 +668,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 #pragma unroll
               for (int m = 0; m < MR; ++m) {
                 const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row;
-                P.y[idx] = store_k<EPI>(vals[rr * MR + m], P, idx);
+                P.y[idx] = store_k<EPI>(dead ? kNaN : vals[rr * MR + m], P, idx);
               }
             }
         }
@@ -842,7 +846,7 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
     L.prob[i].byte_begin = total;
     total += P.N * problem_row_bytes(P);
   }
-  const size_t fixed = sizeof(float) * kRedSlots * kRedSlotFloats + 16 * kRedSlots;
+  const size_t fixed = sizeof(float) * kRedSlots * kRedSlotFloats + 16 * kRedSlots + 16;
   const size_t budget = std::min<size_t>(Q4_GEMV_SMEM_BUDGET, dev.smem_optin);
   if (fixed + 2 * (stage_bytes + 16) > dev.smem_optin) return cudaErrorInvalidConfiguration;
   int stages = static_cast<int>((budget - fixed) / (stage_bytes + 16));

@@ -10,7 +10,7 @@
 // weights once per pair and multiply every weight by every row on the CUDA
 // cores; this kernel reads them once and the rows cost tensor-core time only.
 // Each weight enters the MMA as two bf16 parts hi + lo (q4_tcgen05.cuh,
-// split_hi_lo), within ~2^-16 of the exact s*q + b.
+// dequant_word_hilo), within ~2^-16 of the exact s*q + b.
 //
 // Segmented-K tiles.  The MMA's 128 rows (tensor-memory lanes) are not 128
 // weight rows: a tile is R weight rows x `segs` segments of K (R * segs =
@@ -39,28 +39,27 @@
 // then the same rows of the up weight; the epilogue keeps the gate's fp32
 // sums in registers and writes silu(gate) * up when the up tile completes.
 //
-// Per CTA (one per SM, 768 threads):
+// Per CTA (one per SM, 608 threads):
 //   warp 0       producer: three bulk copies per tile;
-//   warps 1..3   MMA issue (warp 1 also allocates tensor memory): issuer i
-//                takes chunks c == i (mod I) of every tile (I = 3, 2 or 1 by
+//   warps 1..2   MMA issue (warp 1 also allocates tensor memory): issuer i
+//                takes chunks c == i (mod I) of every tile (I = 2 or 1 by
 //                the problem's accumulator width) into its own double-buffered
 //                fp32 tile.  One thread issues an MMA of these shapes only
 //                every ~50 cycles (its instruction stream, not the tensor
 //                core, is the limit), so several issuers keep pace with the
 //                weight stream.  The split depends on the problem alone, so a
 //                result never depends on the batch;
-//   warps 4..19  dequantize: four groups of four warps (one warp per
+//   warps 3..14  dequantize: three groups of four warps (one warp per
 //                tensor-memory lane quarter) take 64-wide K chunks in turn;
 //                a thread turns 64 codes of its (row, segment) into 32 hi and
-//                32 lo bf16 pairs -- "128 + q" by one LOP3 per two codes, q by
-//                an exact packed subtract, then split_hi_lo -- and stores them
-//                to tensor memory (tcgen05.st);
-//   warps 20..23 epilogue: per tile, read the diagonals of the issuers' fp32
+//                32 lo bf16 pairs (dequant_word_hilo) and stores them to
+//                tensor memory (tcgen05.st);
+//   warps 15..18 epilogue: per tile, read the diagonals of the issuers' fp32
 //                tiles from tensor memory, sum them and the segments
 //                (shuffles), write bf16 y; and, at each new problem, lay out
 //                its B operand.
-// The code pairs come out as (q[t], q[t+4]) of each 8-code word; the B
-// operand is built with the same order of k, so the products pair up.
+// Within a 16-byte run the order of k is natural in both operands (a
+// tensor-memory column holds the bf16 pair k = 2i, 2i + 1).
 // Every wait is bounded (q4_device.cuh); a thread whose wait gave up writes
 // NaN.  Programmatic dependent launch as in the GEMV family.
 #include "q4_device.cuh"
@@ -83,11 +82,18 @@ constexpr bool kSleepWaits = Q4_STREAM_WAIT_SLEEP != 0;
 constexpr int kLanes = 128;                                  // tensor-memory lanes = MMA rows
 constexpr int kChunkK = 64;                                  // K per lane per A chunk
 constexpr int kChunkCols = 64;                               // A chunk in tensor memory: hi (32 columns), lo (32)
-constexpr int kGroups = 4;                                   // dequantizing warp groups
-constexpr int kMaxIssuers = 3;                               // MMA-issuing warps
-constexpr int kFirstDqWarp = 1 + kMaxIssuers;                // 4
-constexpr int kFirstEpiWarp = kFirstDqWarp + 4 * kGroups;   // 20
-constexpr int kThreads = 32 * (kFirstEpiWarp + 4);           // 768: 6 warps per SM sub-partition, <= 80 registers
+#ifndef Q4_STREAM_DQ_GROUPS
+#define Q4_STREAM_DQ_GROUPS 3
+#endif
+// Dequantizing warp groups (4 warps each, one per tensor-memory lane quarter).
+// Three keep the CTA at 19 warps, at most 5 per SM sub-partition, which
+// leaves 96 registers a thread (at 23 warps it would be 80, and the
+// dequantization spills).
+constexpr int kGroups = Q4_STREAM_DQ_GROUPS;
+constexpr int kMaxIssuers = 2;                               // MMA-issuing warps
+constexpr int kFirstDqWarp = 1 + kMaxIssuers;                // 3
+constexpr int kFirstEpiWarp = kFirstDqWarp + 4 * kGroups;   // 15 with three groups
+constexpr int kThreads = 32 * (kFirstEpiWarp + 4);           // 608 with three dequantizing groups
 constexpr int kMaxRows = kStreamMaxRows;                     // activation rows per launch
 constexpr int kMinRows = kStreamMinRows;  // below this the CUDA-core GEMV is faster (it reads the weights once for 1-2 rows)
 constexpr uint32_t kTmemCols = 512;
@@ -117,7 +123,7 @@ struct StreamProblem {
 
 template <int NP>
 struct StreamLaunch {
-  int32_t count, M, stages, a_slots;  // a_slots: A ring chunks (a multiple of 4)
+  int32_t count, M, stages, a_slots;  // a_slots: A ring chunks (a multiple of kGroups)
   uint32_t stage_bytes, b_bytes, a_col0, pad_;  // a_col0: first A ring column (after the accumulators)
   int64_t total_bytes;
   StreamProblem prob[NP];
@@ -143,38 +149,22 @@ __device__ __forceinline__ void gather_diag(uint32_t base, uint32_t issuer_strid
 #pragma unroll
     for (int m = 0; m < kMaxRows; ++m)
       if (m < M) {
-        uint32_t r[W];
-        tmem_ld_cols<W>(base + static_cast<uint32_t>(i) * issuer_stride + static_cast<uint32_t>(m * W), r);
-        tmem_wait_ld();
-        part[m] += pick<W>(r, sel);
+        // W columns in pieces of at most 16 (registers), both loads before one wait
+        constexpr int P = W < 16 ? W : 16;
+        uint32_t r[P], r2[P];
+        const uint32_t col = base + static_cast<uint32_t>(i) * issuer_stride + static_cast<uint32_t>(m * W);
+        if constexpr (W <= 16) {
+          tmem_ld_cols<P>(col, r);
+          tmem_wait_ld();
+          part[m] += pick<P>(r, sel);
+        } else {
+          tmem_ld_cols<P>(col, r);
+          tmem_ld_cols<P>(col + P, r2);
+          tmem_wait_ld();
+          part[m] += sel < P ? pick<P>(r, sel) : pick<P>(r2, sel - P);
+        }
       }
   }
-}
-
-// Eight codes (one word: q0..q7 of eight consecutive k) -> the hi and lo
-// bf16 parts of w_hat for the k pairs (t, t + 4), t = 0..3: "128 + q" by one
-// LOP3 per pair (0x43004300 is bf16 (128, 128), whose last significand bit
-// weighs 1), q by an exact packed subtract, then split_hi_lo.  The LOP3
-// constants come in registers held by the caller across its loop.
-__device__ __forceinline__ void dequant_word(uint32_t w, uint16_t s, float b, uint32_t mask, uint32_t magic,
-                                             uint32_t* hi, uint32_t* lo) {
-  uint32_t v[4];
-  asm("{\n\t.reg .b32 t1, t2, t3;\n\t"
-      "shr.b32 t1, %4, 4;\n\tshr.b32 t2, %4, 8;\n\tshr.b32 t3, %4, 12;\n\t"
-      "lop3.b32 %0, %4, %5, %6, 0xEA;\n\tlop3.b32 %1, t1, %5, %6, 0xEA;\n\t"
-      "lop3.b32 %2, t2, %5, %6, 0xEA;\n\tlop3.b32 %3, t3, %5, %6, 0xEA;\n\t"
-      "sub.rn.bf16x2 %0, %0, %6;\n\tsub.rn.bf16x2 %1, %1, %6;\n\t"
-      "sub.rn.bf16x2 %2, %2, %6;\n\tsub.rn.bf16x2 %3, %3, %6;\n\t}"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
-      : "r"(w), "r"(mask), "r"(magic));
-#pragma unroll
-  for (int t = 0; t < 4; ++t) split_hi_lo(v[t], s, b, kBf16MinusOne, hi[t], lo[t]);
-}
-
-// x[k..k+8) (one 16-byte run) in the (t, t + 4) pair order of dequant_word.
-__device__ __forceinline__ uint4 pair_order(uint4 e) {
-  return make_uint4(__byte_perm(e.x, e.z, 0x5410), __byte_perm(e.x, e.z, 0x7632), __byte_perm(e.y, e.w, 0x5410),
-                    __byte_perm(e.y, e.w, 0x7632));
 }
 
 struct ProblemShape {
@@ -188,7 +178,7 @@ struct ProblemShape {
     chunks = (kseg + kChunkK - 1) / kChunkK;
     full_chunks = kseg / kChunkK;  // the last chunk may be 32 wide
     nb = (segs * M + 15) & ~15;  // MMA N (B rows), a multiple of 16, at most 128
-    issuers = nb <= 16 ? 3 : nb <= 32 ? 2 : 1;
+    issuers = nb <= 32 ? 2 : 1;
     dstride = static_cast<uint32_t>(nb);
   }
 };
@@ -315,8 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     }
   } else if (warp <= kMaxIssuers) {
     // ---------------- MMA issuers ----------------
+    // The whole warp runs the loop (warp-uniform operands); the elected lane
+    // issues the MMAs and commits.
     const int me = warp - 1;
-    if (lane == 0) {
+    const bool leader = elect_one();
+    {
       bool dead = false;
       int lp = 0;
       int slot0 = 0;      // A ring slot of the current tile's first chunk
@@ -337,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
         // B of the previous problem is free once its MMAs are done.  Waiting
         // for this problem's B also means the epilogue has drained every
         // earlier tile, so the accumulator layout may change here.
-        if (lp > 0) tc_commit(bempty);
+        if (lp > 0 && leader) tc_commit(bempty);
         if (!dead && !mbar_wait<kSleepWaits>(bfull, static_cast<uint32_t>(lp & 1))) dead = true;
         tc_fence_after();
         for (int64_t v = v0; v < v1; ++v, ++gt) {
@@ -356,17 +349,21 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
               const uint32_t at = a_base + static_cast<uint32_t>(slot) * kChunkCols;
               const uint64_t bd = bdesc0 + static_cast<uint64_t>(c) * atom16;
               const int ksteps = c < S.full_chunks ? 4 : 2;
-              // the first MMA of this issuer in the tile overwrites its accumulator
-              for (int kk = 0; kk < ksteps; ++kk)  // hi
-                tc_mma_ts(dt, at + 8u * kk, bd + 2u * kk, idesc, (c >= S.issuers || kk > 0) ? 1u : 0u);
-              for (int kk = 0; kk < ksteps; ++kk)  // lo, same activations
-                tc_mma_ts(dt, at + 32u + 8u * kk, bd + 2u * kk, idesc, 1u);
-              tc_commit(&aempty[slot]);
+              if (leader) {
+                // the first MMA of this issuer in the tile overwrites its accumulator
+                for (int kk = 0; kk < ksteps; ++kk)  // hi
+                  tc_mma_ts(dt, at + 8u * kk, bd + 2u * kk, idesc, (c >= S.issuers || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < ksteps; ++kk)  // lo, same activations
+                  tc_mma_ts(dt, at + 32u + 8u * kk, bd + 2u * kk, idesc, 1u);
+                tc_commit(&aempty[slot]);
+              }
+              __syncwarp();
             }
           }
           // every issuer, every tile (count kMaxIssuers); an idle issuer's
           // commit arrives once its earlier MMAs are complete
-          tc_commit(&dfull[db]);
+          if (leader) tc_commit(&dfull[db]);
+          __syncwarp();
           slot0 += S.chunks;
           while (slot0 >= A) { slot0 -= A; ph0 ^= 1u; }
         }
@@ -379,11 +376,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     const int grp = (warp - kFirstDqWarp) >> 2;
     const int tl = 32 * quarter + lane;  // tensor-memory lane of this thread
     const uint32_t a_addr = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + a_col0;
-    uint32_t kmask = 0x000F000Fu, kmagic = 0x43004300u;
-    asm volatile("" : "+r"(kmask), "+r"(kmagic));  // opaque: kept in registers, not rebuilt per use
     bool dead = false;
     int s = 0;
-    uint32_t ph = 0, gc = 0;  // gc: chunks of this CTA before the current tile
+    uint32_t ph = 0;
+    int gmod = 0;             // chunks of this CTA before the current tile, mod kGroups
     int slot0 = 0;            // A ring slot of the current tile's first chunk
     uint32_t ph0 = 0;         // and its phase
     for (int p = 0; p < L.count; ++p) {
@@ -396,14 +392,14 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
       const int r = tl / S.segs, seg = tl % S.segs;  // this lane: row r, segment seg
       const int rot = seg % S.pieces;                  // its code runs, rotated by seg
       const int groups = P.K / 32;
-      for (int64_t v = v0; v < v1; ++v, gc += static_cast<uint32_t>(S.chunks)) {
+      for (int64_t v = v0; v < v1; ++v, gmod = (gmod + S.chunks) % kGroups) {
         if (!dead && !mbar_wait<kSleepWaits>(&full[s], ph)) dead = true;
         const uint8_t* st = ring + static_cast<size_t>(s) * L.stage_bytes;
         const uint8_t* crow = st + r * (P.K / 2) + seg * (S.kseg / 2);  // the segment's 16-byte code runs
         const uint16_t* srow = reinterpret_cast<const uint16_t*>(st + S.R * (P.K / 2)) + r * groups + seg * S.pieces;
         const uint16_t* brow = srow + S.R * groups;
         // the chunks of this group: global index == grp (mod kGroups)
-        for (int c = static_cast<int>((static_cast<uint32_t>(grp) - gc) & (kGroups - 1)); c < S.chunks; c += kGroups) {
+        for (int c = (grp - gmod + kGroups) % kGroups; c < S.chunks; c += kGroups) {
           int slot = slot0 + c;  // ring slot and phase of chunk c
           uint32_t sph = ph0;
           while (slot >= A) { slot -= A; sph ^= 1u; }
@@ -417,18 +413,18 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
               int run = 2 * c + h + rot;
               if (run >= S.pieces) run -= S.pieces;
               const uint4 cw = *reinterpret_cast<const uint4*>(crow + 16 * run);
-              const uint16_t sv = srow[run];
-              const float bv = bf16_bits_to_float(brow[run]);
-              // two words (16 codes) at a time: 8 hi and 8 lo columns
-              uint32_t oh[8], ol[8];
-              dequant_word(cw.x, sv, bv, kmask, kmagic, oh + 0, ol + 0);
-              dequant_word(cw.y, sv, bv, kmask, kmagic, oh + 4, ol + 4);
-              tmem_st_x8(taddr + 16u * h, oh);
-              tmem_st_x8(taddr + 32u + 16u * h, ol);
-              dequant_word(cw.z, sv, bv, kmask, kmagic, oh + 0, ol + 0);
-              dequant_word(cw.w, sv, bv, kmask, kmagic, oh + 4, ol + 4);
-              tmem_st_x8(taddr + 16u * h + 8u, oh);
-              tmem_st_x8(taddr + 32u + 16u * h + 8u, ol);
+              const uint64_t s2 = f32x2_splat(bf16_bits_to_float(srow[run]));
+              const uint64_t b2 = f32x2_splat(bf16_bits_to_float(brow[run]));
+              // 16 codes at a time (the register budget of 768 threads)
+              uint32_t hh[8], ll[8];
+              dequant_word_hilo(cw.x, s2, b2, hh + 0, ll + 0);
+              dequant_word_hilo(cw.y, s2, b2, hh + 4, ll + 4);
+              tmem_st_x8(taddr + 16u * h, hh);
+              tmem_st_x8(taddr + 32u + 16u * h, ll);
+              dequant_word_hilo(cw.z, s2, b2, hh + 0, ll + 0);
+              dequant_word_hilo(cw.w, s2, b2, hh + 4, ll + 4);
+              tmem_st_x8(taddr + 16u * h + 8u, hh);
+              tmem_st_x8(taddr + 32u + 16u * h + 8u, ll);
             }
           }
           tmem_wait_st();
@@ -490,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
             if (i < runs) {
               const int run = i & 7, n = (i >> 3) % S.nb, c = (i >> 3) / S.nb;
               *reinterpret_cast<uint4*>(bmat + static_cast<size_t>(c) * S.nb * 128 + n * 128 + ((run ^ (n & 7)) << 4)) =
-                  pair_order(v[u]);
+                  v[u];
             }
           }
         }
@@ -595,7 +591,7 @@ Plan plan_of(const MatmulArgs& a) {
 constexpr size_t kFixedSmem = 1024 /* alignment */ + 8 * (2 * kMaxStages + 2 * kMaxASlots + 6) + 16;
 
 uint32_t acc_cols_of(uint32_t nb) {
-  const uint32_t issuers = nb <= 16 ? 3u : nb <= 32 ? 2u : 1u;  // as ProblemShape
+  const uint32_t issuers = nb <= 32 ? 2u : 1u;  // as ProblemShape
   return 2u * issuers * nb;
 }
 
@@ -640,11 +636,13 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
   L.stages = stages;
   L.pad_ = 0;
   // Tensor memory: the accumulator tiles of the widest problem, then as deep an
-  // A ring as the rest holds (a multiple of 4 chunks: one slot per dequantizing
-  // group per turn).
+  // A ring as the rest holds (a multiple of kGroups chunks: the chunk of global
+  // index c takes slot c mod a_slots and belongs to group c mod kGroups, so each
+  // group owns its slots and never waits for another group's).
   L.a_col0 = (acc_cols + 31u) & ~31u;
-  L.a_slots = static_cast<int32_t>(std::min<uint32_t>(kMaxASlots, (kTmemCols - L.a_col0) / kChunkCols) & ~3u);
-  if (L.a_slots < 4) return cudaErrorInvalidConfiguration;
+  L.a_slots = static_cast<int32_t>(std::min<uint32_t>(kMaxASlots, (kTmemCols - L.a_col0) / kChunkCols) / kGroups *
+                                   kGroups);
+  if (L.a_slots < kGroups) return cudaErrorInvalidConfiguration;
   L.stage_bytes = stage_bytes;
   L.b_bytes = b_bytes;
   L.total_bytes = total;
@@ -692,7 +690,7 @@ bool stream_supported(const MatmulArgs& a, const DeviceInfo& dev) {
   if (a.K > (int64_t(1) << 20)) return false;
   const Plan pl = plan_of(a);
   if (pl.segs == 0 || pl.nb > 128) return false;
-  if ((kTmemCols - ((acc_cols_of(pl.nb) + 31u) & ~31u)) / kChunkCols < 4) return false;
+  if ((kTmemCols - ((acc_cols_of(pl.nb) + 31u) & ~31u)) / kChunkCols < static_cast<uint32_t>(kGroups)) return false;
   return kFixedSmem + pl.b_bytes + 2 * static_cast<size_t>(pl.stage_bytes) <= dev.smem_optin;
 }
 
@@ -701,7 +699,7 @@ bool stream_supported(const MatmulArgs& a, const DeviceInfo& dev) {
 // largest B operand of another may not fit together.
 bool fits_together(uint32_t stage_bytes, uint32_t b_bytes, uint32_t acc_cols, const DeviceInfo& dev) {
   if (kFixedSmem + b_bytes + 2 * static_cast<size_t>(stage_bytes) > dev.smem_optin) return false;
-  return (kTmemCols - ((acc_cols + 31u) & ~31u)) / kChunkCols >= 4;
+  return (kTmemCols - ((acc_cols + 31u) & ~31u)) / kChunkCols >= static_cast<uint32_t>(kGroups);
 }
 
 cudaError_t launch_stream_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev) {

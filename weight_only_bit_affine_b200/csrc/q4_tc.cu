@@ -14,7 +14,7 @@
 // D[n, m] = w_hat . x^T, so the output tile is y^T) x BN activation rows
 // (the MMA's N side, 16..256) x the CTA's K range, walked in atoms of 64
 // inputs (one 128-byte swizzle span of bf16 x).  Each weight enters the MMA
-// as two bf16 parts, hi + lo (q4_tcgen05.cuh, split_hi_lo), so the operand
+// as two bf16 parts, hi + lo (q4_tcgen05.cuh, dequant_word_hilo), so the operand
 // is within ~2^-16 of the exact s*q + b; every atom is two groups of four
 // K16 MMAs (hi, then lo) into the same accumulator.
 //
@@ -101,24 +101,6 @@ __device__ __forceinline__ uint16_t out_tc(float g, float u, const TcParams& p, 
   return float_to_bf16_bits(g);
 }
 
-// Two code words (16 codes in natural k order) -> 8 hi and 8 lo bf16 pairs.
-__device__ __forceinline__ void dequant_words(uint32_t w0, uint32_t w1, uint16_t s, float b, uint32_t (&hi)[8],
-                                              uint32_t (&lo)[8]) {
-  const uint32_t words[2] = {w0, w1};
-#pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    const uint32_t wd = words[w], w4 = wd >> 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      // bytes [wd.i, wd.i, w4.i, w4.i] -> q[2i] at bits 0..3, q[2i+1] at 16..19
-      const uint32_t pr = __byte_perm(wd, w4, i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-      const uint32_t v = (pr & 0x000F000Fu) | 0x43004300u;  // (128 + q, 128 + q') exactly
-      const uint32_t q = bf16x2_sub(v, 0x43004300u);          // (q, q') exactly
-      split_hi_lo(q, s, b, kBf16MinusOne, hi[4 * w + i], lo[4 * w + i]);
-    }
-  }
-}
-
 template <int ATOMS, bool EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
@@ -173,7 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
-    if (lane == 0) {
+    // The whole warp runs the loop; the elected lane issues the copies.
+    const bool leader = elect_one();
+    {
       bool dead = false;
       int s = 0;
       uint32_t ph = 0;
@@ -182,19 +166,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int a = j * ATOMS;
         const bool up = a >= pass_atoms;
         const int k0 = k_begin + (a - (up ? pass_atoms : 0)) * kAtomK;
-        mbar_arrive_expect_tx(&tma_full[s], ATOMS * (b_atom + kCodeAtomBytes));
+        if (leader) {
+          mbar_arrive_expect_tx(&tma_full[s], ATOMS * (b_atom + kCodeAtomBytes));
 #pragma unroll
-        for (int at = 0; at < ATOMS; ++at)
-          tma_load_2d(b_tile(s) + at * b_atom, &tmap_x, k0 + at * kAtomK, static_cast<int>(m0), &tma_full[s]);
-        tma_load_2d(c_tile(s), up ? &tmap_up : &tmap_codes, k0 / 2, static_cast<int>(n0), &tma_full[s]);
+          for (int at = 0; at < ATOMS; ++at)
+            tma_load_2d(b_tile(s) + at * b_atom, &tmap_x, k0 + at * kAtomK, static_cast<int>(m0), &tma_full[s]);
+          tma_load_2d(c_tile(s), up ? &tmap_up : &tmap_codes, k0 / 2, static_cast<int>(n0), &tma_full[s]);
+        }
+        __syncwarp();
         if (++s == p.stages) { s = 0; ph ^= 1u; }
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     // Waits only for the dequantizing warps: they arrive after having waited
-    // for the stage's TMA themselves, so the x tile is in place too.
-    if (lane == 0) {
+    // for the stage's TMA themselves, so the x tile is in place too.  The
+    // whole warp runs the loop (warp-uniform operands); the elected lane
+    // issues the MMAs and commits.
+    const bool leader = elect_one();
+    {
       bool dead = false;
       const uint32_t a_base = tmem_base + p.a_col0;
       int slot = 0, s = 0, sub = 0;
@@ -207,21 +197,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool first = (a == 0) || (a == pass_atoms);
         const uint64_t bd = sw128_desc(smem_u32(b_tile(s) + sub * b_atom));
         const uint32_t at = a_base + static_cast<uint32_t>(slot) * kASlotCols;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < kAtomK / 16; ++kk)  // hi: 8 columns (16 bf16 along K) per MMA
-          tc_mma_ts(acc, at + 8 * kk, bd + 2 * kk, p.idesc, (first && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < kAtomK / 16; ++kk)  // hi: 8 columns (16 bf16 along K) per MMA
+            tc_mma_ts(acc, at + 8 * kk, bd + 2 * kk, p.idesc, (first && kk == 0) ? 0u : 1u);
 #pragma unroll
-        for (int kk = 0; kk < kAtomK / 16; ++kk)  // lo, same activations
-          tc_mma_ts(acc, at + 32 + 8 * kk, bd + 2 * kk, p.idesc, 1u);
-        tc_commit(&a_empty[slot]);
+          for (int kk = 0; kk < kAtomK / 16; ++kk)  // lo, same activations
+            tc_mma_ts(acc, at + 32 + 8 * kk, bd + 2 * kk, p.idesc, 1u);
+          tc_commit(&a_empty[slot]);
+        }
+        __syncwarp();
         if (++slot == p.a_slots) { slot = 0; aph ^= 1u; }
         if (++sub == ATOMS) {
           sub = 0;
-          tc_commit(&stage_free[s]);
+          if (leader) tc_commit(&stage_free[s]);
+          __syncwarp();
           if (++s == p.stages) { s = 0; ph ^= 1u; }
         }
       }
-      tc_commit(accum_full);
+      if (leader) tc_commit(accum_full);
     }
   } else {
     // ---------------- dequantize, then epilogue ----------------
@@ -249,6 +243,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     load_sb(1, s_nxt, b_nxt);
     bool dead = false;
     int cur_u = 0;
+    // Stage and A slot of this group's atoms, advanced incrementally (atom a
+    // sits in stage (a / ATOMS) mod stages and slot a mod a_slots).
+    constexpr int kStageStep = kDqGroups / ATOMS;  // stages per group turn (ATOMS divides kDqGroups)
+    int st = grp / ATOMS, slot = grp;
+    uint32_t ph = 0, sph = 0;
+    while (st >= p.stages) { st -= p.stages; ph ^= 1u; }
+    while (slot >= p.a_slots) { slot -= p.a_slots; sph ^= 1u; }
     for (int a = grp; a < natoms; a += kDqGroups) {
       const int u = a / kAtomsPerSuper;
       if (u != cur_u) {  // atoms advance by kDqGroups < kAtomsPerSuper: at most one super-chunk at a time
@@ -257,32 +258,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         load_sb(u + 1, s_nxt, b_nxt);
         cur_u = u;
       }
-      const int st = (a / ATOMS) % p.stages;
-      const uint32_t ph = static_cast<uint32_t>((a / ATOMS) / p.stages) & 1u;
       if (!dead && !mbar_wait(&tma_full[st], ph)) dead = true;  // codes arrived
       const uint4 cw =
           *reinterpret_cast<const uint4*>(c_tile(st) + row * (32 * ATOMS) + (a % ATOMS) * 32 + half * 16);
       const int gi = 2 * (a % kAtomsPerSuper) + half;  // group within the super-chunk
       const uint32_t sw = (gi < 2) ? s_cur.x : (gi < 4) ? s_cur.y : (gi < 6) ? s_cur.z : s_cur.w;
       const uint32_t bw = (gi < 2) ? b_cur.x : (gi < 4) ? b_cur.y : (gi < 6) ? b_cur.z : b_cur.w;
-      const uint16_t sh = static_cast<uint16_t>((gi & 1) ? (sw >> 16) : (sw & 0xFFFFu));
-      const float bf = __uint_as_float((gi & 1) ? (bw & 0xFFFF0000u) : (bw << 16));
-      const int slot = a % p.a_slots;
-      const uint32_t sph = static_cast<uint32_t>(a / p.a_slots) & 1u;
+      const uint64_t s2 = f32x2_splat(__uint_as_float((gi & 1) ? (sw & 0xFFFF0000u) : (sw << 16)));
+      const uint64_t b2 = f32x2_splat(__uint_as_float((gi & 1) ? (bw & 0xFFFF0000u) : (bw << 16)));
+      // All 32 codes into registers first (separate arrays: a tcgen05.st reads
+      // its source registers after it issues, so none is overwritten early).
+      uint32_t hi0[8], lo0[8], hi1[8], lo1[8];
+      dequant_word_hilo(cw.x, s2, b2, hi0, lo0);
+      dequant_word_hilo(cw.y, s2, b2, hi0 + 4, lo0 + 4);
+      dequant_word_hilo(cw.z, s2, b2, hi1, lo1);
+      dequant_word_hilo(cw.w, s2, b2, hi1 + 4, lo1 + 4);
       if (!dead && !mbar_wait(&a_empty[slot], sph ^ 1u)) dead = true;  // the MMAs of the slot's last atom are done
       tc_fence_after();
       const uint32_t taddr = lane_addr + p.a_col0 + static_cast<uint32_t>(slot) * kASlotCols + 16u * half;
-      uint32_t hi[8], lo[8];  // 16 codes at a time: 8 hi and 8 lo columns
-      dequant_words(cw.x, cw.y, sh, bf, hi, lo);
-      tmem_st_x8(taddr, hi);
-      tmem_st_x8(taddr + 32u, lo);
-      dequant_words(cw.z, cw.w, sh, bf, hi, lo);
-      tmem_st_x8(taddr + 8u, hi);
-      tmem_st_x8(taddr + 40u, lo);
+      tmem_st_x8(taddr, hi0);
+      tmem_st_x8(taddr + 8u, hi1);
+      tmem_st_x8(taddr + 32u, lo0);
+      tmem_st_x8(taddr + 40u, lo1);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&a_full[slot]);
+      st += kStageStep;
+      while (st >= p.stages) { st -= p.stages; ph ^= 1u; }
+      slot += kDqGroups;
+      while (slot >= p.a_slots) { slot -= p.a_slots; sph ^= 1u; }
     }
 
     // ---- epilogue: tensor memory -> y (or partial sums for the cluster) ----
@@ -433,13 +438,19 @@ cudaError_t plan_tc(const MatmulArgs& a, const DeviceInfo& dev, TcLaunch* out) {
   const int64_t n_tiles = (a.N + kTileN - 1) / kTileN;
   const int64_t m_tiles = (a.M + bn - 1) / bn;
   const int supers = static_cast<int>(a.K / kSuperK);
-  // Split K over a cluster when the tiles alone would leave SMs idle.
+  // Split K over a cluster of up to 8 CTAs when the tiles alone would leave
+  // SMs idle: the split minimising waves x (super-chunks per CTA + 1), the
+  // "+ 1" standing for a CTA's fixed cost (pipeline fill, epilogue, the
+  // cluster's reduction).  One CTA per SM, so a wave is sm_count CTAs.
   int splits = 1;
   const int64_t tiles = n_tiles * m_tiles;
-  while (splits < 8 && splits * 2 <= supers && tiles * splits * 2 <= dev.sm_count) splits *= 2;
-  if (splits < 8 && tiles * splits < dev.sm_count) {
-    const int want = static_cast<int>(std::min<int64_t>(8, (dev.sm_count + tiles - 1) / tiles));
-    if (want > splits && want <= supers && tiles * want <= dev.sm_count * 1.05) splits = want;
+  {
+    int64_t best = -1;
+    for (int sp = 1; sp <= 8 && sp <= supers; ++sp) {
+      const int64_t waves = (tiles * sp + dev.sm_count - 1) / dev.sm_count;
+      const int64_t cost = waves * ((supers + sp - 1) / sp + 1);
+      if (best < 0 || cost < best) { best = cost; splits = sp; }
+    }
   }
 
   // Two atoms per stage when at least three such stages fit.

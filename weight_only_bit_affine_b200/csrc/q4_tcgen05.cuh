@@ -57,6 +57,17 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint
       : "memory");
 }
 
+// True in exactly one lane of the (converged) warp, the same lane every time.
+// The MMA-issuing loops run on a whole warp, so their descriptors and
+// tensor-memory addresses are warp-uniform values, and only the issue itself
+// (an MMA, a commit) is made by the elected lane: issued from a lone lane
+// (lane == 0), every operand would first be moved to the uniform datapath.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+  return pred != 0;
+}
+
 // Arrive on `bar` once every tcgen05 operation this thread issued before is complete.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -123,26 +134,64 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[W]) {
 // |w_hat - hi - lo| <= 2^-24 |w_hat| + 2^-8 |w32 - hi| <= ~2^-16 |w_hat|: the
 // operand error is 256 times below the output rounding, with no cancellation
 // anywhere (hi and lo have the sign of w_hat or are far smaller).
+//
+// Instruction count per pair of weights: the codes become exact fp32 values
+// in place (unpack_codes_f32: a LOP3 per code, a packed add per pair), w32 is
+// one packed fp32 fma (fma.rn.f32x2), hi one conversion, the remainder one
+// packed subtraction of hi widened back to fp32 (a shift and an AND), lo one
+// conversion.
 
-// bf16 -1.0: multiplies hi's bf16 halves in the exact subtraction below.
-constexpr uint16_t kBf16MinusOne = 0xBF80u;
+// {v, v} as the 64-bit operand of the packed fp32 instructions.
+__device__ __forceinline__ uint64_t f32x2_splat(float v) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+  return r;
+}
 
-// q2: two exact codes as a bf16 pair (q_lo in bits 0..15, q_hi in 16..31);
-// s: the group's bf16 scale bits; b: its bias as fp32; m1: kBf16MinusOne.
-// Returns the pairs (hi_lo, hi_hi) and (lo_lo, lo_hi) in the same order.
-__device__ __forceinline__ void split_hi_lo(uint32_t q2, uint16_t s, float b, uint16_t m1, uint32_t& hi,
-                                            uint32_t& lo) {
-  asm("{\n\t.reg .b16 ql, qh, hl, hh;\n\t.reg .f32 wl, wh, rl, rh;\n\t"
-      "mov.b32 {ql, qh}, %2;\n\t"
-      "fma.rn.f32.bf16 wl, ql, %3, %4;\n\t"
-      "fma.rn.f32.bf16 wh, qh, %3, %4;\n\t"
-      "cvt.rn.bf16x2.f32 %0, wh, wl;\n\t"
-      "mov.b32 {hl, hh}, %0;\n\t"
-      "fma.rn.f32.bf16 rl, hl, %5, wl;\n\t"
-      "fma.rn.f32.bf16 rh, hh, %5, wh;\n\t"
-      "cvt.rn.bf16x2.f32 %1, rh, rl;\n\t}"
+// One pair (q0, q1) of exact codes in fp32 -> the bf16 pairs hi = (hi0, hi1)
+// and lo = (lo0, lo1) of s*q + b (element 0 in bits 0..15); s2 = {s, s}, b2 =
+// {b, b} from f32x2_splat.
+__device__ __forceinline__ void split_pair(float q0, float q1, uint64_t s2, uint64_t b2, uint32_t& hi,
+                                           uint32_t& lo) {
+  asm("{\n\t.reg .b64 rq, rw, rh, rr;\n\t.reg .f32 w0, w1, r0, r1;\n\t.reg .b32 t0, t1;\n\t"
+      "mov.b64 rq, {%2, %3};\n\t"
+      "fma.rn.f32x2 rw, rq, %4, %5;\n\t"
+      "mov.b64 {w0, w1}, rw;\n\t"
+      "cvt.rn.bf16x2.f32 %0, w1, w0;\n\t"
+      "shl.b32 t0, %0, 16;\n\t"
+      "and.b32 t1, %0, 0xFFFF0000;\n\t"
+      "mov.b64 rh, {t0, t1};\n\t"
+      "sub.rn.f32x2 rr, rw, rh;\n\t"
+      "mov.b64 {r0, r1}, rr;\n\t"
+      "cvt.rn.bf16x2.f32 %1, r1, r0;\n\t}"
       : "=r"(hi), "=r"(lo)
-      : "r"(q2), "h"(s), "f"(b), "h"(m1));
+      : "f"(q0), "f"(q1), "l"(s2), "l"(b2));
+}
+
+// One packed word (codes of eight consecutive k, q_j in bits 4j..4j+3) ->
+// four hi and four lo bf16 pairs, pair i = (k 2i, k 2i+1).  Each code becomes
+// an exact fp32 in place: masked into the significand of 2^(23-p), where its
+// lowest bit p weighs 1, then the offsets 2^(23-p) removed by one packed add
+// per pair (codes 5..7 are shifted down by 12 bits first).
+__device__ __forceinline__ void dequant_word_hilo(uint32_t w, uint64_t s2, uint64_t b2, uint32_t* hi, uint32_t* lo) {
+  const uint32_t ws = w >> 12;
+  float q0, q1;
+  q0 = __uint_as_float((w & 0x0000000Fu) | 0x4B000000u);   // 2^23 + q0
+  q1 = __uint_as_float((w & 0x000000F0u) | 0x49000000u);   // 2^19 + q1
+  fadd2(q0, q1, -8388608.f, -524288.f);
+  split_pair(q0, q1, s2, b2, hi[0], lo[0]);
+  q0 = __uint_as_float((w & 0x00000F00u) | 0x47000000u);   // 2^15 + q2
+  q1 = __uint_as_float((w & 0x0000F000u) | 0x45000000u);   // 2^11 + q3
+  fadd2(q0, q1, -32768.f, -2048.f);
+  split_pair(q0, q1, s2, b2, hi[1], lo[1]);
+  q0 = __uint_as_float((w & 0x000F0000u) | 0x43000000u);   // 2^7 + q4
+  q1 = __uint_as_float((ws & 0x00000F00u) | 0x47000000u);  // 2^15 + q5
+  fadd2(q0, q1, -128.f, -32768.f);
+  split_pair(q0, q1, s2, b2, hi[2], lo[2]);
+  q0 = __uint_as_float((ws & 0x0000F000u) | 0x45000000u);  // 2^11 + q6
+  q1 = __uint_as_float((ws & 0x000F0000u) | 0x43000000u);  // 2^7 + q7
+  fadd2(q0, q1, -2048.f, -128.f);
+  split_pair(q0, q1, s2, b2, hi[3], lo[3]);
 }
 
 }  // namespace q4
