@@ -348,13 +348,20 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
               tc_fence_after();
               const uint32_t at = a_base + static_cast<uint32_t>(slot) * kChunkCols;
               const uint64_t bd = bdesc0 + static_cast<uint64_t>(c) * atom16;
-              const int ksteps = c < S.full_chunks ? 4 : 2;
               if (leader) {
                 // the first MMA of this issuer in the tile overwrites its accumulator
-                for (int kk = 0; kk < ksteps; ++kk)  // hi
-                  tc_mma_ts(dt, at + 8u * kk, bd + 2u * kk, idesc, (c >= S.issuers || kk > 0) ? 1u : 0u);
-                for (int kk = 0; kk < ksteps; ++kk)  // lo, same activations
-                  tc_mma_ts(dt, at + 32u + 8u * kk, bd + 2u * kk, idesc, 1u);
+                const uint32_t acc0 = c >= S.issuers ? 1u : 0u;
+                if (c < S.full_chunks) {  // 64 k: four K16 steps of hi, then of lo
+#pragma unroll
+                  for (int kk = 0; kk < 4; ++kk) tc_mma_ts(dt, at + 8u * kk, bd + 2u * kk, idesc, kk ? 1u : acc0);
+#pragma unroll
+                  for (int kk = 0; kk < 4; ++kk) tc_mma_ts(dt, at + 32u + 8u * kk, bd + 2u * kk, idesc, 1u);
+                } else {  // the segment's last 32 k
+#pragma unroll
+                  for (int kk = 0; kk < 2; ++kk) tc_mma_ts(dt, at + 8u * kk, bd + 2u * kk, idesc, kk ? 1u : acc0);
+#pragma unroll
+                  for (int kk = 0; kk < 2; ++kk) tc_mma_ts(dt, at + 32u + 8u * kk, bd + 2u * kk, idesc, 1u);
+                }
                 tc_commit(&aempty[slot]);
               }
               __syncwarp();
