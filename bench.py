@@ -244,6 +244,9 @@ def _graph_ms(dev, fn, reps):
     return ms
 
 
+GMMA_PATH = ("gmma_kernel: tcgen05 group sums of (128 + q) * x in tensor memory, scale and bias in fp32; "
+             "steps spread evenly over the SMs")
+
 # Rows of the batched-layer workload (M in {4, 64, 256}), with the row counts
 # in between where the kernel choice changes (weight streaming up to 8 rows,
 # tensor-core tiles from 9, one 16-row tile up to 16).
@@ -424,7 +427,7 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
     rows["depformer_steps_M4"] = {
         "batched_us_per_step": round(ms_m4 * 1e3 / steps, 2), "batched_ms_per_frame": round(ms_m4, 4),
         "packed_GBps": round(fbytes / (ms_m4 * 1e-3) / 1e9, 1),
-        "path": "stream_kernel: tcgen05 weight streaming, dequantized hi/lo operand in tensor memory",
+        "path": GMMA_PATH,
         "note": "four conversations' rows per step slice, one q4_matmul_batch launch per codebook step",
     }
     del dep
@@ -445,8 +448,8 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
         rows[f"batched_layer_M{M}"] = {
             "us_per_layer": round(t * 1e3, 2), "TFLOPs": round(tf, 1),
             "frac_of_bf16_peak": round(tf / bf16_peak, 4), "packed_GBps": round(lbytes / (t * 1e-3) / 1e9, 1),
-            "path": ("tc_kernel: tcgen05 tiles, dequantized hi/lo operand in tensor memory" if M > 8 else
-                     "stream_kernel: tcgen05 weight streaming, dequantized hi/lo operand in tensor memory"
+            "path": ("tc_kernel: tcgen05 tiles, dequantized hi/lo operand in tensor memory" if M > 16 else
+                     GMMA_PATH
                      if M >= 3 else "gemv_kernel: CUDA cores"),
         }
     return rows
@@ -534,6 +537,8 @@ class OracleSample:
 #   tc_gate        the gate projection (11264 x 4096) alone at M = 64, then 256.
 #   depformer_step one depformer codebook step (43 step-sliced projections) as
 #                  one q4_matmul_batch.
+#   layer_m1       one temporal layer (7 projections) at M = 1 as one
+#                  q4_matmul_batch.
 #   layer_m4       one temporal layer (7 projections) at M = 4 as one
 #                  q4_matmul_batch: the tensor-core weight-streaming kernel.
 #   layer_m8       the same at M = 8.
@@ -670,7 +675,8 @@ def _tc_gate(dev):
 
 
 PROFILE_CASES = {"stream_small": _stream_small, "tc_layer": _tc_layer, "tc_gate": _tc_gate,
-                 "depformer_step": _depformer_step, "layer_m4": lambda dev: _layer_rows(dev, 4),
+                 "depformer_step": _depformer_step, "layer_m1": lambda dev: _layer_rows(dev, 1),
+                 "layer_m4": lambda dev: _layer_rows(dev, 4),
                  "layer_m8": lambda dev: _layer_rows(dev, 8), "fused_layer": _fused_layer, "q8_layer": _q8_layer}
 
 

@@ -112,17 +112,30 @@ Q4_API q4_status q4_dequantize(const uint8_t* codes, const q4_bf16* scales,
  * are not expanded back to BF16).
  * In:  x [M, K] bf16 (row-major), codes [N, K/2], scales, biases [N, K/32].
  * Out: y [M, N] bf16 (row-major).
- * Kernel by problem (the same for a problem alone or batched, so a batched
- * result is bit-identical to the single call): M = 1, 2 the CUDA-core GEMV
- * (exact products x * (128 + q) in fp32, the offset removed per group);
- * M = 3..8 tensor-core weight streaming where its shared and tensor memory
- * hold the problem (K % 256 == 0, 16-byte aligned scale and bias rows,
- * segments * M <= 128); otherwise, for M >= 3 with K % 256 == 0 and the same
- * alignment, tensor-core tiles; otherwise the GEMV on pairs of activation
- * rows.  Every kernel reads each weight byte once per call, except the GEMV
- * on pairs (once per pair).  The tensor-core kernels feed each weight to the
- * MMA as two bf16 parts hi + lo with |s*q + b - hi - lo| <= ~2^-16 |s*q + b|
- * (two MMAs per K step), so no path rounds w_hat to bf16.
+ * Kernel by problem (the same for a problem alone or batched): M = 1, 2 the
+ * CUDA-core GEMV (exact products x * (128 + q) in fp32, the offset removed
+ * per group); M = 3..16 with K % 256 == 0 and 16-byte aligned x, codes,
+ * scale and bias rows, the group-sum tensor-core kernel (exact sums of
+ * (128 + q) * x per group of 32 on the tensor cores, the group's scale and
+ * bias applied in fp32; the launch's 128-input steps are spread evenly over
+ * the SMs, so a tile may be shared by several CTAs whose fp32 partial sums
+ * are added in a fixed order); otherwise M = 3..8 tensor-core weight
+ * streaming where its shared and tensor memory hold the problem (16-byte
+ * aligned scale and bias rows, segments * M <= 128); otherwise, for M >= 3
+ * with K % 256 == 0 and aligned scale rows, tensor-core tiles; otherwise the
+ * GEMV on pairs of activation rows.  Every kernel reads each weight byte once
+ * per call, except the GEMV on pairs (once per pair).  The streaming and tile
+ * kernels feed each weight to the MMA as two bf16 parts hi + lo with
+ * |s*q + b - hi - lo| <= ~2^-16 |s*q + b| (two MMAs per K step), so no path
+ * rounds w_hat to bf16.  Results are deterministic: the same call gives the
+ * same bits.  On the GEMV, the weight-streaming kernel and the tiles a
+ * problem's result is also the same alone or in any batch; on the group-sum
+ * kernel the fp32 partial sums follow the launch's split over the SMs, so a
+ * problem can differ in the last bits between batches (always within the
+ * acceptance bound).  A group-sum launch that shares tiles takes a small
+ * stream-ordered workspace (cudaMallocAsync / cudaFreeAsync on `stream`:
+ * about 2 * SMs * 128 * 2 * M * 4 bytes plus SMs counters, zeroed by a
+ * cudaMemsetAsync); an allocation failure is Q4_ERR_CUDA.
  * Launch-order contract: the kernels may be launched with programmatic
  * dependent launch; they read nothing written by an earlier kernel in the
  * stream before that kernel has completed.
@@ -210,10 +223,13 @@ Q4_API q4_status q4_matmul_swiglu(const q4_bf16* x, int64_t M, int64_t K, const 
 
 /*
  * q4_matmul_batch -- `count` independent matmuls sharing the number of
- * activation rows M, each computing exactly what q4_matmul computes, enqueued
+ * activation rows M, each computing what q4_matmul computes (on the same
+ * kernel; see q4_matmul for the group-sum kernel's summation order), enqueued
  * as few kernel launches as possible: one for up to 256 problems that take
- * the bulk-copy GEMV path (or the weight-streaming path), one per problem on
- * the tensor-core tile path and on the GEMV's generic fallback.  The Swift/MLX blog ("Performance optimizations":
+ * the bulk-copy GEMV path (or the weight-streaming path), one for up to 160
+ * weights (a SwiGLU problem counts two) with at most 8 distinct activation
+ * tensors on the group-sum path, one per problem on the tensor-core tile
+ * path and on the GEMV's generic fallback.  The Swift/MLX blog ("Performance optimizations":
  * compiling the temporal transformer fuses its ~450 per-step kernel
  * dispatches) and the ONNX README ("All four variants": CUDA Graph capture)
  * both cut per-call launch overhead; this is that fusion for a whole weight
@@ -280,6 +296,20 @@ Q4_API int q4_device_status(int clear);
  * (counted on the host when each launch is issued; graph replays of captured
  * launches are not counted again). */
 Q4_API unsigned long long q4_debug_launch_count(void);
+
+/* Diagnostic: kernel families the matmul dispatch may not choose, as a bit
+ * mask (0 = all allowed, the default): Q4_KERNEL_GROUP_SUM (the group-sum
+ * tensor-core kernel, 3..16 activation rows), Q4_KERNEL_WEIGHT_STREAM (the
+ * weight-streaming tensor-core kernel, 3..8 rows) and Q4_KERNEL_TILES (the
+ * tensor-core tiles, 3 or more rows).  A problem none of its allowed
+ * tensor-core kernels takes goes to the CUDA-core GEMV, which takes every
+ * problem.  For tests that pin a kernel to a problem; process-wide, read at
+ * each call (set it while no other thread enqueues).  Returns the previous
+ * mask. */
+#define Q4_KERNEL_GROUP_SUM 1u
+#define Q4_KERNEL_WEIGHT_STREAM 2u
+#define Q4_KERNEL_TILES 4u
+Q4_API unsigned int q4_debug_disable_kernels(unsigned int mask);
 
 #ifdef __cplusplus
 }

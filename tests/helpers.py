@@ -1,5 +1,7 @@
 """Shared helpers for the GPU parity tests: move seeded inputs to the device,
 call the library through its binding, and compare against the CPU oracle."""
+import contextlib
+
 import numpy as np
 import torch
 
@@ -57,3 +59,14 @@ def gpu_weight(N, K, seed, tensor, device="cuda"):
 
 def quantize_dev(W):
     return q4.q4_quantize(W)
+
+
+@contextlib.contextmanager
+def kernels_disabled(mask: int):
+    """Run the block with the given kernel families (q4.KERNEL_* bits) kept
+    out of the matmul dispatch, to pin a problem to another kernel."""
+    prev = q4.q4_debug_disable_kernels(mask)
+    try:
+        yield
+    finally:
+        q4.q4_debug_disable_kernels(prev)

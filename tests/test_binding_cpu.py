@@ -70,3 +70,13 @@ def test_batch_out_on_another_device(fake):
 def test_empty_batch_needs_no_library(fake):
     assert q4.q4_matmul_batch([]) == []
     assert q4.q4_prepare_batch([]) is None
+
+
+def test_disable_kernels_round_trip():
+    """The dispatch mask is host state: set, read back, restored (no GPU)."""
+    prev = q4.q4_debug_disable_kernels(q4.KERNEL_GROUP_SUM | q4.KERNEL_TILES)
+    try:
+        assert q4.q4_debug_disable_kernels(q4.KERNEL_WEIGHT_STREAM) == q4.KERNEL_GROUP_SUM | q4.KERNEL_TILES
+        assert q4.q4_debug_disable_kernels(0) == q4.KERNEL_WEIGHT_STREAM
+    finally:
+        q4.q4_debug_disable_kernels(prev)

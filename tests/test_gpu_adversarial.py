@@ -3,10 +3,11 @@ all products x_k * w_hat_k non-negative, so |y| = sum |x w_hat| and the bf16
 output rounding alone takes up to 3.9e-3 of the 4e-3 budget, with codes chosen
 so that rounding w_hat to bf16 would push nearly every product the same way.
 
-Rows M = 1, 2 (CUDA-core GEMV), 3..8 (tensor-core weight streaming), 5..15 and
-16..256 (tensor-core tiles, from one 16-row tile to a full 256-row one) at
-K = 4096 and 11264, every element of every output checked, and the fused
-residual and SwiGLU epilogues on the same inputs."""
+Rows M = 1, 2 (CUDA-core GEMV), 3..16 (group-sum tensor-core kernel) and
+64, 256 (tensor-core tiles) at K = 4096 and 11264, every element of every
+output checked, and the fused residual and SwiGLU epilogues on the same
+inputs; the weight-streaming kernel (3..8 rows) and the tiles at 16 rows are
+pinned by keeping the group-sum kernel out of the dispatch."""
 import numpy as np
 import pytest
 import torch
@@ -14,7 +15,7 @@ import torch
 import adversarial
 import oracle
 import weight_only_bit_affine_b200 as q4
-from helpers import ABS, REL
+from helpers import ABS, REL, kernels_disabled
 
 pytestmark = pytest.mark.gpu
 
@@ -93,3 +94,17 @@ def test_swiglu_adversarial(family, M):
     torch.cuda.synchronize()
     ref, bound = oracle.matmul_swiglu_ref(x[:M], gate_h, up_h)
     _check(h, ref, bound, f"swiglu {family} M={M}")
+
+
+@pytest.mark.parametrize("K", [4096, 11264])
+@pytest.mark.parametrize("M", [4, 8, 16])
+@pytest.mark.parametrize("family", adversarial.FAMILIES)
+def test_matmul_adversarial_other_kernels(family, M, K):
+    """The same inputs on the weight-streaming kernel (M = 4, 8) and on the
+    tensor-core tiles (M = 16)."""
+    x, host, xd, dev = _case(family, K)
+    with kernels_disabled(q4.KERNEL_GROUP_SUM):
+        y = q4.q4_matmul(xd[:M].contiguous(), *dev)
+        torch.cuda.synchronize()
+    ref, absdot = oracle.matmul_ref(x[:M], *host)
+    _check(y, ref, REL * absdot + ABS, f"{family} M={M} K={K} (pinned)")

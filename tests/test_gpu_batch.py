@@ -1,7 +1,12 @@
 """q4_matmul_batch: many independent matmuls in few launches.
 
-Each problem must come out exactly as q4_matmul computes it alone (same
-kernel geometry, so bit-identical), and within the oracle bound.
+On the CUDA-core GEMV (1 and 2 activation rows) each problem comes out
+exactly as q4_matmul computes it alone (same kernel geometry, so
+bit-identical).  The group-sum kernel (3..16 rows) spreads a launch's steps
+evenly over the SMs, so where a CTA boundary falls inside a tile depends on
+the whole batch and the order of the fp32 partial sums with it: there each
+problem is checked against the oracle bound, and the batch against itself
+(a call is deterministic).
 """
 import numpy as np
 import pytest
@@ -39,10 +44,15 @@ def test_batch_matches_single_calls(M):
         probs.append((x, c, s, b, out))
         singles.append(q4.q4_matmul(x, c, s, b))
     q4.q4_matmul_batch(probs)
+    first = [out.clone() for *_, out in probs]
+    q4.q4_matmul_batch(probs)
     torch.cuda.synchronize()
-    for (x, c, s, b, out), ref, (N, K) in zip(probs, singles, shapes):
-        assert torch.equal(out, ref), (N, K)
+    for (x, c, s, b, out), ref, again, (N, K) in zip(probs, singles, first, shapes):
+        assert torch.equal(out, again), (N, K)  # deterministic
+        if M <= 2:
+            assert torch.equal(out, ref), (N, K)
         check_matmul(x, c, s, b, out, rows=sample_rows(N, 32, seed=N), what=f"batch {N}x{K} M={M}")
+        check_matmul(x, c, s, b, ref, rows=sample_rows(N, 32, seed=N), what=f"single {N}x{K} M={M}")
 
 
 def test_batch_more_than_one_launch():

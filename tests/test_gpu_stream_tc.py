@@ -1,5 +1,7 @@
 """Tensor-core weight streaming (three or four activation rows, K % 256 == 0,
-16-byte aligned scale rows): parity with the CPU oracle.
+16-byte aligned scale rows): parity with the CPU oracle.  The group-sum kernel
+takes these problems by default; it is kept out of the dispatch here so that
+the weight-streaming kernel runs.
 
 A tile is R weight rows x (128 / R) segments of K in the MMA's 128 rows, with
 R = 4, 8 or 16 depending on K (segments of K/32, K/16 or K/8 inputs); these
@@ -32,7 +34,9 @@ def _gpu():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     q4.q4_device_status(clear=True)
+    prev = q4.q4_debug_disable_kernels(q4.KERNEL_GROUP_SUM)
     yield
+    q4.q4_debug_disable_kernels(prev)
     assert q4.q4_device_status() == 0, "a bounded wait gave up inside a kernel"
 
 

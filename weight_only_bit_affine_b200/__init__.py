@@ -53,6 +53,10 @@ __all__ = [
     "q4_device_status",
     "q4_check_device",
     "q4_debug_launch_count",
+    "q4_debug_disable_kernels",
+    "KERNEL_GROUP_SUM",
+    "KERNEL_WEIGHT_STREAM",
+    "KERNEL_TILES",
 ]
 
 GROUP = 32
@@ -85,6 +89,7 @@ SIGNATURES = {
     "q4_last_error": (ctypes.c_char_p, []),
     "q4_device_status": (_INT, [_INT]),
     "q4_debug_launch_count": (ctypes.c_ulonglong, []),
+    "q4_debug_disable_kernels": (ctypes.c_uint, [ctypes.c_uint]),
 }
 
 
@@ -452,3 +457,12 @@ def q4_check_device(clear: bool = True) -> None:
 def q4_debug_launch_count() -> int:
     """Kernel launches libq4 has enqueued in this process (host-side count)."""
     return int(lib().q4_debug_launch_count())
+
+
+KERNEL_GROUP_SUM, KERNEL_WEIGHT_STREAM, KERNEL_TILES = 1, 2, 4  # Q4_KERNEL_* (include/q4.h)
+
+
+def q4_debug_disable_kernels(mask: int) -> int:
+    """Kernel families the matmul dispatch may not choose (KERNEL_* bits; 0 =
+    all allowed); returns the previous mask.  For tests that pin a kernel."""
+    return int(lib().q4_debug_disable_kernels(ctypes.c_uint(mask)))

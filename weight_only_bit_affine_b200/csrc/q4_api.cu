@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
+#include <algorithm>
 #include <vector>
 
 namespace q4 {
@@ -25,6 +26,7 @@ q4_status fail(q4_status st, const char* fmt, ...) {
 }
 
 std::atomic<unsigned long long> g_launches{0};
+std::atomic<unsigned int> g_disabled_kernels{0};  // q4_debug_disable_kernels
 
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
@@ -107,21 +109,27 @@ q4_status check_epilogue(const char* who, int32_t epi, int32_t reserved, const u
 
 // Enqueues a validated, non-empty list.  Each problem takes the kernel it
 // would take alone (so a batched result is bit-identical to the single
-// call): the weight-streaming kernel where it takes the problem (3..8
-// activation rows), else the tensor-core tiles (3 or more rows), else the
-// CUDA-core GEMV.  Problems on the bulk-copy GEMV and on the weight-streaming
-// kernel share a launch per path; SwiGLU problems run in one pass on every
-// path.  Every host-side step that can fail for a valid call (tensor-map
-// encoding, configuration checks) runs before the first launch.
+// call): the group-sum tensor-core kernel where it takes the problem (1..16
+// activation rows), else the weight-streaming kernel (3..8 rows), else the
+// tensor-core tiles (3 or more rows), else the CUDA-core GEMV.  Problems on
+// the group-sum kernel, the bulk-copy GEMV and the weight-streaming kernel
+// share launches per path; SwiGLU problems run in one pass on every path.
+// Every host-side step that can fail for a valid call (tensor-map encoding,
+// configuration checks) runs before the first launch.
 q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& dev, cudaStream_t cs,
                        const char* what) {
-  std::vector<MatmulArgs> gemv, streamed;
+  std::vector<MatmulArgs> gemv, streamed, grouped;
   thread_local std::vector<TcLaunch> tc;
+  thread_local std::vector<GmmaPlan> gm;
   tc.clear();
+  gm.clear();
+  const unsigned int off = g_disabled_kernels.load(std::memory_order_relaxed);
   for (const MatmulArgs& a : list) {
-    if (stream_supported(a, dev)) {
+    if (!(off & Q4_KERNEL_GROUP_SUM) && gmma_supported(a, dev)) {
+      grouped.push_back(a);
+    } else if (!(off & Q4_KERNEL_WEIGHT_STREAM) && stream_supported(a, dev)) {
       streamed.push_back(a);
-    } else if (a.M >= kTensorCoreMinRows && tc_supported(a)) {
+    } else if (!(off & Q4_KERNEL_TILES) && a.M >= kTensorCoreMinRows && tc_supported(a)) {
       tc.emplace_back();
       const cudaError_t e = plan_tc(a, dev, &tc.back());
       if (e != cudaSuccess) return from_cuda(e, what);
@@ -129,7 +137,39 @@ q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& de
       gemv.push_back(a);
     }
   }
+  if (!grouped.empty()) {
+    const cudaError_t e = plan_gmma(grouped.data(), static_cast<int>(grouped.size()), dev, gm);
+    if (e != cudaSuccess) return from_cuda(e, what);
+  }
   q4_status st = Q4_OK;
+  if (!gm.empty()) {
+    // One stream-ordered workspace for the launches that share tiles between
+    // CTAs: their arrival counters (zeroed here) and then their partial sums.
+    size_t cbytes = 0, pbytes = 0;
+    for (const GmmaPlan& g : gm) {
+      cbytes += g.counter_bytes;
+      pbytes += g.partial_bytes;
+    }
+    unsigned char* ws = nullptr;
+    if (cbytes + pbytes > 0) {
+      cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), cbytes + pbytes, cs);
+      if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, cbytes, cs);
+      if (e != cudaSuccess) return from_cuda(e, what);
+    }
+    size_t co = 0, po = cbytes;
+    for (GmmaPlan& g : gm) {
+      unsigned int* counters = g.counter_bytes ? reinterpret_cast<unsigned int*>(ws + co) : nullptr;
+      float* partials = g.partial_bytes ? reinterpret_cast<float*>(ws + po) : nullptr;
+      co += g.counter_bytes;
+      po += g.partial_bytes;
+      if ((st = from_cuda(launch_planned_gmma(g, counters, partials, cs), what)) != Q4_OK) break;
+    }
+    if (ws != nullptr) {
+      const cudaError_t e = cudaFreeAsync(ws, cs);
+      if (st == Q4_OK && e != cudaSuccess) st = from_cuda(e, what);
+    }
+    if (st != Q4_OK) return st;
+  }
   for (const TcLaunch& t : tc)
     if ((st = from_cuda(launch_planned_tc(t, cs), what)) != Q4_OK) return st;
   if (!streamed.empty() &&
@@ -193,7 +233,7 @@ const DeviceInfo* current_device_info() {
     // cudaFuncSetAttribute applies to the current device, which is `dev`.
     if (d.cc_major == 10 && d.cc_minor == 0) {
       if ((e = gemv_prepare_device(d)) == cudaSuccess && (e = tc_prepare_device(d)) == cudaSuccess &&
-          (e = stream_prepare_device(d)) == cudaSuccess)
+          (e = stream_prepare_device(d)) == cudaSuccess && (e = gmma_prepare_device(d)) == cudaSuccess)
         e = q8_prepare_device(d);
       if (e != cudaSuccess) {
         fail(Q4_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(e));
@@ -361,12 +401,14 @@ const char* q4_last_error(void) { return t_last_error; }
 
 unsigned long long q4_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+unsigned int q4_debug_disable_kernels(unsigned int mask) { return g_disabled_kernels.exchange(mask); }
+
 int q4_device_status(int clear) {
-  unsigned int f = 0, t = 0, s = 0;
+  unsigned int f = 0, t = 0, s = 0, g = 0;
   if (gemv_device_flags(&f, clear != 0) != cudaSuccess || tc_device_flags(&t, clear != 0) != cudaSuccess ||
-      stream_device_flags(&s, clear != 0) != cudaSuccess)
+      stream_device_flags(&s, clear != 0) != cudaSuccess || gmma_device_flags(&g, clear != 0) != cudaSuccess)
     return -1;
-  f |= t | s;
+  f |= t | s | g;
   return static_cast<int>(f);
 }
 

@@ -109,6 +109,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// As mbar_wait, but between polls the thread sleeps about kNs nanoseconds
+// (nanosleep): a polling warp takes no issue slots and no ALU cycles from
+// the warps that do the work on its SM sub-partition while it waits.
+template <unsigned kNs>
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 8; ++i) {
+      __nanosleep(kNs);
+      if (mbar_try_wait(bar, parity)) return true;
+    }
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_device_flags, kFlagWaitTimeout);
+      return false;
+    }
+  }
+}
+
 // ---- bulk (non-tensor TMA) copies and prefetch ----------------------------
 // Global -> shared, completion counted in bytes on `bar`.  dst, src 16-byte
 // aligned; bytes a multiple of 16.

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <atomic>
 #include <cstdint>
+#include <vector>
 
 namespace q4 {
 
@@ -122,12 +123,35 @@ constexpr int kStreamMinRows = 3, kStreamMaxRows = 8;
 bool stream_supported(const MatmulArgs& a, const DeviceInfo& dev);
 cudaError_t launch_stream_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
 
+// Group-sum tensor-core kernel (q4_gmma.cu: tcgen05 sums of 128 + q per
+// group, scales and biases applied in fp32) for kGmmaMinRows..kGmmaMaxRows
+// activation rows (1 and 2 rows stay on the CUDA-core GEMV, which is faster
+// there); a launch takes many problems of one M.  plan_gmma encodes every
+// tensor map (and may fail) before anything is launched.
+constexpr int64_t kGmmaMinRows = 3, kGmmaMaxRows = 16;
+// A launch balances the steps (128 inputs of a 128-row tile) over all SMs;
+// a tile that two or more CTAs share needs a workspace: counter_bytes of
+// arrival counters (zero at launch) and partial_bytes of fp32 partial sums.
+constexpr size_t kGmmaParamBytes = 32768;
+struct GmmaPlan {
+  alignas(64) unsigned char params[kGmmaParamBytes];  // the kernel's parameter block
+  int grid;
+  size_t smem;
+  const void* kern;
+  size_t counter_bytes, partial_bytes;  // both 0: no tile is shared
+};
+bool gmma_supported(const MatmulArgs& a, const DeviceInfo& dev);
+cudaError_t plan_gmma(const MatmulArgs* list, int count, const DeviceInfo& dev, std::vector<GmmaPlan>& plans);
+// counters / partials: the plan's workspace (NULL when its sizes are 0).
+cudaError_t launch_planned_gmma(GmmaPlan& plan, unsigned int* counters, float* partials, cudaStream_t stream);
+
 // One-time settings of a device's kernels (dynamic shared memory, cluster
 // sizes), made before the first launch on the device.
 cudaError_t gemv_prepare_device(const DeviceInfo& dev);
 cudaError_t tc_prepare_device(const DeviceInfo& dev);
 cudaError_t stream_prepare_device(const DeviceInfo& dev);
 cudaError_t q8_prepare_device(const DeviceInfo& dev);
+cudaError_t gmma_prepare_device(const DeviceInfo& dev);
 
 // Counts every kernel launch libq4 enqueues (host side).
 void count_launch();
@@ -136,5 +160,6 @@ void count_launch();
 cudaError_t gemv_device_flags(unsigned int* flags, bool clear);
 cudaError_t tc_device_flags(unsigned int* flags, bool clear);
 cudaError_t stream_device_flags(unsigned int* flags, bool clear);
+cudaError_t gmma_device_flags(unsigned int* flags, bool clear);
 
 }  // namespace q4
