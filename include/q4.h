@@ -246,6 +246,26 @@ Q4_API q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t
                                  q4_stream_t stream);
 
 /*
+ * q4_matmul_batch_noalloc -- q4_matmul_batch (same arguments, validation,
+ * kernels and results) whose group-sum kernel takes its workspace (arrival
+ * counters and fp32 partial sums of shared tiles) from a fixed 16 MiB device
+ * array inside libq4 instead of a stream-ordered allocation: the call makes
+ * no device allocation.  The pages describe no such entry point; it is an
+ * engineering variant of the batch call.
+ * Limits: the array is one per device and shared by every call of this entry
+ * point on it, so calls that may overlap in time (other streams, other host
+ * threads) race on it and must be serialized by the caller; calls in one
+ * stream are ordered and safe.  A call that would need more than the array
+ * holds (about 2 * SMs * 128 * 2 * M * 4 bytes per group-sum launch, plus
+ * counters) returns Q4_ERR_UNSUPPORTED before enqueuing anything.  The first
+ * call on a device looks up the array's address (cudaGetSymbolAddress); make
+ * it before capturing a stream.  Each call zeroes the counters with
+ * cudaMemsetAsync on `stream`.
+ */
+Q4_API q4_status q4_matmul_batch_noalloc(const q4_matmul_desc* descs, int count, int64_t M, int group,
+                                         q4_stream_t stream);
+
+/*
  * The 8-bit variant: the same affine rule with 255 levels and one byte per
  * code.  The pages compare a "standard 8-bit conversion" of the model with
  * the 4-bit builds (TWX4 comparison page, opening section) and ship an INT8

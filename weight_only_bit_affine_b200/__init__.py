@@ -54,6 +54,7 @@ __all__ = [
     "q4_check_device",
     "q4_debug_launch_count",
     "q4_debug_disable_kernels",
+    "q4_matmul_batch_noalloc",
     "KERNEL_GROUP_SUM",
     "KERNEL_WEIGHT_STREAM",
     "KERNEL_TILES",
@@ -83,6 +84,7 @@ SIGNATURES = {
     "q4_matmul_residual": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P, _P]),
     "q4_matmul_swiglu": (_INT, [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I64, _INT, _P, _P]),
     "q4_matmul_batch": (_INT, [_P, _INT, _I64, _INT, _P]),
+    "q4_matmul_batch_noalloc": (_INT, [_P, _INT, _I64, _INT, _P]),
     "q8_quantize": (_INT, [_P, _I64, _I64, _INT, _P, _P, _P, _P]),
     "q8_dequantize": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),
     "q8_matmul": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P]),
@@ -321,6 +323,19 @@ def q4_matmul_batch(problems, group: int = GROUP):
     if batch is None:
         return []
     batch.run()
+    return batch.outputs
+
+
+def q4_matmul_batch_noalloc(problems, group: int = GROUP):
+    """q4_matmul_batch through the entry point that makes no device
+    allocation (its group-sum workspace is a fixed array in libq4, shared by
+    all such calls on a device: serialize calls that may overlap)."""
+    batch = q4_prepare_batch(problems, group)
+    if batch is None:
+        return []
+    with torch.cuda.device(batch.device):
+        _check(lib().q4_matmul_batch_noalloc(ctypes.cast(batch._descs, ctypes.c_void_p), batch._count, batch._M,
+                                             batch._group, _stream(batch.device)))
     return batch.outputs
 
 

@@ -28,6 +28,29 @@ q4_status fail(q4_status st, const char* fmt, ...) {
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<unsigned int> g_disabled_kernels{0};  // q4_debug_disable_kernels
 
+// Scratch for q4_matmul_batch_noalloc: the group-sum kernel's workspace
+// (arrival counters, then fp32 partial sums) in a fixed device array instead
+// of a stream-ordered allocation.  One array per device, shared by every
+// such call on it.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[64] = {};  // per device ordinal, from cudaGetSymbolAddress (once per device)
+
+// The scratch array's device address on the current device (dev.device).
+cudaError_t noalloc_scratch(const DeviceInfo& dev, unsigned char** out) {
+  if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev.device] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev.device] = p;
+  }
+  *out = static_cast<unsigned char*>(g_scratch_addr[dev.device]);
+  return cudaSuccess;
+}
+
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
 std::atomic<bool> g_device_ready[kMaxDevices];
@@ -117,7 +140,7 @@ q4_status check_epilogue(const char* who, int32_t epi, int32_t reserved, const u
 // Every host-side step that can fail for a valid call (tensor-map encoding,
 // configuration checks) runs before the first launch.
 q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& dev, cudaStream_t cs,
-                       const char* what) {
+                       const char* what, bool static_scratch = false) {
   std::vector<MatmulArgs> gemv, streamed, grouped;
   thread_local std::vector<TcLaunch> tc;
   thread_local std::vector<GmmaPlan> gm;
@@ -151,7 +174,14 @@ q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& de
       pbytes += g.partial_bytes;
     }
     unsigned char* ws = nullptr;
-    if (cbytes + pbytes > 0) {
+    if (cbytes + pbytes > 0 && static_scratch) {
+      if (cbytes + pbytes > kNoAllocScratchBytes)
+        return fail(Q4_ERR_UNSUPPORTED, "%s: the call needs %zu bytes of scratch, the fixed array holds %zu", what,
+                    cbytes + pbytes, kNoAllocScratchBytes);
+      cudaError_t e = noalloc_scratch(dev, &ws);
+      if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, cbytes, cs);
+      if (e != cudaSuccess) return from_cuda(e, what);
+    } else if (cbytes + pbytes > 0) {
       cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), cbytes + pbytes, cs);
       if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, cbytes, cs);
       if (e != cudaSuccess) return from_cuda(e, what);
@@ -164,7 +194,7 @@ q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& de
       po += g.partial_bytes;
       if ((st = from_cuda(launch_planned_gmma(g, counters, partials, cs), what)) != Q4_OK) break;
     }
-    if (ws != nullptr) {
+    if (ws != nullptr && !static_scratch) {
       const cudaError_t e = cudaFreeAsync(ws, cs);
       if (st == Q4_OK && e != cudaSuccess) st = from_cuda(e, what);
     }
@@ -346,6 +376,32 @@ q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int
   q4_status st;
   if ((st = check_device(&dev)) != Q4_OK) return st;
   return run_problems(list, *dev, reinterpret_cast<cudaStream_t>(stream), "q4_matmul_batch launch");
+}
+
+q4_status q4_matmul_batch_noalloc(const q4_matmul_desc* descs, int count, int64_t M, int group,
+                                  q4_stream_t stream) {
+  if (count < 0) return fail(Q4_ERR_SHAPE, "q4_matmul_batch_noalloc: negative count %d", count);
+  if (count == 0) return Q4_OK;
+  if (!descs) return fail(Q4_ERR_NULL, "q4_matmul_batch_noalloc: NULL descriptor array");
+  std::vector<MatmulArgs> list;
+  list.reserve(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    const q4_matmul_desc& d = descs[i];
+    bool empty = false;
+    char who[56];
+    snprintf(who, sizeof who, "q4_matmul_batch_noalloc[%d]", i);
+    q4_status st = check_matmul(who, d.x, M, d.K, d.codes, d.scales, d.biases, d.N, group, d.y, &empty);
+    if (st != Q4_OK) return st;
+    MatmulArgs a{d.x, d.codes, d.scales, d.biases, d.y, M, d.N, d.K};
+    if ((st = check_epilogue(who, d.epilogue, d.reserved, d.r, d.up_codes, d.up_scales, d.up_biases, &a)) != Q4_OK)
+      return st;
+    if (!empty) list.push_back(a);
+  }
+  if (list.empty()) return Q4_OK;
+  const DeviceInfo* dev = nullptr;
+  q4_status st;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  return run_problems(list, *dev, reinterpret_cast<cudaStream_t>(stream), "q4_matmul_batch_noalloc launch", true);
 }
 
 // ---- the 8-bit variant (q8.cu) --------------------------------------------
