@@ -251,6 +251,7 @@ GMMA_PATH = ("gmma_kernel: tcgen05 group sums of (128 + q) * x in tensor memory,
 # in between where the kernel choice changes (weight streaming up to 8 rows,
 # tensor-core tiles from 9, one 16-row tile up to 16).
 BATCHED_ROWS = (4, 8, 12, 16, 64, 256)
+STREAM_BATCH_ROWS = (4, 8, 16)
 
 
 def workload_rows(dev, packed, x, x_down, bf16_peak):
@@ -452,6 +453,23 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
                      GMMA_PATH
                      if M >= 3 else "gemv_kernel: CUDA cores"),
         }
+
+    # the whole step (225 projections) as ONE batch for several concurrent
+    # conversations: the group-sum kernel's steady state (one launch's ramp-up
+    # and tail over 4.19 GB instead of over one layer's 128 MB)
+    sbytes = stream_bytes(packed)
+    for M in STREAM_BATCH_ROWS:
+        xs = workloads.activation(M, 4096, seed, 300 + M, device=dev)
+        xsd = workloads.activation(M, 11264, seed, 400 + M, device=dev)
+        yss = y_for(M, packed)
+        probs = [(xsd if p.K == 11264 else xs, c, s_, b, y) for (p, c, s_, b), y in zip(packed, yss)]
+        t = _graph_ms(dev, lambda probs=probs: q4.q4_matmul_batch(probs), 5)
+        rows[f"stream_batch_M{M}"] = {
+            "ms_per_step": round(t, 4), "packed_GBps": round(sbytes / (t * 1e-3) / 1e9, 1),
+            "tokens_per_s": round(M / (t * 1e-3), 1), "path": GMMA_PATH,
+            "note": f"the 225 projections of a decode step for {M} conversations as one q4_matmul_batch call",
+        }
+        del yss, probs
     return rows
 
 
@@ -540,7 +558,9 @@ class OracleSample:
 #   layer_m1       one temporal layer (7 projections) at M = 1 as one
 #                  q4_matmul_batch.
 #   layer_m4       one temporal layer (7 projections) at M = 4 as one
-#                  q4_matmul_batch: the tensor-core weight-streaming kernel.
+#                  q4_matmul_batch: the group-sum tensor-core kernel.
+#   layer_m4_weight_stream  the same with the group-sum kernel kept out of the
+#                  dispatch: the tensor-core weight-streaming kernel.
 #   layer_m8       the same at M = 8.
 #   fused_layer    one temporal layer at M = 1 with its epilogues fused (o and
 #                  down + residual, gate/up as one SwiGLU problem), one
@@ -674,10 +694,30 @@ def _tc_gate(dev):
     return run
 
 
+def _pinned(case, mask):
+    """A profile case run with kernel families kept out of the dispatch."""
+    import weight_only_bit_affine_b200 as q4
+
+    def make(dev):
+        run = case(dev)
+
+        def pinned():
+            prev = q4.q4_debug_disable_kernels(mask)
+            try:
+                run()
+            finally:
+                q4.q4_debug_disable_kernels(prev)
+
+        return pinned
+
+    return make
+
+
 PROFILE_CASES = {"stream_small": _stream_small, "tc_layer": _tc_layer, "tc_gate": _tc_gate,
                  "depformer_step": _depformer_step, "layer_m1": lambda dev: _layer_rows(dev, 1),
                  "layer_m4": lambda dev: _layer_rows(dev, 4),
-                 "layer_m8": lambda dev: _layer_rows(dev, 8), "fused_layer": _fused_layer, "q8_layer": _q8_layer}
+                 "layer_m8": lambda dev: _layer_rows(dev, 8), "fused_layer": _fused_layer, "q8_layer": _q8_layer,
+                 "layer_m4_weight_stream": _pinned(lambda dev: _layer_rows(dev, 4), 1)}
 
 
 def run_profile_case(name: str, reps: int):

@@ -58,15 +58,15 @@ def test_noalloc_equals_batch_on_two_consecutive_calls(M):
 
 
 def test_noalloc_refuses_a_call_larger_than_its_scratch():
-    """Five launches at M = 16 (eight distinct activation tensors per launch)
-    with shared tiles need more than the fixed array: Q4_ERR_UNSUPPORTED, and
-    no output is written."""
-    M, K = 16, 1024
+    """Five launches at M = 16 (eight distinct activation tensors per launch),
+    each spread over every SM with shared tiles, need more than the fixed
+    array: Q4_ERR_UNSUPPORTED, and no output is written."""
+    M, K, N = 16, 1024, 384
     probs = []
     for t in range(40):
         x = workloads.activation(M, K, 90, t, device=DEV)
-        gate, up = _packed(128, K, 90, 2 * t), _packed(128, K, 90, 2 * t + 1)
-        probs.append((x, *gate, torch.full((M, 128), float("nan"), dtype=torch.bfloat16, device=DEV), q4.SwiGLU(*up)))
+        gate, up = _packed(N, K, 90, 2 * t), _packed(N, K, 90, 2 * t + 1)
+        probs.append((x, *gate, torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV), q4.SwiGLU(*up)))
     with pytest.raises(q4.Q4Error) as err:
         q4.q4_matmul_batch_noalloc(probs)
     assert err.value.status == 4  # Q4_ERR_UNSUPPORTED
