@@ -105,6 +105,28 @@ def test_stream_mixed_batch_one_launch(M):
         check_matmul(x, c, s, b, out, rows=sample_rows(N, 48, seed=N + K), what=f"batch {N}x{K} M={M}")
 
 
+def test_stream_mixed_batch_repeated():
+    """The mixed launch above, 150 times over: the chunk count per tile
+    changes between its problems, so an A slot's consecutive uses go to
+    different MMA issuers; every repetition must equal the single calls
+    (with one A-full barrier per slot shared by both issuers, a few percent
+    of repetitions read a chunk before it was written)."""
+    M = 3
+    shapes = [(4096, 4096), (130, 11264), (77, 1024), (1, 256), (2000, 2816), (9, 12288), (333, 4096), (4, 768)]
+    probs, singles = [], []
+    for t, (N, K) in enumerate(shapes):
+        c, s, b = _packed(N, K, 53, t)
+        x = workloads.activation(M, K, 53, 200 + t, device=DEV)
+        probs.append((x, c, s, b, torch.empty((M, N), dtype=torch.bfloat16, device=DEV)))
+        singles.append(q4.q4_matmul(x, c, s, b))
+    for rep in range(150):
+        for p in probs:
+            p[4].fill_(float("nan"))
+        q4.q4_matmul_batch(probs)
+        for (x, c, s, b, out), ref, (N, K) in zip(probs, singles, shapes):
+            assert torch.equal(out, ref), (rep, N, K)
+
+
 def test_stream_large_problem_sampled():
     """The text head shape (32000 x 4096) and a gate projection, every CTA busy."""
     for (N, K) in [(32000, 4096), (11264, 4096), (4096, 11264)]:

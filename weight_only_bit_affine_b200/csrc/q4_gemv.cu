@@ -232,6 +232,9 @@ struct GemvProblem {
   int32_t K, epi;
 };
 
+// CTAs per launch at most (one per SM).
+constexpr int kMaxCtas = 256;
+
 template <int NP>
 struct GemvLaunch {
   int count;
@@ -239,6 +242,13 @@ struct GemvLaunch {
   int stages;
   uint32_t stage_bytes;  // >= every problem's tile and activation block, 128-byte multiple
   int64_t total_bytes;   // packed bytes of the whole list
+  // first[c]: the first problem that ends after CTA c's first byte.  Every
+  // role of the CTA starts its walk over the list there: the problems before
+  // it hold none of its rows, and reading their descriptors (a constant-cache
+  // miss each, ~0.4 us) delayed the last CTAs of a 225-problem launch enough
+  // to cost the whole launch 5 %.  A launch of at most kFewProblems problems
+  // walks from the first.
+  uint16_t first[NP > kFewProblems ? kMaxCtas : 1];
   GemvProblem prob[NP];
 };
 
@@ -368,6 +378,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   // This CTA's share of the list: a contiguous, balanced range of packed bytes.
   const int64_t lo = static_cast<int64_t>(blockIdx.x) * L.total_bytes / gridDim.x;
   const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * L.total_bytes / gridDim.x;
+  const int p0 = NP > kFewProblems ? L.first[blockIdx.x] : 0;
 
   if (warp == consumer_warps) {
     // ---------------- producer warp ----------------
@@ -375,7 +386,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       {  // warm L2 with the first tiles of the range (a hint; changes no value)
         int64_t r0, r1;
         int issued = 0;
-        for (int pi = 0; pi < L.count && issued < L.stages; ++pi) {
+        for (int pi = p0; pi < L.count && issued < L.stages; ++pi) {
           if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
           const GemvProblem& P = L.prob[pi];
           const Geometry geo = geometry_of(P.K, L.consumer_threads);
@@ -399,7 +410,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool dead = false;
-      for (int pi = 0; pi < L.count && !dead; ++pi) {
+      for (int pi = p0; pi < L.count && !dead; ++pi) {
         int64_t r0, r1;
         if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
         if (r0 >= r1) continue;
@@ -456,7 +467,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     int slot = 0;
     uint32_t sph = 0;
     bool dead = false;
-    for (int pi = 0; pi < L.count; ++pi) {
+    for (int pi = p0; pi < L.count; ++pi) {
       int64_t r0, r1;
       if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
       const GemvProblem& P = L.prob[pi];
@@ -497,7 +508,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   int stage = 0, slot = 0;
   uint32_t phase = 0, sph = 0;
   bool dead = false;
-  for (int pi = 0; pi < L.count; ++pi) {
+  for (int pi = p0; pi < L.count; ++pi) {
     int64_t r_begin, r_end;
     if (!segment_of<EPI>(L, pi, lo, hi, &r_begin, &r_end)) break;
     if (r_begin >= r_end) continue;
@@ -859,7 +870,16 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   L.total_bytes = total;
   // Enough CTAs that every one has work; one per SM.
   const int64_t rows = [&] { int64_t r = 0; for (int i = 0; i < count; ++i) r += probs[i].N; return r; }();
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, rows)));
+  const int grid = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>(std::min(dev.sm_count, kMaxCtas), rows)));
+  // each CTA's first problem: the first that ends after the CTA's first byte
+  // (the kernel's byte range formula)
+  int pi = 0;
+  for (int c = 0; c < grid && NP > kFewProblems; ++c) {
+    const int64_t lo = static_cast<int64_t>(c) * total / grid;
+    while (pi < count && L.prob[pi].byte_begin + L.prob[pi].N * problem_row_bytes(L.prob[pi]) <= lo) ++pi;
+    L.first[c] = static_cast<uint16_t>(pi);
+  }
   bool epi = false;
   for (int i = 0; i < count; ++i) epi = epi || probs[i].epi != kEpiNone || is_fused(probs[i]);
   auto kern = epi ? gemv_kernel<MR, kThreads, NP, true> : gemv_kernel<MR, kThreads, NP, false>;

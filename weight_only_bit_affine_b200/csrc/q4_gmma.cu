@@ -88,6 +88,8 @@ constexpr int kSbPrefetch = kSbSlots - 1;
 constexpr int kSbBytes = kSbSlots * 2 * kRows * 16;  // 16 KB
 constexpr int kMaxXMaps = 8;
 constexpr int kMaxEntries = 160;
+constexpr int kMaxCtas = 256;  // CTAs per launch at most (one per SM)
+static_assert(kMaxEntries <= 255, "entry indices fit a byte");
 constexpr float kNaN = __builtin_nanf("");
 // Sleep between polls of a barrier (ns), per role: the producer runs far
 // ahead and waits long; the issuers are on the critical path.
@@ -138,6 +140,12 @@ struct GmmaLaunch {
   unsigned int* counters;
   int64_t total_steps;
   int32_t count, M, stages, x_floats;  // x_floats: group-sum area (largest K / 32) x MC, rounded up to 4
+  // first[c]: the first entry (a SwiGLU pair's gate entry) whose tiles end
+  // after CTA c's first step.  Every role of the CTA walks the entries from
+  // there and stops at the first that starts at or after its last step, so
+  // it reads only the descriptors of its own tiles (each read of another
+  // entry's is a constant-cache miss).
+  uint8_t first[kMaxCtas];
 };
 static_assert(sizeof(GmmaLaunch) <= 32764, "kernel parameter space");
 static_assert(sizeof(GmmaLaunch) <= kGmmaParamBytes, "plan storage");
@@ -275,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) gmma_kernel(const __grid_constant
     bool dead = false;
     int s = 0;
     uint32_t ph = 0;
-    for (int p = 0; p < L.count; p += L.e[p].fused ? 2 : 1) {
+    for (int p = L.first[blockIdx.x]; p < L.count && L.e[p].step_begin < hi; p += L.e[p].fused ? 2 : 1) {
       const GmmaEntry& E = L.e[p];
       int64_t j0, j1;
       tile_range(E, lo, hi, j0, j1);
@@ -315,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) gmma_kernel(const __grid_constant
     int s = me % L.stages, aslot = me % kASlots, dslot = me % kDSlots;
     uint32_t aph = (me / kASlots) & 1u, dph = (me / kDSlots) & 1u;
     int t = me;  // step within the current segment; carried over segment ends
-    for (int p = 0; p < L.count; p += L.e[p].fused ? 2 : 1) {
+    for (int p = L.first[blockIdx.x]; p < L.count && L.e[p].step_begin < hi; p += L.e[p].fused ? 2 : 1) {
       const GmmaEntry& E = L.e[p];
       int64_t j0, j1;
       tile_range(E, lo, hi, j0, j1);
@@ -370,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) gmma_kernel(const __grid_constant
     int s = grp % L.stages, slot = grp % kASlots;
     uint32_t ph = (grp / L.stages) & 1u, sph = (grp / kASlots) & 1u;
     int t = grp;  // step within the current segment; carried over segment ends
-    for (int p = 0; p < L.count; p += L.e[p].fused ? 2 : 1) {
+    for (int p = L.first[blockIdx.x]; p < L.count && L.e[p].step_begin < hi; p += L.e[p].fused ? 2 : 1) {
       const GmmaEntry& E = L.e[p];
       int64_t j0, j1;
       tile_range(E, lo, hi, j0, j1);
@@ -413,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) gmma_kernel(const __grid_constant
     bool dead = false;
     int slot = 0;
     uint32_t sph = 0;
-    for (int p = 0; p < L.count; p += L.e[p].fused ? 2 : 1) {
+    for (int p = L.first[blockIdx.x]; p < L.count && L.e[p].step_begin < hi; p += L.e[p].fused ? 2 : 1) {
       const GmmaEntry& E = L.e[p];
       int64_t j0, j1;
       tile_range(E, lo, hi, j0, j1);
@@ -729,8 +737,19 @@ cudaError_t plan_gmma(const MatmulArgs* list, int count, const DeviceInfo& dev, 
     L.total_steps = total;
     // every SM takes an equal share of the steps (one CTA per SM: each
     // allocates all 512 tensor-memory columns)
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, total));
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(std::min(dev.sm_count, kMaxCtas), total));
     pl.grid = static_cast<int>(grid);
+    // each CTA's first entry: the first whose tiles end after the CTA's first
+    // step (the kernel's cta_first_step formula)
+    for (int64_t c = 0, p = 0; c < grid; ++c) {
+      const int64_t lo = total * c / grid;
+      auto end_of = [&](int64_t q) {
+        const GmmaEntry& E = L.e[q];
+        return E.step_begin + (E.N + kRows - 1) / kRows * (E.K / kStepK) * (E.fused ? 2 : 1);
+      };
+      while (p < ne && end_of(p) <= lo) p += L.e[p].fused ? 2 : 1;
+      L.first[c] = static_cast<uint8_t>(p);
+    }
     pl.smem = dev.smem_optin;
     pl.kern = kernel_of(rows_class(M), epi);
     // Is a tile shared by two CTAs (a CTA boundary inside a tile)?

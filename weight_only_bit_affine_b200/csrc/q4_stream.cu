@@ -101,6 +101,7 @@ constexpr int kMaxASlots = 8;   // A ring in tensor memory: up to 8 chunks of 64
 constexpr int kMaxStages = 12;
 constexpr int kMaxProblems = 256;
 constexpr int kFewProblems = 4;
+constexpr int kMaxCtas = 256;  // CTAs per launch at most (one per SM)
 constexpr float kNaN = __builtin_nanf("");
 
 struct StreamProblem {
@@ -126,6 +127,12 @@ struct StreamLaunch {
   int32_t count, M, stages, a_slots;  // a_slots: A ring chunks (a multiple of kGroups)
   uint32_t stage_bytes, b_bytes, a_col0, pad_;  // a_col0: first A ring column (after the accumulators)
   int64_t total_bytes;
+  // first[c]: the first problem with a tile of CTA c (launches of more than
+  // kFewProblems problems).  Every role walks the list from there and stops
+  // at the first problem that starts at or after the CTA's last byte, so it
+  // reads only its own problems' descriptors (each read of another problem's
+  // is a constant-cache miss).
+  uint16_t first[NP > kFewProblems ? kMaxCtas : 1];
   StreamProblem prob[NP];
 };
 
@@ -218,8 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
   uint8_t* ring = smem + L.b_bytes;   // stages x stage_bytes
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + static_cast<size_t>(L.stages) * L.stage_bytes);
   uint64_t* empty = full + kMaxStages;
-  uint64_t* afull = empty + kMaxStages;
-  uint64_t* aempty = afull + kMaxASlots;
+  // A chunk written: one set per issuer (chunk c of a tile goes to issuer
+  // c % issuers).  With a single set, consecutive uses of a slot could belong
+  // to different issuers (the chunk count per tile varies over a launch's
+  // problems), and an issuer one use ahead would see the parity of the use
+  // before the one it waits for still in progress as "complete".  Per issuer,
+  // its own uses of a slot complete in order and at most one ahead of it.
+  uint64_t* afull = empty + kMaxStages;                // [kMaxIssuers][kMaxASlots]
+  uint64_t* aempty = afull + kMaxIssuers * kMaxASlots;
   uint64_t* dfull = aempty + kMaxASlots;
   uint64_t* dempty = dfull + 2;
   uint64_t* bfull = dempty + 2;
@@ -233,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
       mbar_init(&empty[s], 4 * kGroups);
     }
     for (int a = 0; a < L.a_slots; ++a) {
-      mbar_init(&afull[a], 4);
+      for (int i = 0; i < kMaxIssuers; ++i) mbar_init(&afull[i * kMaxASlots + a], 4);
       mbar_init(&aempty[a], 1);
     }
     for (int d = 0; d < 2; ++d) {
@@ -256,11 +269,12 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
   const int64_t G = gridDim.x;
   const int64_t lo = L.total_bytes * static_cast<int64_t>(blockIdx.x) / G;
   const int64_t hi = L.total_bytes * (static_cast<int64_t>(blockIdx.x) + 1) / G;
+  const int p0 = NP > kFewProblems ? L.first[blockIdx.x] : 0;
 
   pdl_launch_dependents();
   if (warp == 0 && lane == 0) {
     // Before the wait: pull the first tile's codes toward L2 (a hint only).
-    for (int p = 0; p < L.count; ++p) {
+    for (int p = p0; p < L.count && L.prob[p].byte_begin < hi; ++p) {
       const StreamProblem& P = L.prob[p];
       int64_t j0, j1;
       tile_range(P, lo, hi, j0, j1);
@@ -279,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     bool dead = false;
     int s = 0;
     uint32_t ph = 0;
-    for (int p = 0; p < L.count; ++p) {
+    for (int p = p0; p < L.count && L.prob[p].byte_begin < hi; ++p) {
       const StreamProblem& P = L.prob[p];
       int64_t v0, v1;
       int sh;
@@ -313,11 +327,11 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
       bool dead = false;
       int lp = 0;
       int slot0 = 0;      // A ring slot of the current tile's first chunk
-      uint32_t ph0 = 0;   // and its phase
       int64_t gt = 0;
+      uint32_t aph = 0;  // bit a: parity of this issuer's next use of A slot a
       const uint64_t bdesc0 = sw128_desc(smem_u32(bmat));
       const uint32_t a_base = tmem + a_col0;
-      for (int p = 0; p < L.count; ++p) {
+      for (int p = p0; p < L.count && L.prob[p].byte_begin < hi; ++p) {
         const StreamProblem& P = L.prob[p];
         int64_t v0, v1;
         int sh;
@@ -341,10 +355,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
           tc_fence_after();
           if (active) {
             for (int c = me; c < S.chunks; c += S.issuers) {
-              int slot = slot0 + c;  // ring slot and phase of chunk c
-              uint32_t sph = ph0;
-              while (slot >= A) { slot -= A; sph ^= 1u; }
-              if (!dead && !mbar_wait<kSleepWaits>(&afull[slot], sph)) dead = true;
+              int slot = slot0 + c;  // ring slot of chunk c
+              while (slot >= A) slot -= A;
+              if (!dead && !mbar_wait<kSleepWaits>(&afull[me * kMaxASlots + slot], (aph >> slot) & 1u)) dead = true;
+              aph ^= 1u << slot;
               tc_fence_after();
               const uint32_t at = a_base + static_cast<uint32_t>(slot) * kChunkCols;
               const uint64_t bd = bdesc0 + static_cast<uint64_t>(c) * atom16;
@@ -372,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
           if (leader) tc_commit(&dfull[db]);
           __syncwarp();
           slot0 += S.chunks;
-          while (slot0 >= A) { slot0 -= A; ph0 ^= 1u; }
+          while (slot0 >= A) slot0 -= A;
         }
         ++lp;
       }
@@ -389,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     int gmod = 0;             // chunks of this CTA before the current tile, mod kGroups
     int slot0 = 0;            // A ring slot of the current tile's first chunk
     uint32_t ph0 = 0;         // and its phase
-    for (int p = 0; p < L.count; ++p) {
+    for (int p = p0; p < L.count && L.prob[p].byte_begin < hi; ++p) {
       const StreamProblem& P = L.prob[p];
       int64_t v0, v1;
       int sh;
@@ -437,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[slot]);
+          if (lane == 0) mbar_arrive(&afull[(c % S.issuers) * kMaxASlots + slot]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);  // this warp's reads of the stage are done
@@ -455,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     bool dead = false;
     int lp = 0;
     int64_t gt = 0;
-    for (int p = 0; p < L.count; ++p) {
+    for (int p = p0; p < L.count && L.prob[p].byte_begin < hi; ++p) {
       const StreamProblem& P = L.prob[p];
       int64_t v0, v1;
       int sh;
@@ -595,7 +609,7 @@ Plan plan_of(const MatmulArgs& a) {
   return pl;
 }
 
-constexpr size_t kFixedSmem = 1024 /* alignment */ + 8 * (2 * kMaxStages + 2 * kMaxASlots + 6) + 16;
+constexpr size_t kFixedSmem = 1024 /* alignment */ + 8 * (2 * kMaxStages + (kMaxIssuers + 1) * kMaxASlots + 6) + 16;
 
 uint32_t acc_cols_of(uint32_t nb) {
   const uint32_t issuers = nb <= 32 ? 2u : 1u;  // as ProblemShape
@@ -656,7 +670,17 @@ cudaError_t run_stream(const MatmulArgs* list, int count, const DeviceInfo& dev,
   // All of the SM's shared memory: one CTA per SM (each allocates all 512
   // tensor-memory columns).
   const size_t smem = dev.smem_optin;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dev.sm_count, tiles)));
+  const int grid =
+      static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(std::min(dev.sm_count, kMaxCtas), tiles)));
+  // each CTA's first problem: the first whose tiles end after the CTA's first
+  // byte (the kernel's byte range formula)
+  for (int64_t c = 0, i = 0; c < grid && NP > kFewProblems; ++c) {
+    const int64_t lo = total * c / grid;
+    while (i < count && L.prob[i].byte_begin + (L.prob[i].N + kLanes / L.prob[i].segs - 1) /
+                                                   (kLanes / L.prob[i].segs) * L.prob[i].tile_bytes <= lo)
+      ++i;
+    L.first[c] = static_cast<uint16_t>(i);
+  }
   bool epi = false;
   for (int i = 0; i < count; ++i) epi = epi || list[i].epi != kEpiNone || list[i].fused();
   cudaLaunchConfig_t cfg = {};
