@@ -352,12 +352,29 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
     chain()
     chain_launches = q4.q4_debug_launch_count() - n0
     ms_chain = _graph_ms(dev, chain, 20)
+    # The same stages as one q4_matmul_chain call: one persistent launch in
+    # which every CTA takes a share of each stage in turn.
+    stages = []
+    for P in layers_w:
+        stages.append([(h, *P["q"], qkv[0]), (h, *P["k"], qkv[1]), (h, *P["v"], qkv[2])])
+        stages.append([(qkv[2], *P["o"], h, q4.Residual(h))])
+        stages.append([(h, *P["gate"], act, q4.SwiGLU(*P["up"]))])
+        stages.append([(act, *P["down"], h, q4.Residual(h))])
+    stages.append([(h, *packed[-1][1:], logits)])
+    prepared = q4.q4_prepare_chain(stages)
+    n0 = q4.q4_debug_launch_count()
+    prepared.run()
+    one_launches = q4.q4_debug_launch_count() - n0
+    ms_one = _graph_ms(dev, prepared.run, 20)
     rows["decode_chain_M1"] = {
         "ms_per_step": round(ms_chain, 4), "GBps": round(STREAM_BYTES / (ms_chain * 1e-3) / 1e9, 1),
         "launches_per_step": int(chain_launches), "bytes": STREAM_BYTES,
-        "note": "dependent launches per layer: q/k/v batch -> o + residual -> SwiGLU(gate, up) -> down + residual; "
-                "32 layers + head in one CUDA graph; compare stream_ms_batch_graph (one launch over independent "
-                "problems with x reused)",
+        "one_call_ms_per_step": round(ms_one, 4), "one_call_GBps": round(STREAM_BYTES / (ms_one * 1e-3) / 1e9, 1),
+        "one_call_launches_per_step": int(one_launches), "stages": len(stages),
+        "note": "dependent stages per layer: q/k/v batch -> o + residual -> SwiGLU(gate, up) -> down + residual; "
+                "32 layers + head; 'ms_per_step': one launch per stage in one CUDA graph; 'one_call': the same "
+                "stages as one q4_matmul_chain call (a persistent launch, grid-wide barrier between stages), "
+                "graph-replayed; compare stream_ms_batch_graph (one launch over independent problems with x reused)",
     }
 
     # the 8-bit variant of the same layer (9 bits per weight), one q8_matmul per

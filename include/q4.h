@@ -266,6 +266,35 @@ Q4_API q4_status q4_matmul_batch_noalloc(const q4_matmul_desc* descs, int count,
                                          q4_stream_t stream);
 
 /*
+ * q4_matmul_chain -- dependent matmuls: stage s is the next stage_counts[s]
+ * descriptors of `descs` (n_stages entries summing to count), and the call
+ * computes exactly (bit for bit) what q4_matmul_batch on each stage in turn
+ * on `stream` computes.  A stage may read, as x or as a residual operand,
+ * what earlier stages write; within a stage the batch rules hold.  This is
+ * the shape of a decode step (per layer: q, k, v on the layer input; the
+ * attention output adding into the residual stream; gate and up as SwiGLU;
+ * down adding into the stream), whose per-step dispatches the Swift/MLX blog
+ * ("Performance optimizations") and the ONNX README (CUDA Graph capture)
+ * fuse; the pages describe no such entry point, this is an engineering
+ * variant of the batch call for a dependent sequence.
+ * With one or two activation rows and every problem on the bulk-copy GEMV
+ * (K a multiple of 256, 16-byte aligned scale rows), the chain runs as one
+ * persistent cooperative launch per up to 256 stages and 256 problems: one
+ * CTA per SM takes a share of every stage in turn, streaming the next
+ * stages' weights while it waits for the CTAs still finishing a stage (a
+ * grid-wide arrival counter per stage, every wait bounded: a wait that gives
+ * up raises the q4_device_status flag and the outputs it covers are NaN).
+ * It takes a stream-ordered workspace of 4 bytes per stage
+ * (cudaMallocAsync, cudaMemsetAsync, cudaFreeAsync on `stream`).  Otherwise
+ * each stage is one q4_matmul_batch.  `descs` and `stage_counts` are HOST
+ * arrays read before the call returns.  Validation covers every descriptor
+ * before anything is enqueued; counts that do not add up, or a negative
+ * count, are Q4_ERR_SHAPE.
+ */
+Q4_API q4_status q4_matmul_chain(const q4_matmul_desc* descs, int count, const int* stage_counts, int n_stages,
+                                 int64_t M, int group, q4_stream_t stream);
+
+/*
  * The 8-bit variant: the same affine rule with 255 levels and one byte per
  * code.  The pages compare a "standard 8-bit conversion" of the model with
  * the 4-bit builds (TWX4 comparison page, opening section) and ship an INT8

@@ -163,6 +163,26 @@ def test_batch_validates_every_entry_before_the_device():
         assert lib.q4_matmul_batch(ctypes.cast(arr, ctypes.c_void_p), 2, 1, 32, None) == CUDA
 
 
+def test_chain_validation_precedes_the_device(lib):
+    """q4_matmul_chain: stage counts that do not add up to count, a negative
+    stage count, a missing stage array and a bad descriptor in the last stage
+    are reported before any device work."""
+    good = q4.MatmulDesc(P, P, P, P, P, 8, 64)
+    bad = q4.MatmulDesc(P, P, P, P, P + 128, 8, 64)
+    bad.epilogue = 9
+    arr = (q4.MatmulDesc * 3)(good, good, bad)
+    vp = lambda a: ctypes.cast(a, ctypes.c_void_p)
+    counts = (ctypes.c_int * 2)(1, 1)
+    assert lib.q4_matmul_chain(vp(arr), 3, vp(counts), 2, 1, 32, None) == SHAPE
+    neg = (ctypes.c_int * 2)(4, -1)
+    assert lib.q4_matmul_chain(vp(arr), 3, vp(neg), 2, 1, 32, None) == SHAPE
+    assert lib.q4_matmul_chain(vp(arr), 3, None, 2, 1, 32, None) == NULL
+    ok = (ctypes.c_int * 2)(2, 1)
+    assert lib.q4_matmul_chain(vp(arr), 3, vp(ok), 2, 1, 32, None) == UNSUP
+    assert b"q4_matmul_chain[2] (stage 1)" in lib.q4_last_error()
+    assert lib.q4_matmul_chain(vp(arr), 0, None, 0, 1, 32, None) == 0
+
+
 def test_descriptor_layout_matches_c(tmp_path):
     src = tmp_path / "l.c"
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "q4.h"\n'

@@ -55,6 +55,9 @@ __all__ = [
     "q4_debug_launch_count",
     "q4_debug_disable_kernels",
     "q4_matmul_batch_noalloc",
+    "q4_matmul_chain",
+    "q4_prepare_chain",
+    "PreparedChain",
     "KERNEL_GROUP_SUM",
     "KERNEL_WEIGHT_STREAM",
     "KERNEL_TILES",
@@ -85,6 +88,7 @@ SIGNATURES = {
     "q4_matmul_swiglu": (_INT, [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I64, _INT, _P, _P]),
     "q4_matmul_batch": (_INT, [_P, _INT, _I64, _INT, _P]),
     "q4_matmul_batch_noalloc": (_INT, [_P, _INT, _I64, _INT, _P]),
+    "q4_matmul_chain": (_INT, [_P, _INT, _P, _INT, _I64, _INT, _P]),
     "q8_quantize": (_INT, [_P, _I64, _I64, _INT, _P, _P, _P, _P]),
     "q8_dequantize": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),
     "q8_matmul": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P]),
@@ -396,6 +400,48 @@ def q4_prepare_batch(problems, group: int = GROUP) -> Optional[PreparedBatch]:
             raise TypeError(f"problem {i}: epilogue must be Residual or SwiGLU")
         descs[i] = d
     return PreparedBatch(descs, len(problems), M, group, dev, [p[4] for p in problems])
+
+
+def q4_matmul_chain(stages, group: int = GROUP):
+    """Dependent matmuls in order: `stages` is a sequence of stages, each a
+    sequence of q4_matmul_batch problem tuples (every x with the same M);
+    a stage may read, as x or residual, what earlier stages write.  Computes
+    exactly what q4_matmul_batch on each stage in turn computes.  Returns the
+    outputs of all stages in order."""
+    chain = q4_prepare_chain(stages, group)
+    if chain is None:
+        return []
+    chain.run()
+    return chain.outputs
+
+
+class PreparedChain:
+    """A q4_matmul_chain call whose descriptor and stage arrays are built
+    once; run() calls the C entry point with them on the current stream of
+    the problems' device (the tensors must stay alive in between)."""
+
+    def __init__(self, batch: PreparedBatch, counts):
+        self._batch = batch
+        self._counts = (ctypes.c_int * len(counts))(*counts)
+        self._n = len(counts)
+        self.device, self.outputs = batch.device, batch.outputs
+
+    def run(self) -> None:
+        b = self._batch
+        with torch.cuda.device(b.device):
+            _check(lib().q4_matmul_chain(ctypes.cast(b._descs, ctypes.c_void_p), b._count,
+                                         ctypes.cast(self._counts, ctypes.c_void_p), self._n, b._M, b._group,
+                                         _stream(b.device)))
+
+
+def q4_prepare_chain(stages, group: int = GROUP) -> Optional[PreparedChain]:
+    """Validate and marshal a q4_matmul_chain call once; None if it has no
+    problem."""
+    stages = [list(st) for st in stages]
+    batch = q4_prepare_batch([p for st in stages for p in st], group)
+    if batch is None:
+        return None
+    return PreparedChain(batch, [len(st) for st in stages])
 
 
 # ------------------------------------------------------------------ 8-bit codes

@@ -353,6 +353,81 @@ q4_status q4_matmul_step(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* 
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+q4_status q4_matmul_chain(const q4_matmul_desc* descs, int count, const int* stage_counts, int n_stages, int64_t M,
+                          int group, q4_stream_t stream) {
+  if (count < 0 || n_stages < 0) return fail(Q4_ERR_SHAPE, "q4_matmul_chain: negative count or stage count");
+  if (count == 0) return Q4_OK;
+  if (!descs || !stage_counts) return fail(Q4_ERR_NULL, "q4_matmul_chain: NULL descriptor or stage array");
+  int64_t sum = 0;
+  for (int s = 0; s < n_stages; ++s) {
+    if (stage_counts[s] < 0) return fail(Q4_ERR_SHAPE, "q4_matmul_chain: stage %d has a negative count", s);
+    sum += stage_counts[s];
+  }
+  if (sum != count)
+    return fail(Q4_ERR_SHAPE, "q4_matmul_chain: the stages hold %lld descriptors, count is %d", (long long)sum, count);
+  // Validate every descriptor first (nothing is enqueued on failure); empty
+  // problems and stages left empty drop out.
+  std::vector<MatmulArgs> list;
+  std::vector<int> stages;
+  list.reserve(static_cast<size_t>(count));
+  for (int s = 0, i = 0; s < n_stages; ++s) {
+    int kept = 0;
+    for (int k = 0; k < stage_counts[s]; ++k, ++i) {
+      const q4_matmul_desc& d = descs[i];
+      bool empty = false;
+      char who[64];
+      snprintf(who, sizeof who, "q4_matmul_chain[%d] (stage %d)", i, s);
+      q4_status st = check_matmul(who, d.x, M, d.K, d.codes, d.scales, d.biases, d.N, group, d.y, &empty);
+      if (st != Q4_OK) return st;
+      MatmulArgs a{d.x, d.codes, d.scales, d.biases, d.y, M, d.N, d.K};
+      if ((st = check_epilogue(who, d.epilogue, d.reserved, d.r, d.up_codes, d.up_scales, d.up_biases, &a)) != Q4_OK)
+        return st;
+      if (!empty) {
+        list.push_back(a);
+        ++kept;
+      }
+    }
+    if (kept > 0) stages.push_back(kept);
+  }
+  if (list.empty()) return Q4_OK;
+  const DeviceInfo* dev = nullptr;
+  q4_status st;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int n = static_cast<int>(stages.size());
+  if (!gemv_chain_supported(list.data(), static_cast<int>(list.size()))) {
+    // one batch launch (or set of launches) per stage, in order
+    for (int s = 0, i = 0; s < n; i += stages[s], ++s) {
+      std::vector<MatmulArgs> part(list.begin() + i, list.begin() + i + stages[s]);
+      if ((st = run_problems(part, *dev, cs, "q4_matmul_chain launch")) != Q4_OK) return st;
+    }
+    return Q4_OK;
+  }
+  // Persistent launches, each over as many whole stages as its parameter
+  // block holds, with one zeroed arrival counter per stage.
+  unsigned int* done = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&done), sizeof(unsigned int) * n, cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(done, 0, sizeof(unsigned int) * n, cs);
+  if (e != cudaSuccess) return from_cuda(e, "q4_matmul_chain workspace");
+  for (int s = 0, i = 0; s < n && st == Q4_OK;) {
+    int ns = 0, np = 0;
+    while (s + ns < n && ns < kGemvChainMaxStages && np + stages[s + ns] <= kGemvChainMaxProblems) np += stages[s + ns++];
+    if (ns == 0) {  // one stage of more problems than a launch holds: that stage as a batch
+      std::vector<MatmulArgs> part(list.begin() + i, list.begin() + i + stages[s]);
+      st = run_problems(part, *dev, cs, "q4_matmul_chain launch");
+      i += stages[s++];
+      continue;
+    }
+    st = from_cuda(launch_gemv_chain(list.data() + i, np, stages.data() + s, ns, done + s, cs, *dev),
+                   "q4_matmul_chain launch");
+    s += ns;
+    i += np;
+  }
+  e = cudaFreeAsync(done, cs);
+  if (st == Q4_OK && e != cudaSuccess) st = from_cuda(e, "q4_matmul_chain workspace");
+  return st;
+}
+
 q4_status q4_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int group, q4_stream_t stream) {
   if (count < 0) return fail(Q4_ERR_SHAPE, "q4_matmul_batch: negative count %d", count);
   if (count == 0) return Q4_OK;

@@ -128,6 +128,32 @@ __device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity
   }
 }
 
+// ---- grid-wide stage counters (persistent chain launches) ------------------
+// One CTA thread announces that the CTA finished a stage: a GPU-scope fence
+// (cumulative: it orders the writes of the CTA's other threads that this
+// thread has synchronized with, through an mbarrier, before the add) and a
+// release add.
+__device__ __forceinline__ void grid_arrive(unsigned int* counter) {
+  asm volatile("fence.acq_rel.gpu;\n\tred.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
+}
+
+// Waits until *counter >= target (acquire loads at GPU scope, a short sleep
+// between them).  Returns false (and raises the device flag) after
+// kWaitLimitNs.
+__device__ __forceinline__ bool grid_wait(const unsigned int* counter, unsigned int target) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= target) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_device_flags, kFlagWaitTimeout);
+      return false;
+    }
+    __nanosleep(32);
+  }
+}
+
 // ---- bulk (non-tensor TMA) copies and prefetch ----------------------------
 // Global -> shared, completion counted in bytes on `bar`.  dst, src 16-byte
 // aligned; bytes a multiple of 16.

@@ -83,11 +83,15 @@ struct XSlice {
   uint32_t v[WORDS][4][kRegs];
   float sum;
 
+  // kL2: src is global memory another CTA of the launch may have written
+  // (read through L2, not the SM's L1)
+  template <bool kL2 = false>
   __device__ __forceinline__ void load(const uint16_t* src) {
     sum = 0.f;
 #pragma unroll
     for (int w = 0; w < WORDS; ++w) {
-      const uint4 e = *reinterpret_cast<const uint4*>(src + 8 * w);
+      const uint4 e = kL2 ? __ldcg(reinterpret_cast<const uint4*>(src + 8 * w))
+                          : *reinterpret_cast<const uint4*>(src + 8 * w);
       const uint32_t pr[4] = {__byte_perm(e.x, e.z, 0x5410), __byte_perm(e.x, e.z, 0x7632),
                               __byte_perm(e.y, e.w, 0x5410), __byte_perm(e.y, e.w, 0x7632)};
       const uint32_t nat[4] = {e.x, e.y, e.z, e.w};  // (x[8w+2t], x[8w+2t+1])
@@ -234,6 +238,9 @@ struct GemvProblem {
 
 // CTAs per launch at most (one per SM).
 constexpr int kMaxCtas = 256;
+// Stages of a chain launch at most.
+constexpr int kMaxChainStages = kGemvChainMaxStages;
+static_assert(kGemvChainMaxProblems == 256, "chain problems: the large parameter block");
 
 template <int NP>
 struct GemvLaunch {
@@ -241,7 +248,15 @@ struct GemvLaunch {
   int consumer_threads;  // a multiple of 32
   int stages;
   uint32_t stage_bytes;  // >= every problem's tile and activation block, 128-byte multiple
-  int64_t total_bytes;   // packed bytes of the whole list
+  uint32_t x_bytes;      // a chain's activation buffer after the ring (0 for a batch), 128-byte multiple
+  int64_t total_bytes;   // packed bytes of the whole list (a batch launch)
+  // A chain launch: stages run in order, stage s being the problems
+  // [stage_begin[s], stage_begin[s + 1]) split over all CTAs like a batch of
+  // stage_total[s] bytes (byte_begin counts from the stage's start); before
+  // reading its inputs for stage s > 0 every CTA waits until done[s - 1]
+  // (zero at launch) counts all CTAs.
+  int n_stages;
+  unsigned int* done;
   // first[c]: the first problem that ends after CTA c's first byte.  Every
   // role of the CTA starts its walk over the list there: the problems before
   // it hold none of its rows, and reading their descriptors (a constant-cache
@@ -249,6 +264,8 @@ struct GemvLaunch {
   // to cost the whole launch 5 %.  A launch of at most kFewProblems problems
   // walks from the first.
   uint16_t first[NP > kFewProblems ? kMaxCtas : 1];
+  uint16_t stage_begin[NP > kFewProblems ? kMaxChainStages + 1 : 1];
+  int64_t stage_total[NP > kFewProblems ? kMaxChainStages : 1];
   GemvProblem prob[NP];
 };
 
@@ -307,8 +324,14 @@ template <bool EPI>
 __device__ __forceinline__ bool epilogue_warp_k(const GemvProblem& P, const Geometry& g) {
   return g.wpt > 1 || (fused_k<EPI>(P) && g.wpt >= 1);
 }
-template <bool EPI>
+// CHAIN: the residual may have been written by another CTA of the launch
+// (an earlier stage), so it is read through L2.
+template <bool EPI, bool CHAIN>
 __device__ __forceinline__ uint16_t store_k(float v, const GemvProblem& P, int64_t idx) {
+  if constexpr (EPI && CHAIN) {
+    if (P.epi == kEpiResidual) return float_to_bf16_bits(v + bf16_bits_to_float(__ldcg(P.r + idx)));
+    return float_to_bf16_bits(v);
+  }
   if constexpr (EPI) return epilogue_bf16(v, P.epi, P.r, idx);
   return float_to_bf16_bits(v);
 }
@@ -317,13 +340,31 @@ __device__ __forceinline__ uint32_t tile_rows(int64_t r_end, int64_t row0, int r
   return static_cast<uint32_t>((r_end - row0 < rt) ? (r_end - row0) : rt);
 }
 
+// sum over this lane's 32 inputs of x * (mac_offset + q) for one weight row
+// (four code words): the same operations in the same order on every path,
+// so a row's result does not depend on where it falls in a tile.
+__device__ __forceinline__ float row_acc(const uint32_t (&words)[4], const XSlice<4, Q4_GEMV_MAC>& xs, uint32_t kmask,
+                                         uint32_t kmagic) {
+  float acc = 0.f;
+  if constexpr (Q4_GEMV_MAC == kMacMixedBf16) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      word_dot_bf16_acc(words[w], xs.v[w][0][0], xs.v[w][1][0], xs.v[w][2][0], xs.v[w][3][0], acc, kmask, kmagic);
+  } else {
+    float a0[1] = {0.f}, a1[1] = {0.f};
+    dot_plus128<1, 4, Q4_GEMV_MAC>(words, *reinterpret_cast<const XSlice<4, Q4_GEMV_MAC>(*)[1]>(&xs), a0, a1);
+    acc = a0[0] + a1[0];
+  }
+  return acc;
+}
+
 // The rows of problem `pi` that belong to this CTA's byte range [lo, hi) of
 // the concatenated list: [*r0, *r1).  A row belongs to the CTA whose range
-// holds its first packed byte, with segment boundaries rounded up to whole
-// tiles of the problem, so every row has the same place in its tile however
-// the list is split (results do not depend on batching) and each row of the
-// list belongs to exactly one CTA.  Returns false when the problem lies
-// entirely after the range (the caller stops scanning).
+// holds its first packed byte, so each row of the list belongs to exactly one
+// CTA; a row's arithmetic is the same wherever it falls in a tile (row_acc,
+// the fixed reduction trees), so results do not depend on the split.
+// Returns false when the problem lies entirely after the range (the caller
+// stops scanning).
 template <bool EPI, int NP>
 __device__ __forceinline__ bool segment_of(const GemvLaunch<NP>& L, int pi, int64_t lo, int64_t hi, int64_t* r0,
                                            int64_t* r1) {
@@ -333,17 +374,17 @@ __device__ __forceinline__ bool segment_of(const GemvLaunch<NP>& L, int pi, int6
   *r0 = *r1 = 0;
   if (pb >= hi) return false;
   if (pe <= lo) return true;
-  const int64_t rt = rtile_k<EPI>(P, geometry_of(P.K, L.consumer_threads));
   const int64_t a = (lo > pb ? lo : pb) - pb, b = (hi < pe ? hi : pe) - pb;
-  *r0 = ((a + rb - 1) / rb + rt - 1) / rt * rt;
-  *r1 = ((b + rb - 1) / rb + rt - 1) / rt * rt;
+  *r0 = (a + rb - 1) / rb;
+  *r1 = (b + rb - 1) / rb;
   if (*r0 > P.N) *r0 = P.N;
   if (*r1 > P.N) *r1 = P.N;
   return true;
 }
 
-template <int MR, int MAXT, int NP, bool EPI>
+template <int MR, int MAXT, int NP, bool EPI, bool CHAIN>
 __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ GemvLaunch<NP> L) {
+  static_assert(!CHAIN || NP > kFewProblems, "chains use the large parameter block");
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int V = kRpt * MR;
   constexpr int VP = pow2_at_least(V);
@@ -351,14 +392,22 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   const int warp = tid >> 5, lane = tid & 31;
   const int consumer_warps = L.consumer_threads >> 5;
 
-  float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(L.stages) * L.stage_bytes);
+  // A chain's activation block [MR, K] of the current segment, staged once
+  // per CTA (every team reads its lanes' slices from here).
+  uint8_t* xbuf = smem + static_cast<size_t>(L.stages) * L.stage_bytes;
+  float* red = reinterpret_cast<float*>(xbuf + L.x_bytes);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(red + kRedSlots * kRedSlotFloats);
   uint64_t* empty_bar = full_bar + L.stages;
   uint64_t* rfull_bar = empty_bar + L.stages;   // [kRedSlots]
   uint64_t* rempty_bar = rfull_bar + kRedSlots;  // [kRedSlots]
+  // Chains: go (phase s - 1 completes when this CTA may read the inputs of
+  // stage s) and stage_done (phase s completes when every consumer warp and
+  // the epilogue warp finished their writes of stage s).
+  uint64_t* go_bar = rempty_bar + kRedSlots;
+  uint64_t* stage_done_bar = go_bar + 1;
   // Set by any thread whose bounded wait gave up: the epilogue warp then
   // writes NaN for the partial sums it cannot vouch for.
-  volatile uint32_t* gave_up = reinterpret_cast<volatile uint32_t*>(rempty_bar + kRedSlots);
+  volatile uint32_t* gave_up = reinterpret_cast<volatile uint32_t*>(stage_done_bar + 1);
 
   if (tid == 0) {
     for (int s = 0; s < L.stages; ++s) {
@@ -369,24 +418,40 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       mbar_init(&rfull_bar[s], consumer_warps);
       mbar_init(&rempty_bar[s], 1);
     }
+    mbar_init(go_bar, 1);
+    mbar_init(stage_done_bar, consumer_warps + 1);
     *gave_up = 0u;
     fence_mbar_init();
   }
   __syncthreads();
   pdl_launch_dependents();
 
-  // This CTA's share of the list: a contiguous, balanced range of packed bytes.
-  const int64_t lo = static_cast<int64_t>(blockIdx.x) * L.total_bytes / gridDim.x;
-  const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * L.total_bytes / gridDim.x;
-  const int p0 = NP > kFewProblems ? L.first[blockIdx.x] : 0;
+  // The launch's stages (a batch is one) and this CTA's share of each: a
+  // contiguous, balanced range [lo, hi) of the stage's packed bytes, and the
+  // problems [pb, pe) to walk for it.
+  const int n_st = CHAIN ? L.n_stages : 1;
+  auto share = [&](int cs, int64_t& lo, int64_t& hi, int& pb, int& pe) {
+    const int64_t T = CHAIN ? L.stage_total[cs] : L.total_bytes;
+    lo = static_cast<int64_t>(blockIdx.x) * T / gridDim.x;
+    hi = static_cast<int64_t>(blockIdx.x + 1) * T / gridDim.x;
+    if constexpr (CHAIN) {
+      pb = L.stage_begin[cs];
+      pe = L.stage_begin[cs + 1];
+    } else {
+      pb = NP > kFewProblems ? L.first[blockIdx.x] : 0;
+      pe = L.count;
+    }
+  };
 
   if (warp == consumer_warps) {
     // ---------------- producer warp ----------------
     if (lane == 0) {
       {  // warm L2 with the first tiles of the range (a hint; changes no value)
-        int64_t r0, r1;
-        int issued = 0;
-        for (int pi = p0; pi < L.count && issued < L.stages; ++pi) {
+        int64_t r0, r1, lo, hi;
+        int issued = 0, pb, pe;
+        for (int cs = 0; cs < n_st && issued < L.stages; ++cs) {
+        share(cs, lo, hi, pb, pe);
+        for (int pi = pb; pi < pe && issued < L.stages; ++pi) {
           if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
           const GemvProblem& P = L.prob[pi];
           const Geometry geo = geometry_of(P.K, L.consumer_threads);
@@ -404,13 +469,21 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
             }
           }
         }
+        }
       }
       pdl_wait_predecessors();
-      // Ring order per segment: its activation block [MR, K], then its tiles.
+      // Ring order per segment: its activation block [MR, K] (a batch; a
+      // chain's consumers read theirs from global memory once the stage's
+      // inputs are complete), then its tiles.  The producer never waits for
+      // other CTAs: across a chain's stages it streams weights ahead.
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool dead = false;
-      for (int pi = p0; pi < L.count && !dead; ++pi) {
+      for (int cs = 0; cs < n_st && !dead; ++cs) {
+      int64_t lo, hi;
+      int pb, pe;
+      share(cs, lo, hi, pb, pe);
+      for (int pi = pb; pi < pe && !dead; ++pi) {
         int64_t r0, r1;
         if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
         if (r0 >= r1) continue;
@@ -418,7 +491,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         const Geometry geo = geometry_of(P.K, L.consumer_threads);
         const int half_k = P.K >> 1;
         const int rtile = rtile_k<EPI>(P, geo);
-        for (int64_t row0 = r0 - rtile; row0 < r1; row0 += rtile) {  // first pass: x
+        for (int64_t row0 = CHAIN ? r0 : r0 - rtile; row0 < r1; row0 += rtile) {  // a batch's first pass: x
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; *gave_up = 1u; break; }
           uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
           if (row0 < r0) {
@@ -449,6 +522,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
           if (++stage == L.stages) { stage = 0; phase ^= 1u; }
         }
       }
+      }
       // No copy may still target this CTA's shared memory when it exits.
       for (int i = 0; i < min(issued, L.stages); ++i) {
         int s = stage - 1 - i;
@@ -467,7 +541,26 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     int slot = 0;
     uint32_t sph = 0;
     bool dead = false;
-    for (int pi = p0; pi < L.count; ++pi) {
+    for (int cs = 0; cs < n_st; ++cs) {
+    if constexpr (CHAIN) {
+      if (cs > 0) {
+        // Stage cs - 1 is complete in this CTA once its consumer warps and
+        // this warp have arrived: announce it, wait for every CTA, then let
+        // this CTA's consumers read the inputs of stage cs.  (A CTA whose
+        // wait gave up still announces, so no other CTA waits on it.)
+        if (!dead && !mbar_wait(stage_done_bar, static_cast<uint32_t>(cs - 1) & 1u)) { dead = true; *gave_up = 1u; }
+        if (lane == 0) {
+          grid_arrive(&L.done[cs - 1]);
+          if (!dead && !grid_wait(&L.done[cs - 1], gridDim.x)) { dead = true; *gave_up = 1u; }
+          mbar_arrive(go_bar);
+        }
+        dead = __shfl_sync(0xFFFFFFFFu, dead ? 1 : 0, 0) != 0;
+      }
+    }
+    int64_t lo, hi;
+    int pb, pe;
+    share(cs, lo, hi, pb, pe);
+    for (int pi = pb; pi < pe; ++pi) {
       int64_t r0, r1;
       if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
       const GemvProblem& P = L.prob[pi];
@@ -491,13 +584,18 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
             for (int w = 0; w < geo.wpt; ++w) u += rs[(i + n * MR) * geo.wpt + w];
             P.y[idx] = float_to_bf16_bits(silu_f32(v) * u);
           } else {
-            P.y[idx] = store_k<EPI>(v, P, idx);
+            P.y[idx] = store_k<EPI, CHAIN>(v, P, idx);
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&rempty_bar[slot]);
         if (++slot == kRedSlots) { slot = 0; sph ^= 1u; }
       }
+    }
+    if constexpr (CHAIN) {
+      __syncwarp();
+      if (lane == 0 && cs + 1 < n_st) mbar_arrive(stage_done_bar);
+    }
     }
     return;
   }
@@ -508,7 +606,14 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   int stage = 0, slot = 0;
   uint32_t phase = 0, sph = 0;
   bool dead = false;
-  for (int pi = p0; pi < L.count; ++pi) {
+  for (int cs = 0; cs < n_st; ++cs) {
+  if constexpr (CHAIN) {  // the inputs of stage cs are complete (every CTA finished stage cs - 1)
+    if (cs > 0 && !dead && !mbar_wait(go_bar, static_cast<uint32_t>(cs - 1) & 1u)) { dead = true; *gave_up = 1u; }
+  }
+  int64_t lo, hi;
+  int pb, pe;
+  share(cs, lo, hi, pb, pe);
+  for (int pi = pb; pi < pe; ++pi) {
     int64_t r_begin, r_end;
     if (!segment_of<EPI>(L, pi, lo, hi, &r_begin, &r_end)) break;
     if (r_begin >= r_end) continue;
@@ -529,10 +634,28 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     const uint32_t sc_step = static_cast<uint32_t>(geo.teams) * geo.G * 2;
 
     // Activations: this lane's 32 inputs of each row, from the ring stage
-    // that precedes the segment's tiles.
-    if (!dead && !mbar_wait(&full_bar[stage], phase)) { dead = true; *gave_up = 1u; }
+    // that precedes the segment's tiles (a batch) or from global memory (a
+    // chain).
     XSlice<4, Q4_GEMV_MAC> xsl[MR];
-    {
+    if constexpr (CHAIN) {
+      // One L2 read of the block per CTA (the teams would read it once each):
+      // every consumer thread copies 16-byte chunks into the buffer, which
+      // the first barrier shows no thread still reads for the last segment.
+      named_bar_sync(1, L.consumer_threads);
+      const int chunks = MR * P.K / 8;
+      for (int i = tid; i < chunks; i += L.consumer_threads)
+        reinterpret_cast<uint4*>(xbuf)[i] = __ldcg(reinterpret_cast<const uint4*>(P.x) + i);
+      named_bar_sync(1, L.consumer_threads);
+      const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(xbuf);
+#pragma unroll
+      for (int m = 0; m < MR; ++m) {
+        if (active)
+          xsl[m].load(xsrc + m * P.K + j * 32);
+        else
+          xsl[m].zero();
+      }
+    } else {
+      if (!dead && !mbar_wait(&full_bar[stage], phase)) { dead = true; *gave_up = 1u; }
       const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(smem + static_cast<size_t>(stage) * L.stage_bytes);
 #pragma unroll
       for (int m = 0; m < MR; ++m) {
@@ -541,10 +664,10 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         else
           xsl[m].zero();
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[stage]);
+      if (++stage == L.stages) { stage = 0; phase ^= 1u; }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[stage]);
-    if (++stage == L.stages) { stage = 0; phase ^= 1u; }
 
     const bool use_red = epilogue_warp_k<EPI>(P, geo);
     const int rtile = rtile_k<EPI>(P, geo);
@@ -591,21 +714,8 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         for (int rr = 0; rr < kRpt; ++rr) {
           const float c = fmaf(-kOffset, sc[rr], bi[rr]);
 #pragma unroll
-          for (int m = 0; m < MR; ++m) {
-            float acc = 0.f;
-            if constexpr (Q4_GEMV_MAC == kMacMixedBf16) {
-#pragma unroll
-              for (int w = 0; w < 4; ++w)
-                word_dot_bf16_acc(words[rr][w], xsl[m].v[w][0][0], xsl[m].v[w][1][0], xsl[m].v[w][2][0],
-                                  xsl[m].v[w][3][0], acc, kmask, kmagic);
-            } else {
-              float a0[1] = {0.f}, a1[1] = {0.f};
-              dot_plus128<1, 4, Q4_GEMV_MAC>(words[rr], *reinterpret_cast<const XSlice<4, Q4_GEMV_MAC>(*)[1]>(&xsl[m]),
-                                             a0, a1);
-              acc = a0[0] + a1[0];
-            }
-            vals[rr * MR + m] = fmaf(sc[rr], acc, c * xsl[m].sum);
-          }
+          for (int m = 0; m < MR; ++m)
+            vals[rr * MR + m] = fmaf(sc[rr], row_acc(words[rr], xsl[m], kmask, kmagic), c * xsl[m].sum);
         }
       } else {
         uint32_t words[kRpt][4];
@@ -634,13 +744,10 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 #pragma unroll
           for (int rr = 0; rr < kRpt; ++rr) {
             if (geo.team >= 32 && rr >= nv) break;  // warp-uniform
-            float a0[MR], a1[MR];
-#pragma unroll
-            for (int m = 0; m < MR; ++m) a0[m] = a1[m] = 0.f;
-            dot_plus128<MR, 4, Q4_GEMV_MAC>(words[rr], xsl, a0, a1);
             const float c = fmaf(-kOffset, sc[rr], bi[rr]);
 #pragma unroll
-            for (int m = 0; m < MR; ++m) vals[rr * MR + m] = fmaf(sc[rr], a0[m] + a1[m], c * xsl[m].sum);
+            for (int m = 0; m < MR; ++m)
+              vals[rr * MR + m] = fmaf(sc[rr], row_acc(words[rr], xsl[m], kmask, kmagic), c * xsl[m].sum);
           }
         }
       }
@@ -657,7 +764,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
             const int lr = team_idx + rr * geo.teams;  // row within the tile
             if (!use_red) {
               const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row0 + lr;
-              P.y[idx] = store_k<EPI>(dead ? kNaN : tot, P, idx);
+              P.y[idx] = store_k<EPI, CHAIN>(dead ? kNaN : tot, P, idx);
             } else {
               rs[(lr * MR + m) * geo.wpt + warp_in_team] = tot;
             }
@@ -679,12 +786,17 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 #pragma unroll
               for (int m = 0; m < MR; ++m) {
                 const int64_t idx = static_cast<int64_t>(m) * P.y_ld + row;
-                P.y[idx] = store_k<EPI>(dead ? kNaN : vals[rr * MR + m], P, idx);
+                P.y[idx] = store_k<EPI, CHAIN>(dead ? kNaN : vals[rr * MR + m], P, idx);
               }
             }
         }
       }
     }
+  }
+  if constexpr (CHAIN) {  // this warp's writes of stage cs are done
+    __syncwarp();
+    if (lane == 0 && cs + 1 < n_st) mbar_arrive(stage_done_bar);
+  }
   }
 }
 
@@ -834,6 +946,30 @@ cudaError_t run_generic(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, 
   return launch_pdl(gemv_generic_kernel<MR>, dim3(grid), dim3(256), 0, stream, p);
 }
 
+// Grows *stage_bytes to hold a tile of P (and, with_x, its activation block
+// [MR, K]); false if the epilogue warp's reduction slots cannot take P's
+// tiles (they are sized for kConsumers1 / kConsumers2).
+bool ring_stage_fits(const GemvProblem& P, int mr, int consumers, bool with_x, uint32_t& stage_bytes) {
+  const Geometry geo = geometry_of(P.K, consumers);
+  const uint32_t tile = static_cast<uint32_t>(geo.rt) * (P.K / 2) +
+                        2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
+  stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
+  if (with_x) stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(mr) * P.K * 2 + 127u) & ~127u);
+  return !(uses_epilogue_warp(P, geo) && geo.rt * mr * geo.wpt > kRedSlotFloats);
+}
+
+// Ring depth and dynamic shared memory for stages of stage_bytes (and a
+// chain's activation buffer of x_bytes).
+bool ring_of(uint32_t stage_bytes, uint32_t x_bytes, const DeviceInfo& dev, int* stages, size_t* smem) {
+  // activation buffer, reduction slots, their barriers, the chain's two barriers, the flag word
+  const size_t fixed = x_bytes + sizeof(float) * kRedSlots * kRedSlotFloats + 16 * kRedSlots + 16 + 16;
+  const size_t budget = std::min<size_t>(Q4_GEMV_SMEM_BUDGET, dev.smem_optin);
+  if (fixed + 2 * (stage_bytes + 16) > dev.smem_optin) return false;
+  *stages = std::max(2, std::min(static_cast<int>((budget - fixed) / (stage_bytes + 16)), 12));
+  *smem = static_cast<size_t>(*stages) * stage_bytes + fixed + 16 * *stages;
+  return true;
+}
+
 // Launches the bulk-copy kernel over `count` problems of `probs` (all taking
 // this path, all with MR activation rows).
 template <int MR, int NP>
@@ -846,27 +982,19 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   int64_t total = 0;
   for (int i = 0; i < count; ++i) {
     const GemvProblem& P = probs[i];
-    const Geometry geo = geometry_of(P.K, consumers);
-    const uint32_t tile = static_cast<uint32_t>(geo.rt) * (P.K / 2) +
-                          2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
-    stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
-    stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(MR) * P.K * 2 + 127u) & ~127u);
-    if (uses_epilogue_warp(P, geo) && geo.rt * MR * geo.wpt > kRedSlotFloats)
-      return cudaErrorInvalidConfiguration;  // the reduction slots are sized for kConsumers1 / kConsumers2
+    if (!ring_stage_fits(P, MR, consumers, true, stage_bytes)) return cudaErrorInvalidConfiguration;
     L.prob[i] = P;
     L.prob[i].byte_begin = total;
     total += P.N * problem_row_bytes(P);
   }
-  const size_t fixed = sizeof(float) * kRedSlots * kRedSlotFloats + 16 * kRedSlots + 16;
-  const size_t budget = std::min<size_t>(Q4_GEMV_SMEM_BUDGET, dev.smem_optin);
-  if (fixed + 2 * (stage_bytes + 16) > dev.smem_optin) return cudaErrorInvalidConfiguration;
-  int stages = static_cast<int>((budget - fixed) / (stage_bytes + 16));
-  stages = std::max(2, std::min(stages, 12));
-  const size_t smem = static_cast<size_t>(stages) * stage_bytes + fixed + 16 * stages;
+  int stages = 0;
+  size_t smem = 0;
+  if (!ring_of(stage_bytes, 0, dev, &stages, &smem)) return cudaErrorInvalidConfiguration;
   L.count = count;
   L.consumer_threads = consumers;
   L.stages = stages;
   L.stage_bytes = stage_bytes;
+  L.x_bytes = 0;
   L.total_bytes = total;
   // Enough CTAs that every one has work; one per SM.
   const int64_t rows = [&] { int64_t r = 0; for (int i = 0; i < count; ++i) r += probs[i].N; return r; }();
@@ -882,8 +1010,67 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   }
   bool epi = false;
   for (int i = 0; i < count; ++i) epi = epi || probs[i].epi != kEpiNone || is_fused(probs[i]);
-  auto kern = epi ? gemv_kernel<MR, kThreads, NP, true> : gemv_kernel<MR, kThreads, NP, false>;
+  auto kern = epi ? gemv_kernel<MR, kThreads, NP, true, false> : gemv_kernel<MR, kThreads, NP, false, false>;
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, L);
+}
+
+// One chain launch: `count` problems (all taking the bulk-copy kernel, MR
+// activation rows) in n_stages stages of stage_counts[s] problems each;
+// done: n_stages counters, zero.  Every CTA takes part in every stage, so
+// the launch is cooperative (all CTAs resident at once, one per SM).
+template <int MR>
+cudaError_t run_chain(const GemvProblem* probs, int count, const int* stage_counts, int n_stages, unsigned int* done,
+                      const DeviceInfo& dev, cudaStream_t stream) {
+  constexpr int NP = kMaxProblems;
+  constexpr int kThreads = MR == 1 ? kThreads1 : kThreads2;
+  const int consumers = consumers_for(MR);
+  if (count < 1 || count > NP || n_stages < 1 || n_stages > kMaxChainStages) return cudaErrorInvalidValue;
+  thread_local GemvLaunch<NP> L;
+  uint32_t stage_bytes = 128, x_bytes = 128;
+  bool epi = false;
+  int i = 0;
+  for (int s = 0; s < n_stages; ++s) {
+    L.stage_begin[s] = static_cast<uint16_t>(i);
+    int64_t total = 0;
+    for (int k = 0; k < stage_counts[s]; ++k, ++i) {
+      if (i >= count) return cudaErrorInvalidValue;
+      const GemvProblem& P = probs[i];
+      if (!ring_stage_fits(P, MR, consumers, false, stage_bytes)) return cudaErrorInvalidConfiguration;
+      x_bytes = std::max(x_bytes, (static_cast<uint32_t>(MR) * P.K * 2 + 127u) & ~127u);
+      L.prob[i] = P;
+      L.prob[i].byte_begin = total;
+      total += P.N * problem_row_bytes(P);
+      epi = epi || P.epi != kEpiNone || is_fused(P);
+    }
+    L.stage_total[s] = total;
+  }
+  if (i != count) return cudaErrorInvalidValue;
+  L.stage_begin[n_stages] = static_cast<uint16_t>(count);
+  int stages = 0;
+  size_t smem = 0;
+  if (!ring_of(stage_bytes, x_bytes, dev, &stages, &smem)) return cudaErrorInvalidConfiguration;
+  L.count = count;
+  L.consumer_threads = consumers;
+  L.stages = stages;
+  L.stage_bytes = stage_bytes;
+  L.x_bytes = x_bytes;
+  L.total_bytes = 0;
+  L.n_stages = n_stages;
+  L.done = done;
+  const int grid = std::min(dev.sm_count, kMaxCtas);
+  auto kern = epi ? gemv_kernel<MR, kThreads, NP, true, true> : gemv_kernel<MR, kThreads, NP, false, true>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kern, L);
 }
 
 // Launches in groups of at most kMaxProblems problems.
@@ -903,14 +1090,18 @@ cudaError_t run_problems(std::vector<GemvProblem>& probs, const DeviceInfo& dev,
 cudaError_t gemv_device_flags(unsigned int* flags, bool clear) { return tu_device_flags(flags, clear); }
 
 cudaError_t gemv_prepare_device(const DeviceInfo& dev) {
-  for (const void* kern : {reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, true>),
-                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, true>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true>)}) {
+  for (const void* kern : {reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, false, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, true, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false, true>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true, true>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, false, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, true, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true, false>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false, true>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true, true>)}) {
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dev.smem_optin));
     if (e != cudaSuccess) return e;
@@ -957,6 +1148,41 @@ cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t st
 
 cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev) {
   return launch_gemv_batch(&a, 1, stream, dev);
+}
+
+bool gemv_chain_supported(const MatmulArgs* list, int count) {
+  if (count < 1) return false;
+  const int64_t M = list[0].M;
+  if (M < 1 || M > 2) return false;
+  for (int i = 0; i < count; ++i)
+    if (list[i].M != M || !tma_ok(list[i], static_cast<int>(M))) return false;
+  return true;
+}
+
+cudaError_t launch_gemv_chain(const MatmulArgs* list, int count, const int* stage_counts, int n_stages,
+                              unsigned int* done, cudaStream_t stream, const DeviceInfo& dev) {
+  if (count > kGemvChainMaxProblems || n_stages > kGemvChainMaxStages) return cudaErrorInvalidValue;
+  GemvProblem probs[kGemvChainMaxProblems];
+  for (int i = 0; i < count; ++i) {
+    const MatmulArgs& a = list[i];
+    GemvProblem& P = probs[i];
+    P.x = a.x;
+    P.codes = a.codes;
+    P.scales = a.scales;
+    P.biases = a.biases;
+    P.y = a.y;
+    P.r = a.r;
+    P.up_codes = a.up_codes;
+    P.up_scales = a.up_scales;
+    P.up_biases = a.up_biases;
+    P.N = a.N;
+    P.y_ld = a.N;
+    P.K = static_cast<int32_t>(a.K);
+    P.epi = a.epi;
+    P.byte_begin = 0;
+  }
+  return list[0].M == 1 ? run_chain<1>(probs, count, stage_counts, n_stages, done, dev, stream)
+                        : run_chain<2>(probs, count, stage_counts, n_stages, done, dev, stream);
 }
 
 }  // namespace q4

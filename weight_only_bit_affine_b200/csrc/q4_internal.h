@@ -79,6 +79,14 @@ cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceIn
 // Several independent matmuls; those the bulk-copy kernel takes share one
 // launch (per chunk size).
 cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
+// A chain of dependent stages in one persistent launch (q4_matmul_chain):
+// whether it takes `list` (one or two activation rows, every problem on the
+// bulk-copy path), and the launch itself -- stage s is the next
+// stage_counts[s] problems of `list`; done: n_stages counters, zero.
+constexpr int kGemvChainMaxProblems = 256, kGemvChainMaxStages = 256;
+bool gemv_chain_supported(const MatmulArgs* list, int count);
+cudaError_t launch_gemv_chain(const MatmulArgs* list, int count, const int* stage_counts, int n_stages,
+                              unsigned int* done, cudaStream_t stream, const DeviceInfo& dev);
 
 // Tensor-core tiles (tcgen05, dequantized weights in tensor memory) for
 // three or more activation rows (from kTensorCoreMinRows, or where the
