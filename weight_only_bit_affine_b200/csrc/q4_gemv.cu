@@ -83,15 +83,11 @@ struct XSlice {
   uint32_t v[WORDS][4][kRegs];
   float sum;
 
-  // kL2: src is global memory another CTA of the launch may have written
-  // (read through L2, not the SM's L1)
-  template <bool kL2 = false>
   __device__ __forceinline__ void load(const uint16_t* src) {
     sum = 0.f;
 #pragma unroll
     for (int w = 0; w < WORDS; ++w) {
-      const uint4 e = kL2 ? __ldcg(reinterpret_cast<const uint4*>(src + 8 * w))
-                          : *reinterpret_cast<const uint4*>(src + 8 * w);
+      const uint4 e = *reinterpret_cast<const uint4*>(src + 8 * w);
       const uint32_t pr[4] = {__byte_perm(e.x, e.z, 0x5410), __byte_perm(e.x, e.z, 0x7632),
                               __byte_perm(e.y, e.w, 0x5410), __byte_perm(e.y, e.w, 0x7632)};
       const uint32_t nat[4] = {e.x, e.y, e.z, e.w};  // (x[8w+2t], x[8w+2t+1])
@@ -248,7 +244,6 @@ struct GemvLaunch {
   int consumer_threads;  // a multiple of 32
   int stages;
   uint32_t stage_bytes;  // >= every problem's tile and activation block, 128-byte multiple
-  uint32_t x_bytes;      // a chain's activation buffer after the ring (0 for a batch), 128-byte multiple
   int64_t total_bytes;   // packed bytes of the whole list (a batch launch)
   // A chain launch: stages run in order, stage s being the problems
   // [stage_begin[s], stage_begin[s + 1]) split over all CTAs like a batch of
@@ -392,10 +387,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   const int warp = tid >> 5, lane = tid & 31;
   const int consumer_warps = L.consumer_threads >> 5;
 
-  // A chain's activation block [MR, K] of the current segment, staged once
-  // per CTA (every team reads its lanes' slices from here).
-  uint8_t* xbuf = smem + static_cast<size_t>(L.stages) * L.stage_bytes;
-  float* red = reinterpret_cast<float*>(xbuf + L.x_bytes);
+  float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(L.stages) * L.stage_bytes);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(red + kRedSlots * kRedSlotFloats);
   uint64_t* empty_bar = full_bar + L.stages;
   uint64_t* rfull_bar = empty_bar + L.stages;   // [kRedSlots]
@@ -638,15 +630,12 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     // chain).
     XSlice<4, Q4_GEMV_MAC> xsl[MR];
     if constexpr (CHAIN) {
-      // One L2 read of the block per CTA (the teams would read it once each):
-      // every consumer thread copies 16-byte chunks into the buffer, which
-      // the first barrier shows no thread still reads for the last segment.
-      named_bar_sync(1, L.consumer_threads);
-      const int chunks = MR * P.K / 8;
-      for (int i = tid; i < chunks; i += L.consumer_threads)
-        reinterpret_cast<uint4*>(xbuf)[i] = __ldcg(reinterpret_cast<const uint4*>(P.x) + i);
-      named_bar_sync(1, L.consumer_threads);
-      const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(xbuf);
+      // Plain loads: this CTA passed the stage barrier (an acquire at GPU
+      // scope, then the go barrier), after which every write of the earlier
+      // stages is visible to them; the teams after the first hit in L1
+      // (a read through L2 per team, or staging the block in shared memory
+      // at the cost of a ring stage, were both slower).
+      const uint16_t* xsrc = P.x;
 #pragma unroll
       for (int m = 0; m < MR; ++m) {
         if (active)
@@ -958,11 +947,10 @@ bool ring_stage_fits(const GemvProblem& P, int mr, int consumers, bool with_x, u
   return !(uses_epilogue_warp(P, geo) && geo.rt * mr * geo.wpt > kRedSlotFloats);
 }
 
-// Ring depth and dynamic shared memory for stages of stage_bytes (and a
-// chain's activation buffer of x_bytes).
-bool ring_of(uint32_t stage_bytes, uint32_t x_bytes, const DeviceInfo& dev, int* stages, size_t* smem) {
-  // activation buffer, reduction slots, their barriers, the chain's two barriers, the flag word
-  const size_t fixed = x_bytes + sizeof(float) * kRedSlots * kRedSlotFloats + 16 * kRedSlots + 16 + 16;
+// Ring depth and dynamic shared memory for stages of stage_bytes.
+bool ring_of(uint32_t stage_bytes, const DeviceInfo& dev, int* stages, size_t* smem) {
+  // reduction slots, their barriers, the chain's two barriers, the flag word
+  const size_t fixed = sizeof(float) * kRedSlots * kRedSlotFloats + 16 * kRedSlots + 16 + 16;
   const size_t budget = std::min<size_t>(Q4_GEMV_SMEM_BUDGET, dev.smem_optin);
   if (fixed + 2 * (stage_bytes + 16) > dev.smem_optin) return false;
   *stages = std::max(2, std::min(static_cast<int>((budget - fixed) / (stage_bytes + 16)), 12));
@@ -989,12 +977,11 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   }
   int stages = 0;
   size_t smem = 0;
-  if (!ring_of(stage_bytes, 0, dev, &stages, &smem)) return cudaErrorInvalidConfiguration;
+  if (!ring_of(stage_bytes, dev, &stages, &smem)) return cudaErrorInvalidConfiguration;
   L.count = count;
   L.consumer_threads = consumers;
   L.stages = stages;
   L.stage_bytes = stage_bytes;
-  L.x_bytes = 0;
   L.total_bytes = total;
   // Enough CTAs that every one has work; one per SM.
   const int64_t rows = [&] { int64_t r = 0; for (int i = 0; i < count; ++i) r += probs[i].N; return r; }();
@@ -1026,7 +1013,7 @@ cudaError_t run_chain(const GemvProblem* probs, int count, const int* stage_coun
   const int consumers = consumers_for(MR);
   if (count < 1 || count > NP || n_stages < 1 || n_stages > kMaxChainStages) return cudaErrorInvalidValue;
   thread_local GemvLaunch<NP> L;
-  uint32_t stage_bytes = 128, x_bytes = 128;
+  uint32_t stage_bytes = 128;
   bool epi = false;
   int i = 0;
   for (int s = 0; s < n_stages; ++s) {
@@ -1036,7 +1023,6 @@ cudaError_t run_chain(const GemvProblem* probs, int count, const int* stage_coun
       if (i >= count) return cudaErrorInvalidValue;
       const GemvProblem& P = probs[i];
       if (!ring_stage_fits(P, MR, consumers, false, stage_bytes)) return cudaErrorInvalidConfiguration;
-      x_bytes = std::max(x_bytes, (static_cast<uint32_t>(MR) * P.K * 2 + 127u) & ~127u);
       L.prob[i] = P;
       L.prob[i].byte_begin = total;
       total += P.N * problem_row_bytes(P);
@@ -1048,12 +1034,11 @@ cudaError_t run_chain(const GemvProblem* probs, int count, const int* stage_coun
   L.stage_begin[n_stages] = static_cast<uint16_t>(count);
   int stages = 0;
   size_t smem = 0;
-  if (!ring_of(stage_bytes, x_bytes, dev, &stages, &smem)) return cudaErrorInvalidConfiguration;
+  if (!ring_of(stage_bytes, dev, &stages, &smem)) return cudaErrorInvalidConfiguration;
   L.count = count;
   L.consumer_threads = consumers;
   L.stages = stages;
   L.stage_bytes = stage_bytes;
-  L.x_bytes = x_bytes;
   L.total_bytes = 0;
   L.n_stages = n_stages;
   L.done = done;
