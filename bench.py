@@ -394,9 +394,24 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
             q4.q8_matmul(x_down if p.K == 11264 else x, c, s, b, out=y)
 
     ms8 = _graph_ms(dev, q8_layers, 50) / 4
-    rows["q8_layer_M1"] = {"us_per_layer": round(ms8 * 1e3, 2), "GBps": round(bytes8 / (ms8 * 1e-3) / 1e9, 1),
-                           "bytes": bytes8, "launches_per_layer": 7,
-                           "path": "q8_gemv_kernel: CUDA cores, warp per row (8-bit codes, 9 bits per weight)"}
+    lays = [lay8[7 * i:7 * i + 7] for i in range(4)]
+    ysl = [ys8[7 * i:7 * i + 7] for i in range(4)]
+
+    def q8_layers_batched():
+        for l, ys in zip(lays, ysl):
+            q4.q8_matmul_batch([(x_down if p.K == 11264 else x, c, s, b, y) for (p, c, s, b), y in zip(l, ys)])
+
+    n0 = q4.q4_debug_launch_count()
+    q8_layers_batched()
+    launches8 = (q4.q4_debug_launch_count() - n0) / 4
+    ms8b = _graph_ms(dev, q8_layers_batched, 50) / 4
+    rows["q8_layer_M1"] = {"us_per_layer": round(ms8b * 1e3, 2), "GBps": round(bytes8 / (ms8b * 1e-3) / 1e9, 1),
+                           "bytes": bytes8, "launches_per_layer": launches8,
+                           "single_calls_us_per_layer": round(ms8 * 1e3, 2),
+                           "single_calls_GBps": round(bytes8 / (ms8 * 1e-3) / 1e9, 1),
+                           "path": "gemv_kernel<8-bit rows>: bulk-copy ring, codes as exact fp32 in packed fp32 "
+                                   "FMAs (9 bits per weight); one q8_matmul_batch per layer, 'single_calls' = "
+                                   "one q8_matmul per projection"}
     del lay8
 
     # depformer: stacked [16 N, K] weights per projection, drawn and quantized on the GPU

@@ -320,11 +320,27 @@ Q4_API q4_status q8_dequantize(const uint8_t* codes, const q4_bf16* scales, cons
  * y [M, N] = x . w_hat^T with 8-bit codes: fp32 accumulation of exact
  * products (each code an exact fp32, x in fp32), bf16 output.  CUDA-core
  * GEMV for every M (activation rows in pairs; each pair reads the weights
- * once).  K <= 196608 (Q4_ERR_UNSUPPORTED above).
+ * once): the 4-bit calls' bulk-copy GEMV with 8-bit rows where K is a
+ * multiple of 256 and the scale and bias rows are 16-byte aligned (and K
+ * fits one team of lanes: K <= 22528 for one row, 12288 for a pair), a
+ * warp-per-row kernel otherwise.  K <= 196608 (Q4_ERR_UNSUPPORTED above).
  */
 Q4_API q4_status q8_matmul(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes,
                            const q4_bf16* scales, const q4_bf16* biases, int64_t N, int group,
                            q4_bf16* y, q4_stream_t stream);
+
+/*
+ * q8_matmul_batch -- independent 8-bit matmuls sharing M: q4_matmul_batch's
+ * descriptor array with 8-bit codes ([N, K] bytes) in `codes`, each computed
+ * exactly as q8_matmul computes it alone; the problems the bulk-copy GEMV
+ * takes share one launch (per activation-row pair size, up to 256 problems),
+ * the rest run one q8_matmul launch each.  No epilogue (Q4_ERR_UNSUPPORTED
+ * for a nonzero `epilogue` or `reserved`).  Validation covers every entry
+ * before anything is enqueued.  The pages describe no such entry point; it
+ * is the 4-bit batch call for the 8-bit variant.
+ */
+Q4_API q4_status q8_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int group,
+                                 q4_stream_t stream);
 
 /* Message for the calling thread's last non-OK status ("" if none). */
 Q4_API const char* q4_last_error(void);

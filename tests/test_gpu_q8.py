@@ -91,3 +91,39 @@ def test_q8_empty_sizes():
     e = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
     ce, se, be = q4.q8_quantize(e)
     assert ce.shape == (0, 64) and se.shape == (0, 2)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3])
+def test_q8_batch_matches_single_calls(M):
+    """q8_matmul_batch: the problems the bulk-copy GEMV takes (K a multiple
+    of 256) share a launch and come out bit-identical to their single calls;
+    a K = 96 problem runs on the warp-per-row kernel, also as alone."""
+    shapes = [(4096, 4096), (77, 1024), (1, 256), (300, 2816), (33, 11264), (9, 96), (1000, 4096)]
+    probs, singles = [], []
+    for t, (N, K) in enumerate(shapes):
+        c, s, b = q4.q8_quantize(workloads.weight(N, K, 85, t, device=DEV))
+        x = workloads.activation(M, K, 85, 50 + t, device=DEV)
+        probs.append((x, c, s, b, torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)))
+        singles.append(q4.q8_matmul(x, c, s, b))
+    n0 = q4.q4_debug_launch_count()
+    q4.q8_matmul_batch(probs)
+    launches = q4.q4_debug_launch_count() - n0
+    # one GEMV launch per activation-row pair size, and the K = 96 problem's own launches (one per pair)
+    assert launches == (2 if M != 3 else 4), launches
+    for (x, c, s, b, out), ref, (N, K) in zip(probs, singles, shapes):
+        assert torch.equal(out, ref), (N, K)
+    x, c, s, b, y = probs[4]
+    ref, absdot = oracle.q8_matmul_ref(bits(x), c.cpu().numpy(), bits(s), bits(b))
+    assert oracle.tolerance_ok(y.float().cpu().double().numpy(), ref, absdot).all()
+
+
+def test_q8_batch_refuses_epilogues():
+    W = workloads.weight(64, 256, 86, 0, device=DEV)
+    c, s, b = q4.q8_quantize(W)
+    x = workloads.activation(1, 256, 86, 1, device=DEV)
+    y = torch.empty((1, 64), dtype=torch.bfloat16, device=DEV)
+    d = q4.MatmulDesc(x.data_ptr(), c.data_ptr(), s.data_ptr(), b.data_ptr(), y.data_ptr(), 64, 256)
+    d.epilogue, d.r = q4.EPI_RESIDUAL, y.data_ptr()
+    arr = (q4.MatmulDesc * 1)(d)
+    import ctypes
+    assert q4.lib().q8_matmul_batch(ctypes.cast(arr, ctypes.c_void_p), 1, 1, 32, None) == 4  # Q4_ERR_UNSUPPORTED

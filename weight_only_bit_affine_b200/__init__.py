@@ -50,6 +50,7 @@ __all__ = [
     "q8_quantize",
     "q8_dequantize",
     "q8_matmul",
+    "q8_matmul_batch",
     "q4_device_status",
     "q4_check_device",
     "q4_debug_launch_count",
@@ -92,6 +93,7 @@ SIGNATURES = {
     "q8_quantize": (_INT, [_P, _I64, _I64, _INT, _P, _P, _P, _P]),
     "q8_dequantize": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),
     "q8_matmul": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _P, _P]),
+    "q8_matmul_batch": (_INT, [_P, _INT, _I64, _INT, _P]),
     "q4_last_error": (ctypes.c_char_p, []),
     "q4_device_status": (_INT, [_INT]),
     "q4_debug_launch_count": (ctypes.c_ulonglong, []),
@@ -495,6 +497,38 @@ def q8_matmul(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases
         _check(lib().q8_matmul(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(biases), N, group, _ptr(out),
                                _stream(x.device)))
     return out
+
+
+def q8_matmul_batch(problems, group: int = GROUP):
+    """Independent 8-bit matmuls sharing M, in as few launches as possible:
+    (x, codes, scales, biases, out) tuples with codes [N, K] uint8 (no
+    epilogue).  Returns the list of outputs."""
+    problems = list(problems)
+    if not problems:
+        return []
+    descs = (MatmulDesc * len(problems))()
+    M = dev = None
+    for i, prob in enumerate(problems):
+        if len(prob) != 5:
+            raise ValueError(f"problem {i}: (x, codes, scales, biases, out)")
+        x, codes, scales, biases, out = prob
+        _want(x, "x", torch.bfloat16, 2)
+        Mi, K = x.shape
+        _q8_shapes(codes, scales, biases, K)
+        if not (x.device == codes.device == scales.device == biases.device):
+            raise ValueError(f"problem {i}: all tensors must be on the same device")
+        if M is None:
+            M, dev = Mi, x.device
+        elif Mi != M or x.device != dev:
+            raise ValueError("all problems of a batch need the same M and device")
+        _want(out, "out", torch.bfloat16, 2)
+        if out.shape != (M, codes.shape[0]) or out.device != dev:
+            raise ValueError(f"out of problem {i} must be [{M}, {codes.shape[0]}] on {dev}")
+        descs[i] = MatmulDesc(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
+                              codes.shape[0], K)
+    with torch.cuda.device(dev):
+        _check(lib().q8_matmul_batch(ctypes.cast(descs, ctypes.c_void_p), len(problems), M, group, _stream(dev)))
+    return [p[4] for p in problems]
 
 
 def q4_device_status(clear: bool = False) -> int:

@@ -528,6 +528,39 @@ q4_status q8_matmul(const q4_bf16* x, int64_t M, int64_t K, const uint8_t* codes
   return from_cuda(launch_q8_matmul(a, reinterpret_cast<cudaStream_t>(stream), *dev), "q8_matmul launch");
 }
 
+q4_status q8_matmul_batch(const q4_matmul_desc* descs, int count, int64_t M, int group, q4_stream_t stream) {
+  if (count < 0) return fail(Q4_ERR_SHAPE, "q8_matmul_batch: negative count %d", count);
+  if (count == 0) return Q4_OK;
+  if (!descs) return fail(Q4_ERR_NULL, "q8_matmul_batch: NULL descriptor array");
+  std::vector<MatmulArgs> fast, rest;
+  for (int i = 0; i < count; ++i) {
+    const q4_matmul_desc& d = descs[i];
+    bool empty = false;
+    char who[48];
+    snprintf(who, sizeof who, "q8_matmul_batch[%d]", i);
+    q4_status st = check_matmul(who, d.x, M, d.K, d.codes, d.scales, d.biases, d.N, group, d.y, &empty);
+    if (st != Q4_OK) return st;
+    if (d.epilogue != Q4_EPI_NONE || d.reserved != 0)
+      return fail(Q4_ERR_UNSUPPORTED, "%s: 8-bit problems take no epilogue", who);
+    if (d.K > kQ8MaxK)
+      return fail(Q4_ERR_UNSUPPORTED, "%s: K = %lld above %lld", who, (long long)d.K, (long long)kQ8MaxK);
+    if (empty) continue;
+    const MatmulArgs a{d.x, d.codes, d.scales, d.biases, d.y, M, d.N, d.K};
+    (gemv8_supported(a) ? fast : rest).push_back(a);
+  }
+  const DeviceInfo* dev = nullptr;
+  q4_status st;
+  if ((st = check_device(&dev)) != Q4_OK) return st;
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (!fast.empty() &&
+      (st = from_cuda(launch_gemv8_batch(fast.data(), static_cast<int>(fast.size()), cs, *dev),
+                      "q8_matmul_batch launch")) != Q4_OK)
+    return st;
+  for (const MatmulArgs& a : rest)
+    if ((st = from_cuda(launch_q8_matmul(a, cs, *dev), "q8_matmul_batch launch")) != Q4_OK) return st;
+  return Q4_OK;
+}
+
 const char* q4_last_error(void) { return t_last_error; }
 
 unsigned long long q4_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -168,6 +168,10 @@ __device__ __forceinline__ void load_words_smem(const uint8_t* p, uint32_t (&wor
   if constexpr (WORDS == 4) {
     const uint4 v = *reinterpret_cast<const uint4*>(p);
     words[0] = v.x; words[1] = v.y; words[2] = v.z; words[3] = v.w;
+  } else if constexpr (WORDS == 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p), u = *reinterpret_cast<const uint4*>(p + 16);
+    words[0] = v.x; words[1] = v.y; words[2] = v.z; words[3] = v.w;
+    words[4] = u.x; words[5] = u.y; words[6] = u.z; words[7] = u.w;
   } else if constexpr (WORDS == 2) {
     const uint2 v = *reinterpret_cast<const uint2*>(p);
     words[0] = v.x; words[1] = v.y;
@@ -212,11 +216,14 @@ constexpr int kFewProblems = 4;
 #ifndef Q4_GEMV_RPT
 #define Q4_GEMV_RPT 4
 #endif
-constexpr int kRpt = Q4_GEMV_RPT;  // weight rows per team per tile
+constexpr int kRpt = Q4_GEMV_RPT;  // weight rows per team per tile (4-bit codes)
+// 8-bit codes (q8_matmul): a row is twice the bytes, so a team takes two
+// rows per tile and a tile stays near the 4-bit one's size.
+constexpr int kRpt8 = 2;
 
 struct GemvProblem {
   const uint16_t* x;       // [MR, K]
-  const uint8_t* codes;    // [N, K/2]
+  const uint8_t* codes;    // [N, K/2] (4-bit codes) or [N, K] (8-bit)
   const uint16_t* scales;  // [N, K/32]
   const uint16_t* biases;  // [N, K/32]
   uint16_t* y;             // [MR, y_ld]
@@ -276,7 +283,7 @@ struct Geometry {
   int wpt;    // warps per team (0 when a warp holds several teams)
   int rt;     // rows per tile
 };
-__host__ __device__ inline Geometry geometry_of(int K, int consumer_threads) {
+__host__ __device__ inline Geometry geometry_of(int K, int consumer_threads, int bits = 4) {
   Geometry g;
   g.G = K / 32;
   if (g.G >= 32) {
@@ -287,14 +294,18 @@ __host__ __device__ inline Geometry geometry_of(int K, int consumer_threads) {
   }
   g.teams = consumer_threads / g.team;
   g.wpt = g.team >= 32 ? g.team / 32 : 0;
-  g.rt = g.teams * kRpt;
+  g.rt = g.teams * (bits == 4 ? kRpt : kRpt8);
   return g;
 }
-__host__ __device__ inline int64_t packed_row_bytes(int K) { return K / 2 + (K / 32) * 4; }
+// Code bytes of a weight row, and its packed bytes (codes, scales, biases).
+__host__ __device__ inline int code_row_bytes(int K, int bits) { return bits == 4 ? K / 2 : K; }
+__host__ __device__ inline int64_t packed_row_bytes(int K, int bits = 4) {
+  return code_row_bytes(K, bits) + (K / 32) * 4;
+}
 __host__ __device__ inline bool is_fused(const GemvProblem& P) { return P.up_codes != nullptr; }
 // Packed bytes per output row (gate + up when fused).
-__host__ __device__ inline int64_t problem_row_bytes(const GemvProblem& P) {
-  return packed_row_bytes(P.K) * (is_fused(P) ? 2 : 1);
+__host__ __device__ inline int64_t problem_row_bytes(const GemvProblem& P, int bits = 4) {
+  return packed_row_bytes(P.K, bits) * (is_fused(P) ? 2 : 1);
 }
 // Does the problem's tile finish in the epilogue warp (sums across a team's
 // warps, or the pairing of gate and up rows)?
@@ -353,6 +364,37 @@ __device__ __forceinline__ float row_acc(const uint32_t (&words)[4], const XSlic
   return acc;
 }
 
+// The same for a row of 8-bit codes (eight words; byte i of word w is the
+// code of input 4w + i): each code becomes an exact fp32 -- the byte under
+// the exponent of 2^23, minus 2^23 -- and two at a time meet the lane's x
+// pairs (x[8v + t], x[8v + t + 4]), whose codes are byte t of words 2v and
+// 2v + 1, in one packed fp32 FMA.  The products are exact; no offset.
+__device__ __forceinline__ float row_acc8(const uint32_t (&words)[8], const XSlice<4, kMacMixedBf16>& xs) {
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float q0 = __uint_as_float(__byte_perm(words[2 * v], 0x4B000000u, 0x7540u | t));
+      float q1 = __uint_as_float(__byte_perm(words[2 * v + 1], 0x4B000000u, 0x7540u | t));
+      fadd2(q0, q1, -8388608.f, -8388608.f);
+      const uint32_t xp = xs.v[v][t][0];
+      ffma2(a0, a1, q0, q1, __uint_as_float(xp << 16), __uint_as_float(xp & 0xFFFF0000u));
+    }
+  return a0 + a1;
+}
+
+template <int BITS, int CW>
+__device__ __forceinline__ float row_acc_bits(const uint32_t (&words)[CW], const XSlice<4, Q4_GEMV_MAC>& xs,
+                                              uint32_t kmask, uint32_t kmagic) {
+  if constexpr (BITS == 4) {
+    return row_acc(words, xs, kmask, kmagic);
+  } else {
+    static_assert(Q4_GEMV_MAC == kMacMixedBf16, "8-bit rows use the bf16 pair layout of x");
+    return row_acc8(words, xs);
+  }
+}
+
 // The rows of problem `pi` that belong to this CTA's byte range [lo, hi) of
 // the concatenated list: [*r0, *r1).  A row belongs to the CTA whose range
 // holds its first packed byte, so each row of the list belongs to exactly one
@@ -360,11 +402,11 @@ __device__ __forceinline__ float row_acc(const uint32_t (&words)[4], const XSlic
 // the fixed reduction trees), so results do not depend on the split.
 // Returns false when the problem lies entirely after the range (the caller
 // stops scanning).
-template <bool EPI, int NP>
+template <bool EPI, int BITS, int NP>
 __device__ __forceinline__ bool segment_of(const GemvLaunch<NP>& L, int pi, int64_t lo, int64_t hi, int64_t* r0,
                                            int64_t* r1) {
   const GemvProblem& P = L.prob[pi];
-  const int64_t rb = packed_row_bytes(P.K) * (fused_k<EPI>(P) ? 2 : 1);
+  const int64_t rb = packed_row_bytes(P.K, BITS) * (fused_k<EPI>(P) ? 2 : 1);
   const int64_t pb = P.byte_begin, pe = pb + P.N * rb;
   *r0 = *r1 = 0;
   if (pb >= hi) return false;
@@ -377,11 +419,15 @@ __device__ __forceinline__ bool segment_of(const GemvLaunch<NP>& L, int pi, int6
   return true;
 }
 
-template <int MR, int MAXT, int NP, bool EPI, bool CHAIN>
+// BITS: 4-bit codes (two per byte) or 8-bit codes (q8_matmul).
+template <int MR, int MAXT, int NP, bool EPI, bool CHAIN, int BITS>
 __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ GemvLaunch<NP> L) {
   static_assert(!CHAIN || NP > kFewProblems, "chains use the large parameter block");
+  static_assert(BITS == 4 || BITS == 8, "code width");
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int V = kRpt * MR;
+  constexpr int RPT = BITS == 4 ? kRpt : kRpt8;  // rows per team per tile
+  constexpr int CW = BITS == 4 ? 4 : 8;          // code words per lane per row (32 codes)
+  constexpr int V = RPT * MR;
   constexpr int VP = pow2_at_least(V);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -444,18 +490,18 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         for (int cs = 0; cs < n_st && issued < L.stages; ++cs) {
         share(cs, lo, hi, pb, pe);
         for (int pi = pb; pi < pe && issued < L.stages; ++pi) {
-          if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
+          if (!segment_of<EPI, BITS>(L, pi, lo, hi, &r0, &r1)) break;
           const GemvProblem& P = L.prob[pi];
-          const Geometry geo = geometry_of(P.K, L.consumer_threads);
-          const int half_k = P.K >> 1;
+          const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
+          const int code_bytes = code_row_bytes(P.K, BITS);  // code bytes per row
           const int rtile = rtile_k<EPI>(P, geo);
           for (int64_t row0 = r0; row0 < r1 && issued < L.stages; row0 += rtile, ++issued) {
             const uint32_t rows = tile_rows(r1, row0, rtile);
-            bulk_prefetch_l2(P.codes + row0 * half_k, rows * half_k);
+            bulk_prefetch_l2(P.codes + row0 * code_bytes, rows * code_bytes);
             bulk_prefetch_l2(P.scales + row0 * geo.G, rows * geo.G * 2);
             bulk_prefetch_l2(P.biases + row0 * geo.G, rows * geo.G * 2);
             if (fused_k<EPI>(P)) {
-              bulk_prefetch_l2(P.up_codes + row0 * half_k, rows * half_k);
+              bulk_prefetch_l2(P.up_codes + row0 * code_bytes, rows * code_bytes);
               bulk_prefetch_l2(P.up_scales + row0 * geo.G, rows * geo.G * 2);
               bulk_prefetch_l2(P.up_biases + row0 * geo.G, rows * geo.G * 2);
             }
@@ -477,11 +523,11 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       share(cs, lo, hi, pb, pe);
       for (int pi = pb; pi < pe && !dead; ++pi) {
         int64_t r0, r1;
-        if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
+        if (!segment_of<EPI, BITS>(L, pi, lo, hi, &r0, &r1)) break;
         if (r0 >= r1) continue;
         const GemvProblem& P = L.prob[pi];
-        const Geometry geo = geometry_of(P.K, L.consumer_threads);
-        const int half_k = P.K >> 1;
+        const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
+        const int code_bytes = code_row_bytes(P.K, BITS);  // code bytes per row
         const int rtile = rtile_k<EPI>(P, geo);
         for (int64_t row0 = CHAIN ? r0 : r0 - rtile; row0 < r1; row0 += rtile) {  // a batch's first pass: x
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; *gave_up = 1u; break; }
@@ -496,16 +542,16 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
             // rows right after the gate rows in each of the three regions
             // (2 * rows <= rt, and every offset stays a multiple of 16 bytes).
             const uint32_t rows = tile_rows(r1, row0, rtile);
-            const uint32_t cb = rows * half_k, sb = rows * geo.G * 2;
-            const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
+            const uint32_t cb = rows * code_bytes, sb = rows * geo.G * 2;
+            const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * code_bytes;
             const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
             const bool fused = fused_k<EPI>(P);
             mbar_arrive_expect_tx(&full_bar[stage], (fused ? 2u : 1u) * (cb + 2 * sb));
-            bulk_g2s(st, P.codes + row0 * half_k, cb, &full_bar[stage]);
+            bulk_g2s(st, P.codes + row0 * code_bytes, cb, &full_bar[stage]);
             bulk_g2s(st + sb_off, P.scales + row0 * geo.G, sb, &full_bar[stage]);
             bulk_g2s(st + sb_off + sb_tile, P.biases + row0 * geo.G, sb, &full_bar[stage]);
             if (fused) {
-              bulk_g2s(st + cb, P.up_codes + row0 * half_k, cb, &full_bar[stage]);
+              bulk_g2s(st + cb, P.up_codes + row0 * code_bytes, cb, &full_bar[stage]);
               bulk_g2s(st + sb_off + sb, P.up_scales + row0 * geo.G, sb, &full_bar[stage]);
               bulk_g2s(st + sb_off + sb_tile + sb, P.up_biases + row0 * geo.G, sb, &full_bar[stage]);
             }
@@ -554,9 +600,9 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     share(cs, lo, hi, pb, pe);
     for (int pi = pb; pi < pe; ++pi) {
       int64_t r0, r1;
-      if (!segment_of<EPI>(L, pi, lo, hi, &r0, &r1)) break;
+      if (!segment_of<EPI, BITS>(L, pi, lo, hi, &r0, &r1)) break;
       const GemvProblem& P = L.prob[pi];
-      const Geometry geo = geometry_of(P.K, L.consumer_threads);
+      const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
       if (!epilogue_warp_k<EPI>(P, geo)) continue;
       const int rtile = rtile_k<EPI>(P, geo);
       const bool fused = fused_k<EPI>(P);
@@ -607,21 +653,21 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   share(cs, lo, hi, pb, pe);
   for (int pi = pb; pi < pe; ++pi) {
     int64_t r_begin, r_end;
-    if (!segment_of<EPI>(L, pi, lo, hi, &r_begin, &r_end)) break;
+    if (!segment_of<EPI, BITS>(L, pi, lo, hi, &r_begin, &r_end)) break;
     if (r_begin >= r_end) continue;
     const GemvProblem& P = L.prob[pi];
-    const Geometry geo = geometry_of(P.K, L.consumer_threads);
-    const int half_k = P.K >> 1;
+    const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
+    const int code_bytes = code_row_bytes(P.K, BITS);  // code bytes per row
     const int team_idx = tid / geo.team;
     const int j = tid - team_idx * geo.team;
     const bool active = team_idx < geo.teams && j < geo.G;
     const int warp_in_team = (geo.team >= 32) ? (j >> 5) : 0;
-    const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * half_k;
+    const uint32_t sb_off = static_cast<uint32_t>(geo.rt) * code_bytes;
     const uint32_t sb_tile = (static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u;
     // Byte offsets inside a stage of this lane's first row (row team_idx) and
     // the step to its next row (teams rows further).
-    const uint32_t code_off0 = static_cast<uint32_t>(team_idx) * half_k + j * 16;
-    const uint32_t code_step = static_cast<uint32_t>(geo.teams) * half_k;
+    const uint32_t code_off0 = static_cast<uint32_t>(team_idx) * code_bytes + j * (4 * CW);
+    const uint32_t code_step = static_cast<uint32_t>(geo.teams) * code_bytes;
     const uint32_t sc_off0 = sb_off + (static_cast<uint32_t>(team_idx) * geo.G + j) * 2;
     const uint32_t sc_step = static_cast<uint32_t>(geo.teams) * geo.G * 2;
 
@@ -660,7 +706,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 
     const bool use_red = epilogue_warp_k<EPI>(P, geo);
     const int rtile = rtile_k<EPI>(P, geo);
-    constexpr float kOffset = mac_offset<Q4_GEMV_MAC>();
+    constexpr float kOffset = BITS == 4 ? mac_offset<Q4_GEMV_MAC>() : 0.f;
 
     for (int64_t row0 = r_begin; row0 < r_end; row0 += rtile) {
       if (!dead && !mbar_wait(&full_bar[stage], phase)) { dead = true; *gave_up = 1u; }
@@ -673,24 +719,24 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       const int tile_out = static_cast<int>((r_end - row0 < rtile) ? (r_end - row0) : rtile);
       const int tile_n = fused_k<EPI>(P) ? 2 * tile_out : tile_out;
       const int nv = (team_idx >= geo.teams || team_idx >= tile_n) ? 0
-                     : (tile_n == geo.rt)                          ? kRpt
+                     : (tile_n == geo.rt)                          ? RPT
                                                                    : (tile_n - team_idx + geo.teams - 1) / geo.teams;
       float vals[VP];
 #pragma unroll
       for (int i = 0; i < VP; ++i) vals[i] = 0.f;
       bool compute = true;
 
-      if (geo.team >= 32 && nv == kRpt) {
+      if (geo.team >= 32 && nv == RPT) {
         // Fast path: every row of this team is present (warp-uniform).
         // Lanes past G (padding) read in-stage bytes but take s = b = 0 and
         // a zero x slice, so they add exactly nothing.
-        uint32_t words[kRpt][4];
-        float sc[kRpt], bi[kRpt];
+        uint32_t words[RPT][CW];
+        float sc[RPT], bi[RPT];
         const uint8_t* cp = st + code_off0;
         const uint8_t* sp = st + sc_off0;
 #pragma unroll
-        for (int rr = 0; rr < kRpt; ++rr) {
-          load_words_smem<4>(cp + rr * code_step, words[rr]);
+        for (int rr = 0; rr < RPT; ++rr) {
+          load_words_smem<CW>(cp + rr * code_step, words[rr]);
           const uint16_t sh = *reinterpret_cast<const uint16_t*>(sp + rr * sc_step);
           const uint16_t bh = *reinterpret_cast<const uint16_t*>(sp + rr * sc_step + sb_tile);
           sc[rr] = active ? bf16_bits_to_float(sh) : 0.f;
@@ -700,25 +746,25 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         if (lane == 0) mbar_arrive(&empty_bar[stage]);
         if (++stage == L.stages) { stage = 0; phase ^= 1u; }
 #pragma unroll
-        for (int rr = 0; rr < kRpt; ++rr) {
+        for (int rr = 0; rr < RPT; ++rr) {
           const float c = fmaf(-kOffset, sc[rr], bi[rr]);
 #pragma unroll
           for (int m = 0; m < MR; ++m)
-            vals[rr * MR + m] = fmaf(sc[rr], row_acc(words[rr], xsl[m], kmask, kmagic), c * xsl[m].sum);
+            vals[rr * MR + m] = fmaf(sc[rr], row_acc_bits<BITS>(words[rr], xsl[m], kmask, kmagic), c * xsl[m].sum);
         }
       } else {
-        uint32_t words[kRpt][4];
-        float sc[kRpt], bi[kRpt];
+        uint32_t words[RPT][CW];
+        float sc[RPT], bi[RPT];
         const bool lane_on = active && nv > 0;
 #pragma unroll
-        for (int rr = 0; rr < kRpt; ++rr) {  // all shared-memory loads first
+        for (int rr = 0; rr < RPT; ++rr) {  // all shared-memory loads first
           if (lane_on && rr < nv) {
-            load_words_smem<4>(st + code_off0 + rr * code_step, words[rr]);
+            load_words_smem<CW>(st + code_off0 + rr * code_step, words[rr]);
             sc[rr] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + sc_off0 + rr * sc_step));
             bi[rr] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + sc_off0 + rr * sc_step + sb_tile));
           } else {
 #pragma unroll
-            for (int w = 0; w < 4; ++w) words[rr][w] = 0u;
+            for (int w = 0; w < CW; ++w) words[rr][w] = 0u;
             sc[rr] = bi[rr] = 0.f;
           }
         }
@@ -731,12 +777,12 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
           compute = false;  // a whole idle warp
         } else {
 #pragma unroll
-          for (int rr = 0; rr < kRpt; ++rr) {
+          for (int rr = 0; rr < RPT; ++rr) {
             if (geo.team >= 32 && rr >= nv) break;  // warp-uniform
             const float c = fmaf(-kOffset, sc[rr], bi[rr]);
 #pragma unroll
             for (int m = 0; m < MR; ++m)
-              vals[rr * MR + m] = fmaf(sc[rr], row_acc(words[rr], xsl[m], kmask, kmagic), c * xsl[m].sum);
+              vals[rr * MR + m] = fmaf(sc[rr], row_acc_bits<BITS>(words[rr], xsl[m], kmask, kmagic), c * xsl[m].sum);
           }
         }
       }
@@ -769,7 +815,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         for (int i = 0; i < V; ++i) vals[i] = seg_allreduce_dyn(vals[i], geo.team);
         if (j == 0) {
 #pragma unroll
-          for (int rr = 0; rr < kRpt; ++rr)
+          for (int rr = 0; rr < RPT; ++rr)
             if (rr < nv) {
               const int64_t row = row0 + team_idx + rr * geo.teams;
 #pragma unroll
@@ -900,13 +946,13 @@ constexpr int kConsumers2 = Q4_GEMV_CONSUMERS2, kThreads2 = kConsumers2 + 64;  /
 int consumers_for(int mr) { return mr == 1 ? kConsumers1 : kConsumers2; }
 
 // Does the bulk-copy kernel take this problem (else: the generic kernel)?
-bool tma_ok(const MatmulArgs& a, int mr) {
+bool tma_ok(const MatmulArgs& a, int mr, int bits = 4) {
   const int64_t G = a.K / 32;
   if (G % 8 != 0) return false;  // scale rows must be whole 16-byte runs for bulk copies
   uintptr_t sb = reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases);
   if (a.fused()) sb |= reinterpret_cast<uintptr_t>(a.up_scales) | reinterpret_cast<uintptr_t>(a.up_biases);
   if (sb & 15u) return false;
-  const Geometry geo = geometry_of(static_cast<int>(a.K), consumers_for(mr));
+  const Geometry geo = geometry_of(static_cast<int>(a.K), consumers_for(mr), bits);
   // A fused tile pairs gate and up rows in the epilogue warp, which needs
   // teams of whole warps.
   if (a.fused() && geo.team < 32) return false;
@@ -938,9 +984,10 @@ cudaError_t run_generic(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, 
 // Grows *stage_bytes to hold a tile of P (and, with_x, its activation block
 // [MR, K]); false if the epilogue warp's reduction slots cannot take P's
 // tiles (they are sized for kConsumers1 / kConsumers2).
-bool ring_stage_fits(const GemvProblem& P, int mr, int consumers, bool with_x, uint32_t& stage_bytes) {
-  const Geometry geo = geometry_of(P.K, consumers);
-  const uint32_t tile = static_cast<uint32_t>(geo.rt) * (P.K / 2) +
+bool ring_stage_fits(const GemvProblem& P, int mr, int consumers, bool with_x, uint32_t& stage_bytes,
+                     int bits = 4) {
+  const Geometry geo = geometry_of(P.K, consumers, bits);
+  const uint32_t tile = static_cast<uint32_t>(geo.rt) * code_row_bytes(P.K, bits) +
                         2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
   stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
   if (with_x) stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(mr) * P.K * 2 + 127u) & ~127u);
@@ -960,7 +1007,7 @@ bool ring_of(uint32_t stage_bytes, const DeviceInfo& dev, int* stages, size_t* s
 
 // Launches the bulk-copy kernel over `count` problems of `probs` (all taking
 // this path, all with MR activation rows).
-template <int MR, int NP>
+template <int MR, int NP, int BITS = 4>
 cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev, cudaStream_t stream) {
   constexpr int kThreads = MR == 1 ? kThreads1 : kThreads2;
   const int consumers = consumers_for(MR);
@@ -970,10 +1017,10 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   int64_t total = 0;
   for (int i = 0; i < count; ++i) {
     const GemvProblem& P = probs[i];
-    if (!ring_stage_fits(P, MR, consumers, true, stage_bytes)) return cudaErrorInvalidConfiguration;
+    if (!ring_stage_fits(P, MR, consumers, true, stage_bytes, BITS)) return cudaErrorInvalidConfiguration;
     L.prob[i] = P;
     L.prob[i].byte_begin = total;
-    total += P.N * problem_row_bytes(P);
+    total += P.N * problem_row_bytes(P, BITS);
   }
   int stages = 0;
   size_t smem = 0;
@@ -992,12 +1039,12 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   int pi = 0;
   for (int c = 0; c < grid && NP > kFewProblems; ++c) {
     const int64_t lo = static_cast<int64_t>(c) * total / grid;
-    while (pi < count && L.prob[pi].byte_begin + L.prob[pi].N * problem_row_bytes(L.prob[pi]) <= lo) ++pi;
+    while (pi < count && L.prob[pi].byte_begin + L.prob[pi].N * problem_row_bytes(L.prob[pi], BITS) <= lo) ++pi;
     L.first[c] = static_cast<uint16_t>(pi);
   }
   bool epi = false;
   for (int i = 0; i < count; ++i) epi = epi || probs[i].epi != kEpiNone || is_fused(probs[i]);
-  auto kern = epi ? gemv_kernel<MR, kThreads, NP, true, false> : gemv_kernel<MR, kThreads, NP, false, false>;
+  auto kern = epi ? gemv_kernel<MR, kThreads, NP, true, false, BITS> : gemv_kernel<MR, kThreads, NP, false, false, BITS>;
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, L);
 }
 
@@ -1043,7 +1090,7 @@ cudaError_t run_chain(const GemvProblem* probs, int count, const int* stage_coun
   L.n_stages = n_stages;
   L.done = done;
   const int grid = std::min(dev.sm_count, kMaxCtas);
-  auto kern = epi ? gemv_kernel<MR, kThreads, NP, true, true> : gemv_kernel<MR, kThreads, NP, false, true>;
+  auto kern = epi ? gemv_kernel<MR, kThreads, NP, true, true, 4> : gemv_kernel<MR, kThreads, NP, false, true, 4>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
@@ -1059,12 +1106,12 @@ cudaError_t run_chain(const GemvProblem* probs, int count, const int* stage_coun
 }
 
 // Launches in groups of at most kMaxProblems problems.
-template <int MR>
+template <int MR, int BITS = 4>
 cudaError_t run_problems(std::vector<GemvProblem>& probs, const DeviceInfo& dev, cudaStream_t stream) {
   for (size_t i = 0; i < probs.size(); i += kMaxProblems) {
     const int n = static_cast<int>(std::min<size_t>(kMaxProblems, probs.size() - i));
-    cudaError_t e = (n <= kFewProblems) ? run_list<MR, kFewProblems>(probs.data() + i, n, dev, stream)
-                                        : run_list<MR, kMaxProblems>(probs.data() + i, n, dev, stream);
+    cudaError_t e = (n <= kFewProblems) ? run_list<MR, kFewProblems, BITS>(probs.data() + i, n, dev, stream)
+                                        : run_list<MR, kMaxProblems, BITS>(probs.data() + i, n, dev, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -1075,18 +1122,26 @@ cudaError_t run_problems(std::vector<GemvProblem>& probs, const DeviceInfo& dev,
 cudaError_t gemv_device_flags(unsigned int* flags, bool clear) { return tu_device_flags(flags, clear); }
 
 cudaError_t gemv_prepare_device(const DeviceInfo& dev) {
-  for (const void* kern : {reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, false, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, true, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false, true>),
-                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true, true>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, false, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, true, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true, false>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false, true>),
-                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true, true>)}) {
+  for (const void* kern : {reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, false, false, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, true, false, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false, false, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true, false, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false, true, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true, true, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, false, false, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, true, false, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false, false, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true, false, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false, true, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true, true, 4>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, false, false, 8>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kFewProblems, true, false, 8>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, false, false, 8>),
+                           reinterpret_cast<const void*>(gemv_kernel<1, kThreads1, kMaxProblems, true, false, 8>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, false, false, 8>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kFewProblems, true, false, 8>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, false, false, 8>),
+                           reinterpret_cast<const void*>(gemv_kernel<2, kThreads2, kMaxProblems, true, false, 8>)}) {
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dev.smem_optin));
     if (e != cudaSuccess) return e;
@@ -1133,6 +1188,42 @@ cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t st
 
 cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev) {
   return launch_gemv_batch(&a, 1, stream, dev);
+}
+
+bool gemv8_supported(const MatmulArgs& a) {
+  if (a.fused() || a.epi != kEpiNone) return false;
+  for (int mr = 1; mr <= 2 && mr <= a.M; ++mr)
+    if (!tma_ok(a, mr, 8)) return false;
+  return true;
+}
+
+cudaError_t launch_gemv8_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev) {
+  std::vector<GemvProblem> one, two;
+  for (int i = 0; i < count; ++i) {
+    const MatmulArgs& a = list[i];
+    for (int64_t m0 = 0; m0 < a.M; m0 += 2) {
+      GemvProblem P;
+      P.x = a.x + m0 * a.K;
+      P.codes = a.codes;
+      P.scales = a.scales;
+      P.biases = a.biases;
+      P.y = a.y + m0 * a.N;
+      P.r = nullptr;
+      P.up_codes = nullptr;
+      P.up_scales = nullptr;
+      P.up_biases = nullptr;
+      P.N = a.N;
+      P.y_ld = a.N;
+      P.K = static_cast<int32_t>(a.K);
+      P.epi = kEpiNone;
+      P.byte_begin = 0;
+      (a.M - m0 >= 2 ? two : one).push_back(P);
+    }
+  }
+  cudaError_t e = cudaSuccess;
+  if (!two.empty()) e = run_problems<2, 8>(two, dev, stream);
+  if (e == cudaSuccess && !one.empty()) e = run_problems<1, 8>(one, dev, stream);
+  return e;
 }
 
 bool gemv_chain_supported(const MatmulArgs* list, int count) {

@@ -79,6 +79,12 @@ cudaError_t launch_gemv(const MatmulArgs& a, cudaStream_t stream, const DeviceIn
 // Several independent matmuls; those the bulk-copy kernel takes share one
 // launch (per chunk size).
 cudaError_t launch_gemv_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
+// 8-bit codes (q8_matmul, q8_matmul_batch) on the same bulk-copy GEMV:
+// whether it takes a problem (no epilogue, K a multiple of 256, 16-byte
+// aligned scale rows), and the launch of a list of such problems (activation
+// rows in pairs; all pairs of one size share a launch of up to 256).
+bool gemv8_supported(const MatmulArgs& a);
+cudaError_t launch_gemv8_batch(const MatmulArgs* list, int count, cudaStream_t stream, const DeviceInfo& dev);
 // A chain of dependent stages in one persistent launch (q4_matmul_chain):
 // whether it takes `list` (one or two activation rows, every problem on the
 // bulk-copy path), and the launch itself -- stage s is the next

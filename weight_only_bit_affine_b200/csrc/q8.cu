@@ -9,8 +9,11 @@
 // clamped to 0..255; one byte per code, codes [N, K]; scales and biases
 // [N, K/32] bf16; w_hat = scale * q + bias.
 //
-// The matmul is a CUDA-core GEMV (one warp per weight row, lanes over the
-// row's groups; activation rows in chunks of two).  At 1.125 bytes per weight
+// The matmul runs on the bulk-copy GEMV of q4_gemv.cu (8-bit rows: a lane's
+// 32 codes become exact fp32 values meeting its x pairs in packed fp32 FMAs)
+// where that kernel takes the problem (K a multiple of 256, 16-byte aligned
+// scale rows); otherwise on the kernel below, a CUDA-core GEMV (one warp per
+// weight row, lanes over the row's groups; activation rows in chunks of two).  At 1.125 bytes per weight
 // an HBM-bound pass needs 1.8x fewer weights per second than the 4-bit one,
 // so the arithmetic per weight can be heavier: each code becomes an exact
 // fp32 (the byte under the exponent of 2^23, minus 2^23) and meets an fp32
@@ -236,6 +239,9 @@ cudaError_t launch_q8_dequantize(const uint8_t* codes, const uint16_t* scales, c
 }
 
 cudaError_t launch_q8_matmul(const MatmulArgs& a, cudaStream_t stream, const DeviceInfo& dev) {
+  // The bulk-copy GEMV (q4_gemv.cu, 8-bit rows) where it takes the problem;
+  // this file's warp-per-row kernel otherwise.
+  if (gemv8_supported(a)) return launch_gemv8_batch(&a, 1, stream, dev);
   for (int64_t m0 = 0; m0 < a.M; m0 += 2) {
     const cudaError_t e = (a.M - m0 >= 2) ? run_q8_gemv<2>(a, m0, dev, stream) : run_q8_gemv<1>(a, m0, dev, stream);
     if (e != cudaSuccess) return e;
