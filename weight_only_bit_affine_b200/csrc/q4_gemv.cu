@@ -180,6 +180,20 @@ __device__ __forceinline__ void load_words_smem(const uint8_t* p, uint32_t (&wor
   }
 }
 
+// A lane's code words of one row: 4-bit rows as load_words_smem; 8-bit rows
+// (two 16-byte chunks) with the chunks in swapped order when swz is set.
+template <int CW>
+__device__ __forceinline__ void load_code_words(const uint8_t* p, bool swz, uint32_t (&words)[CW]) {
+  if constexpr (CW == 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p + (swz ? 16 : 0));
+    const uint4 u = *reinterpret_cast<const uint4*>(p + (swz ? 0 : 16));
+    words[0] = v.x; words[1] = v.y; words[2] = v.z; words[3] = v.w;
+    words[4] = u.x; words[5] = u.y; words[6] = u.z; words[7] = u.w;
+  } else {
+    load_words_smem<CW>(p, words);
+  }
+}
+
 // Sum V values across the 32 lanes of a warp at once (V a power of two):
 // after the call, lane l holds the total of value l >> (5 - log2 V).  Costs
 // V - 1 + 5 - log2 V shuffles instead of 5 V.
@@ -704,6 +718,23 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       if (++stage == L.stages) { stage = 0; phase ^= 1u; }
     }
 
+    // 8-bit rows: a lane's 32 codes are two 16-byte chunks 32 bytes apart
+    // from the next lane's; lanes 4..7 of every eight read their second chunk
+    // first, so each quarter-warp load covers 128 distinct bytes (no bank
+    // conflict), and their x slices swap halves to match.
+    const bool swz = BITS == 8 && ((lane >> 2) & 1);
+    if constexpr (BITS == 8) {
+#pragma unroll
+      for (int m = 0; m < MR; ++m)
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const uint32_t a = xsl[m].v[w][t][0], b = xsl[m].v[w + 2][t][0];
+            xsl[m].v[w][t][0] = swz ? b : a;
+            xsl[m].v[w + 2][t][0] = swz ? a : b;
+          }
+    }
     const bool use_red = epilogue_warp_k<EPI>(P, geo);
     const int rtile = rtile_k<EPI>(P, geo);
     constexpr float kOffset = BITS == 4 ? mac_offset<Q4_GEMV_MAC>() : 0.f;
@@ -736,7 +767,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         const uint8_t* sp = st + sc_off0;
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr) {
-          load_words_smem<CW>(cp + rr * code_step, words[rr]);
+          load_code_words<CW>(cp + rr * code_step, swz, words[rr]);
           const uint16_t sh = *reinterpret_cast<const uint16_t*>(sp + rr * sc_step);
           const uint16_t bh = *reinterpret_cast<const uint16_t*>(sp + rr * sc_step + sb_tile);
           sc[rr] = active ? bf16_bits_to_float(sh) : 0.f;
@@ -759,7 +790,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr) {  // all shared-memory loads first
           if (lane_on && rr < nv) {
-            load_words_smem<CW>(st + code_off0 + rr * code_step, words[rr]);
+            load_code_words<CW>(st + code_off0 + rr * code_step, swz, words[rr]);
             sc[rr] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + sc_off0 + rr * sc_step));
             bi[rr] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + sc_off0 + rr * sc_step + sb_tile));
           } else {
