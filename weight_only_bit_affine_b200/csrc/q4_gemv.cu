@@ -11,14 +11,14 @@
 // One launch runs a LIST of independent matmuls ("problems"): the temporal
 // step's projections, or a single q4_matmul.  Design (bandwidth-bound at
 // ~1.6 flop per packed byte):
-//  * One persistent CTA per SM takes a balanced contiguous share of the rows
-//    of every problem in turn.  A producer warp streams those rows (codes,
-//    scales, biases: contiguous byte ranges) through a ring of shared-memory
-//    stages with 1-D bulk (TMA) copies; each problem's activations travel
-//    through the same ring just ahead of its tiles, so the ring never drains
-//    between problems and the next problem's inputs arrive early.
+//  * One persistent CTA per SM takes a balanced contiguous share of the
+//    list's packed bytes (its rows of every problem in turn).  A producer
+//    warp streams those rows (codes, scales, biases: contiguous byte ranges)
+//    through a ring of shared-memory stages with 1-D bulk (TMA) copies, so
+//    the ring never drains between problems.
 //  * Consumer threads form "teams" of K/32 lanes; a team owns one weight row
-//    at a time and lane j always covers input group j, so its slice of x sits
+//    at a time and lane j always covers input group j, so its slice of x
+//    (read once per problem from global memory, L1 shared by the teams) sits
 //    in registers for the whole problem.  Each warp sums its lanes with a
 //    transpose-reduce; the sums across a team's warps are finished by an
 //    epilogue warp behind mbarriers, so consumers never block on each other.
@@ -264,7 +264,7 @@ struct GemvLaunch {
   int count;
   int consumer_threads;  // a multiple of 32
   int stages;
-  uint32_t stage_bytes;  // >= every problem's tile and activation block, 128-byte multiple
+  uint32_t stage_bytes;  // >= every problem's tile, 128-byte multiple
   int64_t total_bytes;   // packed bytes of the whole list (a batch launch)
   // A chain launch: stages run in order, stage s being the problems
   // [stage_begin[s], stage_begin[s + 1]) split over all CTAs like a batch of
@@ -524,10 +524,9 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         }
       }
       pdl_wait_predecessors();
-      // Ring order per segment: its activation block [MR, K] (a batch; a
-      // chain's consumers read theirs from global memory once the stage's
-      // inputs are complete), then its tiles.  The producer never waits for
-      // other CTAs: across a chain's stages it streams weights ahead.
+      // The ring carries weight tiles only (the consumers read their
+      // activations from global memory); the producer never waits for other
+      // CTAs: across a chain's stages it streams weights ahead.
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool dead = false;
@@ -543,14 +542,10 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
         const int code_bytes = code_row_bytes(P.K, BITS);  // code bytes per row
         const int rtile = rtile_k<EPI>(P, geo);
-        for (int64_t row0 = CHAIN ? r0 : r0 - rtile; row0 < r1; row0 += rtile) {  // a batch's first pass: x
+        for (int64_t row0 = r0; row0 < r1; row0 += rtile) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) { dead = true; *gave_up = 1u; break; }
           uint8_t* st = smem + static_cast<size_t>(stage) * L.stage_bytes;
-          if (row0 < r0) {
-            const uint32_t xbytes = static_cast<uint32_t>(MR) * P.K * 2;
-            mbar_arrive_expect_tx(&full_bar[stage], xbytes);
-            bulk_g2s(st, P.x, xbytes, &full_bar[stage]);
-          } else {
+          {
             // Stage layout: codes of the tile's rows from 0, scales from
             // sb_off, biases from sb_off + sb_tile; a fused tile puts the up
             // rows right after the gate rows in each of the three regions
@@ -685,37 +680,21 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     const uint32_t sc_off0 = sb_off + (static_cast<uint32_t>(team_idx) * geo.G + j) * 2;
     const uint32_t sc_step = static_cast<uint32_t>(geo.teams) * geo.G * 2;
 
-    // Activations: this lane's 32 inputs of each row, from the ring stage
-    // that precedes the segment's tiles (a batch) or from global memory (a
-    // chain).
+    // Activations: this lane's 32 inputs of each row, read from global memory
+    // with plain loads once the launch's inputs are complete (after the
+    // programmatic-dependent-launch wait; in a chain, after the stage barrier:
+    // an acquire at GPU scope, then the go barrier).  The teams after the
+    // first hit in L1.  (Sending them through the ring ahead of the tiles
+    // took a stage per segment and was 2 % slower on the stream; in a chain a
+    // read through L2 per team, or staging in shared memory at the cost of a
+    // ring stage, were slower too.)
     XSlice<4, Q4_GEMV_MAC> xsl[MR];
-    if constexpr (CHAIN) {
-      // Plain loads: this CTA passed the stage barrier (an acquire at GPU
-      // scope, then the go barrier), after which every write of the earlier
-      // stages is visible to them; the teams after the first hit in L1
-      // (a read through L2 per team, or staging the block in shared memory
-      // at the cost of a ring stage, were both slower).
-      const uint16_t* xsrc = P.x;
 #pragma unroll
-      for (int m = 0; m < MR; ++m) {
-        if (active)
-          xsl[m].load(xsrc + m * P.K + j * 32);
-        else
-          xsl[m].zero();
-      }
-    } else {
-      if (!dead && !mbar_wait(&full_bar[stage], phase)) { dead = true; *gave_up = 1u; }
-      const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(smem + static_cast<size_t>(stage) * L.stage_bytes);
-#pragma unroll
-      for (int m = 0; m < MR; ++m) {
-        if (active)
-          xsl[m].load(xsrc + m * P.K + j * 32);
-        else
-          xsl[m].zero();
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[stage]);
-      if (++stage == L.stages) { stage = 0; phase ^= 1u; }
+    for (int m = 0; m < MR; ++m) {
+      if (active)
+        xsl[m].load(P.x + m * P.K + j * 32);
+      else
+        xsl[m].zero();
     }
 
     // 8-bit rows: a lane's 32 codes are two 16-byte chunks 32 bytes apart
@@ -1012,16 +991,14 @@ cudaError_t run_generic(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, 
   return launch_pdl(gemv_generic_kernel<MR>, dim3(grid), dim3(256), 0, stream, p);
 }
 
-// Grows *stage_bytes to hold a tile of P (and, with_x, its activation block
-// [MR, K]); false if the epilogue warp's reduction slots cannot take P's
-// tiles (they are sized for kConsumers1 / kConsumers2).
-bool ring_stage_fits(const GemvProblem& P, int mr, int consumers, bool with_x, uint32_t& stage_bytes,
-                     int bits = 4) {
+// Grows *stage_bytes to hold a tile of P; false if the epilogue warp's
+// reduction slots cannot take P's tiles (they are sized for kConsumers1 /
+// kConsumers2).
+bool ring_stage_fits(const GemvProblem& P, int mr, int consumers, uint32_t& stage_bytes, int bits = 4) {
   const Geometry geo = geometry_of(P.K, consumers, bits);
   const uint32_t tile = static_cast<uint32_t>(geo.rt) * code_row_bytes(P.K, bits) +
                         2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
   stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
-  if (with_x) stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(mr) * P.K * 2 + 127u) & ~127u);
   return !(uses_epilogue_warp(P, geo) && geo.rt * mr * geo.wpt > kRedSlotFloats);
 }
 
@@ -1048,7 +1025,7 @@ cudaError_t run_list(const GemvProblem* probs, int count, const DeviceInfo& dev,
   int64_t total = 0;
   for (int i = 0; i < count; ++i) {
     const GemvProblem& P = probs[i];
-    if (!ring_stage_fits(P, MR, consumers, true, stage_bytes, BITS)) return cudaErrorInvalidConfiguration;
+    if (!ring_stage_fits(P, MR, consumers, stage_bytes, BITS)) return cudaErrorInvalidConfiguration;
     L.prob[i] = P;
     L.prob[i].byte_begin = total;
     total += P.N * problem_row_bytes(P, BITS);
@@ -1100,7 +1077,7 @@ cudaError_t run_chain(const GemvProblem* probs, int count, const int* stage_coun
     for (int k = 0; k < stage_counts[s]; ++k, ++i) {
       if (i >= count) return cudaErrorInvalidValue;
       const GemvProblem& P = probs[i];
-      if (!ring_stage_fits(P, MR, consumers, false, stage_bytes)) return cudaErrorInvalidConfiguration;
+      if (!ring_stage_fits(P, MR, consumers, stage_bytes)) return cudaErrorInvalidConfiguration;
       L.prob[i] = P;
       L.prob[i].byte_begin = total;
       total += P.N * problem_row_bytes(P);
