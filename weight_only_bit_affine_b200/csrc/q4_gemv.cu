@@ -227,10 +227,21 @@ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
 // (a small instance for single calls, a large one for batches).
 constexpr int kMaxProblems = 256;
 constexpr int kFewProblems = 4;
-#ifndef Q4_GEMV_RPT
-#define Q4_GEMV_RPT 4
+// Weight rows per team per tile (4-bit codes), for one activation row and for
+// two: larger tiles amortize the per-tile work (barriers, reductions, the
+// scale and bias of every row) over more weights.  The temporal stream at one
+// row: 805 us at 4 (four 56 KB ring stages), 774 us at 5 (three of 70 KB),
+// 883 us at 3; at two rows 1346 us at 4, 1311 us at 5.  Six would overflow
+// the epilogue warp's reduction slots at K = 11264.  A chain keeps four: its
+// stages give each CTA a few tiles at most, where finer tiles balance better
+// (the 129-stage decode chain: 1.53 ms at 4, 1.66 ms at 5).
+#ifndef Q4_GEMV_RPT1
+#define Q4_GEMV_RPT1 5
 #endif
-constexpr int kRpt = Q4_GEMV_RPT;  // weight rows per team per tile (4-bit codes)
+#ifndef Q4_GEMV_RPT2
+#define Q4_GEMV_RPT2 5
+#endif
+constexpr int kRpt1 = Q4_GEMV_RPT1, kRpt2 = Q4_GEMV_RPT2, kRptChain = 4;
 // 8-bit codes (q8_matmul): a row is twice the bytes, so a team takes two
 // rows per tile and a tile stays near the 4-bit one's size.
 constexpr int kRpt8 = 2;
@@ -287,7 +298,7 @@ struct GemvLaunch {
 
 constexpr float kNaN = __builtin_nanf("");  // written by a thread whose bounded wait gave up
 constexpr int kRedSlots = 8;    // tiles of cross-warp partial sums in flight to the epilogue warp
-constexpr int kRedSlotFloats = 64 * 2;  // >= rt * MR * warps-per-team (<= 4 * 22 at MR = 1, 4 * 2 * 12 at MR = 2)
+constexpr int kRedSlotFloats = 64 * 2;  // >= rt * MR * warps-per-team (<= 110 at MR = 1, 120 at MR = 2)
 
 // Shape of one problem for a given consumer count (host and device agree).
 struct Geometry {
@@ -297,7 +308,10 @@ struct Geometry {
   int wpt;    // warps per team (0 when a warp holds several teams)
   int rt;     // rows per tile
 };
-__host__ __device__ inline Geometry geometry_of(int K, int consumer_threads, int bits = 4) {
+__host__ __device__ constexpr int rows_per_team(int bits, int mr, bool chain) {
+  return bits == 8 ? kRpt8 : chain ? kRptChain : (mr == 1 ? kRpt1 : kRpt2);
+}
+__host__ __device__ inline Geometry geometry_of(int K, int consumer_threads, int bits, int mr, bool chain = false) {
   Geometry g;
   g.G = K / 32;
   if (g.G >= 32) {
@@ -308,7 +322,7 @@ __host__ __device__ inline Geometry geometry_of(int K, int consumer_threads, int
   }
   g.teams = consumer_threads / g.team;
   g.wpt = g.team >= 32 ? g.team / 32 : 0;
-  g.rt = g.teams * (bits == 4 ? kRpt : kRpt8);
+  g.rt = g.teams * rows_per_team(bits, mr, chain);
   return g;
 }
 // Code bytes of a weight row, and its packed bytes (codes, scales, biases).
@@ -439,7 +453,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
   static_assert(!CHAIN || NP > kFewProblems, "chains use the large parameter block");
   static_assert(BITS == 4 || BITS == 8, "code width");
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int RPT = BITS == 4 ? kRpt : kRpt8;  // rows per team per tile
+  constexpr int RPT = rows_per_team(BITS, MR, CHAIN);  // rows per team per tile
   constexpr int CW = BITS == 4 ? 4 : 8;          // code words per lane per row (32 codes)
   constexpr int V = RPT * MR;
   constexpr int VP = pow2_at_least(V);
@@ -506,7 +520,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         for (int pi = pb; pi < pe && issued < L.stages; ++pi) {
           if (!segment_of<EPI, BITS>(L, pi, lo, hi, &r0, &r1)) break;
           const GemvProblem& P = L.prob[pi];
-          const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
+          const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS, MR, CHAIN);
           const int code_bytes = code_row_bytes(P.K, BITS);  // code bytes per row
           const int rtile = rtile_k<EPI>(P, geo);
           for (int64_t row0 = r0; row0 < r1 && issued < L.stages; row0 += rtile, ++issued) {
@@ -539,7 +553,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
         if (!segment_of<EPI, BITS>(L, pi, lo, hi, &r0, &r1)) break;
         if (r0 >= r1) continue;
         const GemvProblem& P = L.prob[pi];
-        const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
+        const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS, MR, CHAIN);
         const int code_bytes = code_row_bytes(P.K, BITS);  // code bytes per row
         const int rtile = rtile_k<EPI>(P, geo);
         for (int64_t row0 = r0; row0 < r1; row0 += rtile) {
@@ -611,7 +625,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
       int64_t r0, r1;
       if (!segment_of<EPI, BITS>(L, pi, lo, hi, &r0, &r1)) break;
       const GemvProblem& P = L.prob[pi];
-      const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
+      const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS, MR, CHAIN);
       if (!epilogue_warp_k<EPI>(P, geo)) continue;
       const int rtile = rtile_k<EPI>(P, geo);
       const bool fused = fused_k<EPI>(P);
@@ -665,7 +679,7 @@ __global__ void __launch_bounds__(MAXT, 1) gemv_kernel(const __grid_constant__ G
     if (!segment_of<EPI, BITS>(L, pi, lo, hi, &r_begin, &r_end)) break;
     if (r_begin >= r_end) continue;
     const GemvProblem& P = L.prob[pi];
-    const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS);
+    const Geometry geo = geometry_of(P.K, L.consumer_threads, BITS, MR, CHAIN);
     const int code_bytes = code_row_bytes(P.K, BITS);  // code bytes per row
     const int team_idx = tid / geo.team;
     const int j = tid - team_idx * geo.team;
@@ -962,7 +976,7 @@ bool tma_ok(const MatmulArgs& a, int mr, int bits = 4) {
   uintptr_t sb = reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases);
   if (a.fused()) sb |= reinterpret_cast<uintptr_t>(a.up_scales) | reinterpret_cast<uintptr_t>(a.up_biases);
   if (sb & 15u) return false;
-  const Geometry geo = geometry_of(static_cast<int>(a.K), consumers_for(mr), bits);
+  const Geometry geo = geometry_of(static_cast<int>(a.K), consumers_for(mr), bits, mr);
   // A fused tile pairs gate and up rows in the epilogue warp, which needs
   // teams of whole warps.
   if (a.fused() && geo.team < 32) return false;
@@ -994,8 +1008,9 @@ cudaError_t run_generic(const MatmulArgs& a, int64_t m0, const DeviceInfo& dev, 
 // Grows *stage_bytes to hold a tile of P; false if the epilogue warp's
 // reduction slots cannot take P's tiles (they are sized for kConsumers1 /
 // kConsumers2).
-bool ring_stage_fits(const GemvProblem& P, int mr, int consumers, uint32_t& stage_bytes, int bits = 4) {
-  const Geometry geo = geometry_of(P.K, consumers, bits);
+bool ring_stage_fits(const GemvProblem& P, int mr, int consumers, uint32_t& stage_bytes, int bits = 4,
+                     bool chain = false) {
+  const Geometry geo = geometry_of(P.K, consumers, bits, mr, chain);
   const uint32_t tile = static_cast<uint32_t>(geo.rt) * code_row_bytes(P.K, bits) +
                         2 * ((static_cast<uint32_t>(geo.rt) * geo.G * 2 + 15u) & ~15u);
   stage_bytes = std::max(stage_bytes, (tile + 127u) & ~127u);
@@ -1077,7 +1092,7 @@ cudaError_t run_chain(const GemvProblem* probs, int count, const int* stage_coun
     for (int k = 0; k < stage_counts[s]; ++k, ++i) {
       if (i >= count) return cudaErrorInvalidValue;
       const GemvProblem& P = probs[i];
-      if (!ring_stage_fits(P, MR, consumers, stage_bytes)) return cudaErrorInvalidConfiguration;
+      if (!ring_stage_fits(P, MR, consumers, stage_bytes, 4, true)) return cudaErrorInvalidConfiguration;
       L.prob[i] = P;
       L.prob[i].byte_begin = total;
       total += P.N * problem_row_bytes(P);
