@@ -218,3 +218,33 @@ def test_chain_three_rows_runs_stage_by_stage():
     assert launches == len(stages), launches
     for i, (a, b) in enumerate(zip(out_a, out_b)):
         assert torch.equal(a, b), i
+
+
+def test_chain_off_the_bulk_copy_path_and_empty_stages():
+    """A stage holding a problem the bulk-copy GEMV does not take (K = 96:
+    the generic kernel) makes the whole chain run one batch per stage; empty
+    stages (a zero count, or only empty problems) drop out.  Either way the
+    result equals the stage-by-stage batches."""
+    M = 1
+    w96 = _packed(64, 96, 170, 0)
+    w256 = _packed(96, 256, 170, 1)
+    x = workloads.activation(M, 256, 170, 2, device=DEV)
+
+    def build(h):
+        y1 = torch.full((M, 96), float("nan"), dtype=torch.bfloat16, device=DEV)
+        y2 = torch.full((M, 64), float("nan"), dtype=torch.bfloat16, device=DEV)
+        return [[(h, *w256, y1)], [], [(y1, *w96, y2)]], [y1, y2]
+
+    build.d = 256
+    h0 = x.clone()
+    st_a, out_a = build(h0.clone())
+    st_b, out_b = build(h0.clone())
+    n0 = q4.q4_debug_launch_count()
+    q4.q4_matmul_chain(st_a)
+    assert q4.q4_debug_launch_count() - n0 == 2  # one batch per non-empty stage
+    for st in st_b:
+        q4.q4_matmul_batch(st)
+    torch.cuda.synchronize()
+    for i, (a, b) in enumerate(zip(out_a, out_b)):
+        assert torch.equal(a, b), i
+

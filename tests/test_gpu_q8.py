@@ -127,3 +127,18 @@ def test_q8_batch_refuses_epilogues():
     arr = (q4.MatmulDesc * 1)(d)
     import ctypes
     assert q4.lib().q8_matmul_batch(ctypes.cast(arr, ctypes.c_void_p), 1, 1, 32, None) == 4  # Q4_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("M,K", [(1, 22528), (2, 12288), (2, 16384)])
+def test_q8_widest_rows(M, K):
+    """The widest rows a team of the bulk-copy GEMV holds (K = 22528 at one
+    activation row, 12288 at two) and one past it at two rows (K = 16384: the
+    warp-per-row kernel), against the oracle on sampled rows."""
+    N = 300
+    c, s, b = q4.q8_quantize(workloads.weight(N, K, 87, K + M, device=DEV))
+    x = workloads.activation(M, K, 87, M, device=DEV)
+    y = q4.q8_matmul(x, c, s, b)
+    rows = sample_rows(N, 48, seed=K)
+    y_ref, absdot = oracle.q8_matmul_ref(bits(x), c.cpu().numpy(), bits(s), bits(b), rows=rows)
+    ok = oracle.tolerance_ok(y.float().cpu().double().numpy()[:, rows], y_ref, absdot)
+    assert ok.all(), f"{int((~ok).sum())} elements outside the bound (M={M}, K={K})"
