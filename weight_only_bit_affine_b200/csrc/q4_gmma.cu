@@ -501,8 +501,10 @@ __global__ void __launch_bounds__(kThreads, 1) gmma_kernel(const __grid_constant
               if (!dead && !mbar_wait_backoff<kSleepEpi>(&d_full[slot], sph)) dead = true;
               tc_fence_after();
               const uint32_t dcol = lane_addr + static_cast<uint32_t>(slot) * kDCols;
-              // the groups' sums, as many groups per load as keep them in 16 registers
-              constexpr int kGL = MC <= 2 ? 4 : MC <= 4 ? 2 : 1;
+              // the groups' sums, several groups per load (one wait): 4 at 1..2
+              // rows, 2 at 4 and at 16 (16 rows: 1,643 -> 1,558 us on the decode
+              // step), 1 at 8 (2 measured slightly slower there)
+              constexpr int kGL = MC <= 2 ? 4 : MC == 8 ? 1 : 2;
 #pragma unroll
               for (int g0 = 0; g0 < kGroupsPerStep; g0 += kGL) {
                 uint32_t d[kGL][MC];
