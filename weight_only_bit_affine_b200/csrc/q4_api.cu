@@ -130,85 +130,107 @@ q4_status check_epilogue(const char* who, int32_t epi, int32_t reserved, const u
   return fail(Q4_ERR_UNSUPPORTED, "%s: unknown epilogue %d", who, static_cast<int>(epi));
 }
 
-// Enqueues a validated, non-empty list.  Each problem takes the kernel it
-// would take alone (so a batched result is bit-identical to the single
+// The launches of a validated, non-empty list.  Each problem takes the kernel
+// it would take alone (so a batched result is bit-identical to the single
 // call): the group-sum tensor-core kernel where it takes the problem (1..16
 // activation rows), else the weight-streaming kernel (3..8 rows), else the
 // tensor-core tiles (3 or more rows), else the CUDA-core GEMV.  Problems on
 // the group-sum kernel, the bulk-copy GEMV and the weight-streaming kernel
 // share launches per path; SwiGLU problems run in one pass on every path.
 // Every host-side step that can fail for a valid call (tensor-map encoding,
-// configuration checks) runs before the first launch.
-q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& dev, cudaStream_t cs,
-                       const char* what, bool static_scratch = false) {
-  std::vector<MatmulArgs> gemv, streamed, grouped;
-  thread_local std::vector<TcLaunch> tc;
-  thread_local std::vector<GmmaPlan> gm;
-  tc.clear();
-  gm.clear();
+// configuration checks) runs here, before the first launch.
+struct ListPlan {
+  std::vector<MatmulArgs> gemv, streamed;
+  std::vector<TcLaunch> tc;
+  std::vector<GmmaPlan> gm;
+  size_t counter_bytes = 0, partial_bytes = 0;  // the group-sum launches' workspace
+};
+
+q4_status plan_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& dev, const char* what,
+                        ListPlan& pl) {
+  std::vector<MatmulArgs> grouped;
   const unsigned int off = g_disabled_kernels.load(std::memory_order_relaxed);
   for (const MatmulArgs& a : list) {
     if (!(off & Q4_KERNEL_GROUP_SUM) && gmma_supported(a, dev)) {
       grouped.push_back(a);
     } else if (!(off & Q4_KERNEL_WEIGHT_STREAM) && stream_supported(a, dev)) {
-      streamed.push_back(a);
+      pl.streamed.push_back(a);
     } else if (!(off & Q4_KERNEL_TILES) && a.M >= kTensorCoreMinRows && tc_supported(a)) {
-      tc.emplace_back();
-      const cudaError_t e = plan_tc(a, dev, &tc.back());
+      pl.tc.emplace_back();
+      const cudaError_t e = plan_tc(a, dev, &pl.tc.back());
       if (e != cudaSuccess) return from_cuda(e, what);
     } else {
-      gemv.push_back(a);
+      pl.gemv.push_back(a);
     }
   }
   if (!grouped.empty()) {
-    const cudaError_t e = plan_gmma(grouped.data(), static_cast<int>(grouped.size()), dev, gm);
+    const cudaError_t e = plan_gmma(grouped.data(), static_cast<int>(grouped.size()), dev, pl.gm);
     if (e != cudaSuccess) return from_cuda(e, what);
   }
-  q4_status st = Q4_OK;
-  if (!gm.empty()) {
-    // One stream-ordered workspace for the launches that share tiles between
-    // CTAs: their arrival counters (zeroed here) and then their partial sums.
-    size_t cbytes = 0, pbytes = 0;
-    for (const GmmaPlan& g : gm) {
-      cbytes += g.counter_bytes;
-      pbytes += g.partial_bytes;
-    }
-    unsigned char* ws = nullptr;
-    if (cbytes + pbytes > 0 && static_scratch) {
-      if (cbytes + pbytes > kNoAllocScratchBytes)
-        return fail(Q4_ERR_UNSUPPORTED, "%s: the call needs %zu bytes of scratch, the fixed array holds %zu", what,
-                    cbytes + pbytes, kNoAllocScratchBytes);
-      cudaError_t e = noalloc_scratch(dev, &ws);
-      if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, cbytes, cs);
-      if (e != cudaSuccess) return from_cuda(e, what);
-    } else if (cbytes + pbytes > 0) {
-      cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), cbytes + pbytes, cs);
-      if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, cbytes, cs);
-      if (e != cudaSuccess) return from_cuda(e, what);
-    }
-    size_t co = 0, po = cbytes;
-    for (GmmaPlan& g : gm) {
-      unsigned int* counters = g.counter_bytes ? reinterpret_cast<unsigned int*>(ws + co) : nullptr;
-      float* partials = g.partial_bytes ? reinterpret_cast<float*>(ws + po) : nullptr;
-      co += g.counter_bytes;
-      po += g.partial_bytes;
-      if ((st = from_cuda(launch_planned_gmma(g, counters, partials, cs), what)) != Q4_OK) break;
-    }
-    if (ws != nullptr && !static_scratch) {
-      const cudaError_t e = cudaFreeAsync(ws, cs);
-      if (st == Q4_OK && e != cudaSuccess) st = from_cuda(e, what);
-    }
-    if (st != Q4_OK) return st;
+  for (const GmmaPlan& g : pl.gm) {
+    pl.counter_bytes += g.counter_bytes;
+    pl.partial_bytes += g.partial_bytes;
   }
-  for (const TcLaunch& t : tc)
+  return Q4_OK;
+}
+
+// Enqueues a plan's launches.  ws: the group-sum launches' workspace, its
+// arrival counters zero ([0, counter_region) holds the counters, the partial
+// sums start at counter_region); NULL when the plan needs none.  The launches
+// leave every counter zero again, so one workspace serves a sequence of plans.
+q4_status launch_plan(ListPlan& pl, const DeviceInfo& dev, cudaStream_t cs, const char* what, unsigned char* ws,
+                      size_t counter_region) {
+  q4_status st = Q4_OK;
+  size_t co = 0, po = counter_region;
+  for (GmmaPlan& g : pl.gm) {
+    unsigned int* counters = g.counter_bytes ? reinterpret_cast<unsigned int*>(ws + co) : nullptr;
+    float* partials = g.partial_bytes ? reinterpret_cast<float*>(ws + po) : nullptr;
+    co += g.counter_bytes;
+    po += g.partial_bytes;
+    if ((st = from_cuda(launch_planned_gmma(g, counters, partials, cs), what)) != Q4_OK) return st;
+  }
+  for (const TcLaunch& t : pl.tc)
     if ((st = from_cuda(launch_planned_tc(t, cs), what)) != Q4_OK) return st;
-  if (!streamed.empty() &&
-      (st = from_cuda(launch_stream_batch(streamed.data(), static_cast<int>(streamed.size()), cs, dev), what)) != Q4_OK)
+  if (!pl.streamed.empty() &&
+      (st = from_cuda(launch_stream_batch(pl.streamed.data(), static_cast<int>(pl.streamed.size()), cs, dev),
+                      what)) != Q4_OK)
     return st;
-  if (!gemv.empty() &&
-      (st = from_cuda(launch_gemv_batch(gemv.data(), static_cast<int>(gemv.size()), cs, dev), what)) != Q4_OK)
+  if (!pl.gemv.empty() &&
+      (st = from_cuda(launch_gemv_batch(pl.gemv.data(), static_cast<int>(pl.gemv.size()), cs, dev), what)) != Q4_OK)
     return st;
   return Q4_OK;
+}
+
+// Plans and enqueues a list with its own workspace: a stream-ordered
+// allocation (cudaMallocAsync, counters zeroed by cudaMemsetAsync, released
+// by cudaFreeAsync), or with static_scratch the fixed array of
+// q4_matmul_batch_noalloc.
+q4_status run_problems(const std::vector<MatmulArgs>& list, const DeviceInfo& dev, cudaStream_t cs,
+                       const char* what, bool static_scratch = false) {
+  thread_local ListPlan pl;
+  pl = ListPlan();
+  q4_status st = plan_problems(list, dev, what, pl);
+  if (st != Q4_OK) return st;
+  const size_t cbytes = pl.counter_bytes, pbytes = pl.partial_bytes;
+  unsigned char* ws = nullptr;
+  if (cbytes + pbytes > 0 && static_scratch) {
+    if (cbytes + pbytes > kNoAllocScratchBytes)
+      return fail(Q4_ERR_UNSUPPORTED, "%s: the call needs %zu bytes of scratch, the fixed array holds %zu", what,
+                  cbytes + pbytes, kNoAllocScratchBytes);
+    cudaError_t e = noalloc_scratch(dev, &ws);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, cbytes, cs);
+    if (e != cudaSuccess) return from_cuda(e, what);
+  } else if (cbytes + pbytes > 0) {
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), cbytes + pbytes, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, cbytes, cs);
+    if (e != cudaSuccess) return from_cuda(e, what);
+  }
+  st = launch_plan(pl, dev, cs, what, ws, cbytes);
+  if (ws != nullptr && !static_scratch) {
+    const cudaError_t e = cudaFreeAsync(ws, cs);
+    if (st == Q4_OK && e != cudaSuccess) st = from_cuda(e, what);
+  }
+  return st;
 }
 
 // One matmul with an epilogue (q4_matmul, q4_matmul_step, q4_matmul_residual,
@@ -396,12 +418,30 @@ q4_status q4_matmul_chain(const q4_matmul_desc* descs, int count, const int* sta
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int n = static_cast<int>(stages.size());
   if (!gemv_chain_supported(list.data(), static_cast<int>(list.size()))) {
-    // one batch launch (or set of launches) per stage, in order
+    // One batch launch (or set of launches) per stage, in order, every stage
+    // planned first; the stages' group-sum launches share one workspace
+    // (their counters return to zero after each launch), allocated and zeroed
+    // once for the call.
+    std::vector<ListPlan> plans(static_cast<size_t>(n));
+    size_t cmax = 0, pmax = 0;
     for (int s = 0, i = 0; s < n; i += stages[s], ++s) {
       std::vector<MatmulArgs> part(list.begin() + i, list.begin() + i + stages[s]);
-      if ((st = run_problems(part, *dev, cs, "q4_matmul_chain launch")) != Q4_OK) return st;
+      if ((st = plan_problems(part, *dev, "q4_matmul_chain launch", plans[s])) != Q4_OK) return st;
+      cmax = std::max(cmax, plans[s].counter_bytes);
+      pmax = std::max(pmax, plans[s].partial_bytes);
     }
-    return Q4_OK;
+    unsigned char* ws = nullptr;
+    if (cmax + pmax > 0) {
+      cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), cmax + pmax, cs);
+      if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, cmax, cs);
+      if (e != cudaSuccess) return from_cuda(e, "q4_matmul_chain workspace");
+    }
+    for (int s = 0; s < n && st == Q4_OK; ++s) st = launch_plan(plans[s], *dev, cs, "q4_matmul_chain launch", ws, cmax);
+    if (ws != nullptr) {
+      const cudaError_t e = cudaFreeAsync(ws, cs);
+      if (st == Q4_OK && e != cudaSuccess) st = from_cuda(e, "q4_matmul_chain workspace");
+    }
+    return st;
   }
   // Persistent launches, each over as many whole stages as its parameter
   // block holds, with one zeroed arrival counter per stage.
