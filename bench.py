@@ -366,6 +366,27 @@ def workload_rows(dev, packed, x, x_down, bf16_peak):
     prepared.run()
     one_launches = q4.q4_debug_launch_count() - n0
     ms_one = _graph_ms(dev, prepared.run, 20)
+    # The same chain for four conversations (M = 4): q4_matmul_chain runs one
+    # group-sum launch per stage there.
+    h4 = workloads.activation(4, 4096, 3, 74, device=dev)
+    qkv4 = [torch.empty((4, 4096), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    act4 = torch.empty((4, 11264), dtype=torch.bfloat16, device=dev)
+    logits4 = torch.empty((4, packed[-1][0].N), dtype=torch.bfloat16, device=dev)
+    stages4 = []
+    for P in layers_w:
+        stages4.append([(h4, *P["q"], qkv4[0]), (h4, *P["k"], qkv4[1]), (h4, *P["v"], qkv4[2])])
+        stages4.append([(qkv4[2], *P["o"], h4, q4.Residual(h4))])
+        stages4.append([(h4, *P["gate"], act4, q4.SwiGLU(*P["up"]))])
+        stages4.append([(act4, *P["down"], h4, q4.Residual(h4))])
+    stages4.append([(h4, *packed[-1][1:], logits4)])
+    prepared4 = q4.q4_prepare_chain(stages4)
+    ms_m4 = _graph_ms(dev, prepared4.run, 10)
+    rows["decode_chain_M4"] = {
+        "ms_per_step": round(ms_m4, 4), "GBps": round(STREAM_BYTES / (ms_m4 * 1e-3) / 1e9, 1),
+        "tokens_per_s": round(4 / (ms_m4 * 1e-3), 1), "stages": len(stages4), "path": GMMA_PATH,
+        "note": "the decode chain for four conversations: one q4_matmul_chain call, one group-sum launch per "
+                "stage (129, graph); compare stream_batch_M4 (the same projections as independent problems)",
+    }
     rows["decode_chain_M1"] = {
         "ms_per_step": round(ms_chain, 4), "GBps": round(STREAM_BYTES / (ms_chain * 1e-3) / 1e9, 1),
         "launches_per_step": int(chain_launches), "bytes": STREAM_BYTES,
@@ -703,11 +724,36 @@ def _q8_layer(dev):
         c, s, b = q4.q8_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
         items.append((xd if p.K == 11264 else x, c, s, b, torch.empty((1, p.N), dtype=torch.bfloat16, device=dev)))
 
-    def run():
-        for xx, c, s, b, y in items:
-            q4.q8_matmul(xx, c, s, b, out=y)
+    return lambda: q4.q8_matmul_batch(items)
 
-    return run
+
+def _chain_small(dev):
+    """The first three temporal layers and the head as a dependent chain (13
+    stages, one q4_matmul_chain call)."""
+    import torch
+
+    import workloads
+    import weight_only_bit_affine_b200 as q4
+
+    projs = workloads.stream_projs()
+    seed = workloads.seed_of("temporal_stream")
+    h = workloads.activation(1, 4096, seed, 10000, device=dev)
+    W = {}
+    for t, p in enumerate(projs):
+        if p.name.startswith(("L0.", "L1.", "L2.")) or t == len(projs) - 1:
+            W[p.name] = q4.q4_quantize(workloads.weight(p.N, p.K, seed, t, device=dev))
+    qkv = [torch.empty((1, 4096), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    act = torch.empty((1, 11264), dtype=torch.bfloat16, device=dev)
+    logits = torch.empty((1, projs[-1].N), dtype=torch.bfloat16, device=dev)
+    stages = []
+    for l in range(3):
+        P = {n: W[f"L{l}.{n}"] for n in ("q", "k", "v", "o", "gate", "up", "down")}
+        stages.append([(h, *P["q"], qkv[0]), (h, *P["k"], qkv[1]), (h, *P["v"], qkv[2])])
+        stages.append([(qkv[2], *P["o"], h, q4.Residual(h))])
+        stages.append([(h, *P["gate"], act, q4.SwiGLU(*P["up"]))])
+        stages.append([(act, *P["down"], h, q4.Residual(h))])
+    stages.append([(h, *W[projs[-1].name], logits)])
+    return q4.q4_prepare_chain(stages).run
 
 
 def _tc_gate(dev):
@@ -749,6 +795,7 @@ PROFILE_CASES = {"stream_small": _stream_small, "tc_layer": _tc_layer, "tc_gate"
                  "depformer_step": _depformer_step, "layer_m1": lambda dev: _layer_rows(dev, 1),
                  "layer_m4": lambda dev: _layer_rows(dev, 4),
                  "layer_m8": lambda dev: _layer_rows(dev, 8), "fused_layer": _fused_layer, "q8_layer": _q8_layer,
+                 "chain_small": _chain_small,
                  "layer_m4_weight_stream": _pinned(lambda dev: _layer_rows(dev, 4), 1)}
 
 
