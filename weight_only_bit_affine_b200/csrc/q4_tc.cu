@@ -25,10 +25,11 @@
 //   warp 1       allocates tensor memory; one thread issues the MMAs (A from
 //                tensor memory, B = the x tile in shared memory) and commits
 //                them to the barriers that free the A slot and the stage;
-//   warps 2..17  dequantize, in two groups of eight warps taking the atoms in
-//                turn: the thread of lane r and half h turns the 32 codes of
-//                group h of weight row r in an atom into 16 hi and 16 lo
-//                bf16 pairs and stores them to its tensor-memory lane
+//   warps 2..17  dequantize, in four groups of four warps (one per
+//                tensor-memory lane quarter) taking the atoms in turn, so
+//                four atoms are in flight: the thread of weight row r turns
+//                the row's 64 codes of an atom into 32 hi and 32 lo bf16
+//                pairs and stores them to its tensor-memory lane
 //                (tcgen05.st) in the atom's A slot, a ring of slots after
 //                the accumulators; then the epilogue (tensor memory ->
 //                registers -> bf16 y).
@@ -37,7 +38,8 @@
 // epilogue writes silu(gate) * up from the two fp32 results.
 // Split-K: when there are too few tiles to fill the GPU, the K range is split
 // across the CTAs of a thread-block cluster, and the fp32 partial tiles are
-// summed through distributed shared memory (no global workspace).
+// summed through distributed shared memory (no global workspace), laid out so
+// that every warp's remote load reads 512 contiguous bytes.
 // Every wait is bounded (q4_device.cuh); a thread whose wait gave up writes
 // NaN.  Programmatic dependent launch as in the GEMV family.
 #include "q4_device.cuh"
@@ -57,8 +59,8 @@ constexpr int kTileN = 128;                  // weight rows per tile (MMA M, ten
 constexpr int kAtomK = 64;                   // K per atom (one 128-byte swizzle span of bf16)
 constexpr int kSuperK = 256;                 // K per scale/bias load (8 groups = 16 bytes per row)
 constexpr int kAtomsPerSuper = kSuperK / kAtomK;
-constexpr int kDqGroups = 2;                 // dequantizing warp groups, taking atoms in turn
-constexpr int kDqWarpsPerGroup = 8;          // two per tensor-memory lane quarter (one per group of an atom)
+constexpr int kDqGroups = 4;                 // dequantizing warp groups, taking atoms in turn
+constexpr int kDqWarpsPerGroup = 4;          // one per tensor-memory lane quarter
 constexpr int kDqWarps = kDqGroups * kDqWarpsPerGroup;
 constexpr int kThreads = 64 + 32 * kDqWarps;  // 576
 constexpr uint32_t kTmemCols = 512;
@@ -220,29 +222,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- dequantize, then epilogue ----------------
     const int quarter = warp & 3;  // the tensor-memory lanes this warp may access
-    const int half = ((warp - 2) >> 2) & 1;
-    const int grp = (warp - 2) >> 3;
+    const int grp = (warp - 2) >> 2;
     const int row = 32 * quarter + lane;  // weight row within the tile
     const int64_t grow = n0 + row;
     const bool row_ok = grow < p.N;
     const int G = p.K / 32;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
-    // Scales and biases of this row, 8 groups (one super-chunk) per 16-byte
-    // load, fetched one super-chunk ahead; u counts super-chunks over both
-    // passes of a SwiGLU tile.
-    auto load_sb = [&](int u, uint4& sv, uint4& bv) {
-      sv = bv = make_uint4(0, 0, 0, 0);
+    // A group takes every kDqGroups-th atom: one per super-chunk (8 groups of
+    // 32), always the same atom of it, so it needs one 32-bit word (two bf16)
+    // of the row's scales and of its biases per super-chunk, fetched one
+    // super-chunk ahead; u counts super-chunks over both passes of a SwiGLU
+    // tile.
+    static_assert(kDqGroups == kAtomsPerSuper, "one atom per super-chunk per group");
+    auto load_sb = [&](int u, uint32_t& sv, uint32_t& bv) {
+      sv = bv = 0u;
       if (!row_ok || u >= pass_supers * p.nacc) return;
       const bool up = u >= pass_supers;
-      const int64_t off = grow * G + static_cast<int64_t>(sc_begin + u - (up ? pass_supers : 0)) * (kSuperK / 32);
-      sv = *reinterpret_cast<const uint4*>((up ? p.up_scales : p.scales) + off);
-      bv = *reinterpret_cast<const uint4*>((up ? p.up_biases : p.biases) + off);
+      const int64_t off =
+          grow * G + static_cast<int64_t>(sc_begin + u - (up ? pass_supers : 0)) * (kSuperK / 32) + 2 * grp;
+      sv = *reinterpret_cast<const uint32_t*>((up ? p.up_scales : p.scales) + off);
+      bv = *reinterpret_cast<const uint32_t*>((up ? p.up_biases : p.biases) + off);
     };
-    uint4 s_cur, b_cur, s_nxt, b_nxt;
+    uint32_t s_cur, b_cur, s_nxt, b_nxt;
     load_sb(0, s_cur, b_cur);
     load_sb(1, s_nxt, b_nxt);
     bool dead = false;
-    int cur_u = 0;
     // Stage and A slot of this group's atoms, advanced incrementally (atom a
     // sits in stage (a / ATOMS) mod stages and slot a mod a_slots).
     constexpr int kStageStep = kDqGroups / ATOMS;  // stages per group turn (ATOMS divides kDqGroups)
@@ -250,36 +254,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0, sph = 0;
     while (st >= p.stages) { st -= p.stages; ph ^= 1u; }
     while (slot >= p.a_slots) { slot -= p.a_slots; sph ^= 1u; }
-    for (int a = grp; a < natoms; a += kDqGroups) {
-      const int u = a / kAtomsPerSuper;
-      if (u != cur_u) {  // atoms advance by kDqGroups < kAtomsPerSuper: at most one super-chunk at a time
+    for (int a = grp, u = 0; a < natoms; a += kDqGroups, ++u) {
+      if (u > 0) {
         s_cur = s_nxt;
         b_cur = b_nxt;
         load_sb(u + 1, s_nxt, b_nxt);
-        cur_u = u;
       }
       if (!dead && !mbar_wait(&tma_full[st], ph)) dead = true;  // codes arrived
-      const uint4 cw =
-          *reinterpret_cast<const uint4*>(c_tile(st) + row * (32 * ATOMS) + (a % ATOMS) * 32 + half * 16);
-      const int gi = 2 * (a % kAtomsPerSuper) + half;  // group within the super-chunk
-      const uint32_t sw = (gi < 2) ? s_cur.x : (gi < 4) ? s_cur.y : (gi < 6) ? s_cur.z : s_cur.w;
-      const uint32_t bw = (gi < 2) ? b_cur.x : (gi < 4) ? b_cur.y : (gi < 6) ? b_cur.z : b_cur.w;
-      const uint64_t s2 = f32x2_splat(__uint_as_float((gi & 1) ? (sw & 0xFFFF0000u) : (sw << 16)));
-      const uint64_t b2 = f32x2_splat(__uint_as_float((gi & 1) ? (bw & 0xFFFF0000u) : (bw << 16)));
-      // All 32 codes into registers first (separate arrays: a tcgen05.st reads
+      const uint4* cp = reinterpret_cast<const uint4*>(c_tile(st) + row * (32 * ATOMS) + (a % ATOMS) * 32);
+      const uint4 cw0 = cp[0], cw1 = cp[1];  // the atom's two groups of 32 codes of this row
+      const uint32_t sw = s_cur, bw = b_cur;
+      const uint64_t s20 = f32x2_splat(__uint_as_float(sw << 16)), b20 = f32x2_splat(__uint_as_float(bw << 16));
+      const uint64_t s21 = f32x2_splat(__uint_as_float(sw & 0xFFFF0000u));
+      const uint64_t b21 = f32x2_splat(__uint_as_float(bw & 0xFFFF0000u));
+      // All 64 codes into registers first (separate arrays: a tcgen05.st reads
       // its source registers after it issues, so none is overwritten early).
-      uint32_t hi0[8], lo0[8], hi1[8], lo1[8];
-      dequant_word_hilo(cw.x, s2, b2, hi0, lo0);
-      dequant_word_hilo(cw.y, s2, b2, hi0 + 4, lo0 + 4);
-      dequant_word_hilo(cw.z, s2, b2, hi1, lo1);
-      dequant_word_hilo(cw.w, s2, b2, hi1 + 4, lo1 + 4);
+      uint32_t hi0[16], lo0[16], hi1[16], lo1[16];
+      dequant_word_hilo(cw0.x, s20, b20, hi0, lo0);
+      dequant_word_hilo(cw0.y, s20, b20, hi0 + 4, lo0 + 4);
+      dequant_word_hilo(cw0.z, s20, b20, hi0 + 8, lo0 + 8);
+      dequant_word_hilo(cw0.w, s20, b20, hi0 + 12, lo0 + 12);
+      dequant_word_hilo(cw1.x, s21, b21, hi1, lo1);
+      dequant_word_hilo(cw1.y, s21, b21, hi1 + 4, lo1 + 4);
+      dequant_word_hilo(cw1.z, s21, b21, hi1 + 8, lo1 + 8);
+      dequant_word_hilo(cw1.w, s21, b21, hi1 + 12, lo1 + 12);
       if (!dead && !mbar_wait(&a_empty[slot], sph ^ 1u)) dead = true;  // the MMAs of the slot's last atom are done
       tc_fence_after();
-      const uint32_t taddr = lane_addr + p.a_col0 + static_cast<uint32_t>(slot) * kASlotCols + 16u * half;
-      tmem_st_x8(taddr, hi0);
-      tmem_st_x8(taddr + 8u, hi1);
-      tmem_st_x8(taddr + 32u, lo0);
-      tmem_st_x8(taddr + 40u, lo1);
+      const uint32_t taddr = lane_addr + p.a_col0 + static_cast<uint32_t>(slot) * kASlotCols;
+      tmem_st_x16(taddr, hi0);
+      tmem_st_x16(taddr + 16u, hi1);
+      tmem_st_x16(taddr + 32u, lo0);
+      tmem_st_x16(taddr + 48u, lo1);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -294,8 +299,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!dead && !mbar_wait(accum_full, 0)) dead = true;
     tc_fence_after();
     const int part = (warp - 2) >> 2;  // 0..3: which column octets this warp reads
-    float* red = reinterpret_cast<float*>(smem);  // reuses the stage area (all MMAs are done)
-    const int red_ld = p.nacc * p.bn + 4;          // 16-byte rows; row r and r + 1 four banks apart
+    // Partial tile for the cluster's sum, in the stage area (all MMAs are
+    // done): four columns per 16-byte unit, the 128 rows of a unit
+    // consecutive (unit c4 of row r at c4 * 128 + r), so a warp's store and a
+    // peer warp's load each cover 512 contiguous bytes.
+    float4* red = reinterpret_cast<float4*>(smem);
     for (int c0 = 8 * part; c0 < p.bn; c0 += 32) {
       uint32_t gr[8], ur[8];
       tmem_ld_cols<8>(lane_addr + c0, gr);
@@ -314,13 +322,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row_ok && m < p.M) p.y[m * p.N + grow] = out_tc<EPI>(g[i], u[i], p, m * p.N + grow);
         }
       } else {
-        float4* dst = reinterpret_cast<float4*>(red + row * red_ld + c0);
-        dst[0] = make_float4(g[0], g[1], g[2], g[3]);
-        dst[1] = make_float4(g[4], g[5], g[6], g[7]);
+        red[(c0 / 4) * kTileN + row] = make_float4(g[0], g[1], g[2], g[3]);
+        red[(c0 / 4 + 1) * kTileN + row] = make_float4(g[4], g[5], g[6], g[7]);
         if (p.nacc == 2) {
-          float4* du = reinterpret_cast<float4*>(red + row * red_ld + p.bn + c0);
-          du[0] = make_float4(u[0], u[1], u[2], u[3]);
-          du[1] = make_float4(u[4], u[5], u[6], u[7]);
+          red[((p.bn + c0) / 4) * kTileN + row] = make_float4(u[0], u[1], u[2], u[3]);
+          red[((p.bn + c0) / 4 + 1) * kTileN + row] = make_float4(u[4], u[5], u[6], u[7]);
         }
       }
     }
@@ -334,10 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = tid - 64;
       const int trow = t & (kTileN - 1);
       const int64_t grow = n0 + trow;
-      const int red_ld = p.nacc * p.bn + 4;
       // Column slice of this CTA, in float4 units (bn and the slice are multiples of 4).
       const int q_beg = split * (p.bn / 4) / p.splits, q_end = (split + 1) * (p.bn / 4) / p.splits;
-      const uint32_t row_addr = smem_u32(smem) + static_cast<uint32_t>(trow * red_ld) * 4u;
+      const uint32_t row_addr = smem_u32(smem) + static_cast<uint32_t>(trow) * 16u;
       uint32_t peer[8];
 #pragma unroll
       for (int r = 0; r < 8; ++r) peer[r] = dsmem_map(row_addr, static_cast<uint32_t>(r < p.splits ? r : 0));
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int r = 0; r < 8; ++r)  // all peers' loads first, then the sums
             if (r < p.splits)
-              v[r] = ld_dsmem_v4(peer[r] + static_cast<uint32_t>(w * p.bn) * 4u + static_cast<uint32_t>(q) * 16u);
+              v[r] = ld_dsmem_v4(peer[r] + static_cast<uint32_t>((w * (p.bn / 4) + q) * kTileN) * 16u);
           float4 t = v[0];
 #pragma unroll
           for (int r = 1; r < 8; ++r)
@@ -501,7 +506,7 @@ cudaError_t plan_tc(const MatmulArgs& a, const DeviceInfo& dev, TcLaunch* out) {
   p.splits = splits;
   p.b_atom_bytes = b_atom;
   p.stage_bytes = stage_size(atoms);
-  const size_t red_bytes = static_cast<size_t>(kTileN) * (nacc * bn + 4) * 4;
+  const size_t red_bytes = static_cast<size_t>(kTileN) * nacc * bn * 4;  // the partial tile of the split-K sum
   p.stages = static_cast<int>(std::min<size_t>(kMaxStages, avail / p.stage_bytes));
   while (p.stages < kMaxStages && static_cast<size_t>(p.stages) * p.stage_bytes < red_bytes) ++p.stages;
   if (p.stages < 2 || static_cast<size_t>(p.stages) * p.stage_bytes < red_bytes ||
