@@ -114,6 +114,32 @@ def test_swiglu_matches_oracle(M, N, K):
     _assert_within(h, ref, bound, rows, f"swiglu M={M} {N}x{K}")
 
 
+# The tile kernel's widest epilogue tiles, split over a cluster of up to
+# eight CTAs: SwiGLU with 128 activation rows a tile (its two accumulators
+# fill tensor memory) and with a second, ragged row tile; the residual with
+# 256 rows a tile and with a second, ragged row tile.
+@pytest.mark.parametrize("M", [128, 200])
+@pytest.mark.parametrize("N,K", [(300, 1024), (1024, 4096)])
+def test_swiglu_wide_tiles(M, N, K):
+    gate = _packed(N, K, 65, N + K)
+    up = _packed(N, K, 65, 7 * N + K)
+    x = workloads.activation(M, K, 65, 3000 + M, device=DEV)
+    h = q4.q4_matmul_swiglu(x, gate, up)
+    ref, bound = oracle.matmul_swiglu_ref(bits(x), packed_to_host(*gate), packed_to_host(*up))
+    _assert_within(h, ref, bound, None, f"swiglu M={M} {N}x{K}")
+
+
+@pytest.mark.parametrize("M", [256, 300])
+@pytest.mark.parametrize("N,K", [(300, 1024), (1024, 11264)])
+def test_residual_wide_tiles(M, N, K):
+    c, s, b = _packed(N, K, 66, N + K)
+    x = workloads.activation(M, K, 66, 1000 + M, device=DEV)
+    r = workloads.activation(M, N, 66, 2000 + M, device=DEV)
+    y = q4.q4_matmul_residual(x, c, s, b, r)
+    ref, bound = oracle.matmul_residual_ref(bits(x), *packed_to_host(c, s, b), bits(r))
+    _assert_within(y, ref, bound, None, f"residual M={M} {N}x{K}")
+
+
 @pytest.mark.parametrize("M", [1, 2, 4, 8, 16, 64])
 def test_swiglu_one_pass_is_one_launch(M):
     gate, up = _packed(2816, 1024, 64, 0), _packed(2816, 1024, 64, 1)
