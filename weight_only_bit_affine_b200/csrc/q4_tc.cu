@@ -444,16 +444,18 @@ cudaError_t plan_tc(const MatmulArgs& a, const DeviceInfo& dev, TcLaunch* out) {
   const int64_t m_tiles = (a.M + bn - 1) / bn;
   const int supers = static_cast<int>(a.K / kSuperK);
   // Split K over a cluster of up to 8 CTAs when the tiles alone would leave
-  // SMs idle: the split minimising waves x (super-chunks per CTA + 1), the
-  // "+ 1" standing for a CTA's fixed cost (pipeline fill, epilogue, the
-  // cluster's reduction).  One CTA per SM, so a wave is sm_count CTAs.
+  // SMs idle: the split minimising waves x (super-chunks per CTA + 4), the
+  // "+ 4" standing for a CTA's fixed cost, measured at about four
+  // super-chunks of main loop (the pipeline's fill, its drain and the
+  // epilogue); ties go to the smaller split, which also saves the
+  // cluster's sum.  One CTA per SM, so a wave is sm_count CTAs.
   int splits = 1;
   const int64_t tiles = n_tiles * m_tiles;
   {
     int64_t best = -1;
     for (int sp = 1; sp <= 8 && sp <= supers; ++sp) {
       const int64_t waves = (tiles * sp + dev.sm_count - 1) / dev.sm_count;
-      const int64_t cost = waves * ((supers + sp - 1) / sp + 1);
+      const int64_t cost = waves * ((supers + sp - 1) / sp + 4);
       if (best < 0 || cost < best) { best = cost; splits = sp; }
     }
   }
